@@ -1,0 +1,334 @@
+"""Benchmark of the sparse-MLA decode step on B200: indexer -> top-k -> sparse MLA.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload batched_decode]
+
+One step = one layer's sparse attention over one batch: the default workload is
+32 requests x 1 query token, contexts uniform in [8,192, 65,536], 16 MLA heads,
+64 indexer heads of dim 128, top-2048, 64-token pages over a permuted shared
+pool (one TP8 rank of batched decode).  Inputs are seeded synthetic data.
+
+Timing: W untimed warm-up steps; then K steps, each preceded by a 256 MiB write
+that flushes L2, each timed on its stream with CUDA events around the three
+stage calls (events between them give per-kernel times); a barrier and a device
+synchronize bracket the timed region; the max over ranks is taken.  Under
+torchrun each rank runs its own batch on its own GPU (independent requests:
+weak scaling, no data-path collective).
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the float64 CPU
+oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_mla_attention_indexer_b200 import sml, synth  # noqa: E402
+from sparse_mla_attention_indexer_b200.device import DeviceWorkload  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+FLUSH_BYTES = 256 << 20
+# dram__bytes_read.sum + dram__bytes_write.sum of one indexer launch on this
+# workload, from the ncu capture summarised in profiles/ (None = not captured
+# for the current kernel).
+INDEXER_NCU_TRAFFIC_BYTES = None
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_units(wl):
+    """Algorithmic bytes of the indexer scan and gathered tokens of the attention."""
+    from_ctx = 0
+    n_sum = 0
+    cu = wl.cu_q
+    for r in range(wl.B):
+        Q = int(cu[r + 1] - cu[r])
+        L = int(wl.ctx_len[r])
+        from_ctx += L                      # every visible cache token read once per request
+        n_sum += sum(L - Q + j + 1 for j in range(Q))
+    idx_bytes = from_ctx * 132 + n_sum * 4 + wl.T * (64 * 128 + 4 + 64 * 4)
+    gathered = sum(min(wl.topk, n) for n in _visible(wl))
+    rope = wl.layers[0].rope_dim
+    mla_bytes = gathered * (656 if rope else 528)
+    mla_flops = gathered * 2 * wl.num_heads * ((512 + rope) + 512)
+    return dict(indexer_bytes=idx_bytes, gathered=gathered, mla_bytes=mla_bytes, mla_flops=mla_flops,
+                topk_bytes=n_sum * 4)
+
+
+def _visible(wl):
+    out = []
+    for r in range(wl.B):
+        Q = int(wl.cu_q[r + 1] - wl.cu_q[r])
+        L = int(wl.ctx_len[r])
+        out += [L - Q + j + 1 for j in range(Q)]
+    return out
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.file.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = np.array([float(r[1]) for r in rows if r[1].replace(".", "").isdigit()])
+        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if len(sm) else None, "sm_max_mhz": mx,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def time_ours(args, wl, rank):
+    dw = DeviceWorkload(wl)
+    p = dw.problem(0)
+    lay = dw.layers[0]
+    ws = dw.workspace(sml.SML_STAGE_LAYER)
+    idx, ln, out, lse = dw.outputs()
+    scores = dw.scores()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        sml.sml_indexer_scores(p, lay.iq8, lay.iq_scale, lay.iw, dw.index_cache, scores, ws, stream)
+        ev[1].record(stream)
+        sml.sml_topk(p, scores, idx, ln, ws, stream)
+        ev[2].record(stream)
+        sml.sml_sparse_mla_decode(p, lay.q, dw.latent, idx, ln, out, lse, ws, stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        step()
+        ev[3].record(stream)
+    torch.cuda.synchronize()
+    code, bits = sml.sml_read_device_status(ws)
+    if code != sml.SML_OK:
+        raise RuntimeError(f"device status {code} bits {bits:#x}")
+
+    events = []
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        for _ in range(args.steps):
+            flush.fill_(1)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            ev[0].record(stream)
+            step()
+            ev[3].record(stream)
+            events.append(ev)
+        torch.cuda.synchronize()
+        barrier()
+    per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]),
+                     e[0].elapsed_time(e[3])] for e in events])
+    code, bits = sml.sml_read_device_status(ws)
+    if code != sml.SML_OK:
+        raise RuntimeError(f"device status {code} bits {bits:#x}")
+
+    # End to end through the one-call entry point from pinned host buffers:
+    # per step, copy the step's inputs (queries, indexer queries, batch
+    # metadata) host -> device, run the layer, read the outputs back.
+    h_in = [t.cpu().pin_memory() for t in (lay.q, lay.iq8, lay.iq_scale, lay.iw, dw.cu_q, dw.ctx_len,
+                                            dw.block_table)]
+    d_in = [lay.q, lay.iq8, lay.iq_scale, lay.iw, dw.cu_q, dw.ctx_len, dw.block_table]
+    h_out = [torch.empty_like(t, device="cpu").pin_memory() for t in (out, lse, idx, ln)]
+    d_out = [out, lse, idx, ln]
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for d, h in zip(d_in, h_in):
+            d.copy_(h, non_blocking=True)
+        sml.sml_run_layer(p, lay.q, lay.iq8, lay.iq_scale, lay.iw, dw.latent, dw.index_cache, None, None,
+                          idx, ln, out, lse, ws, stream)
+        for d, h in zip(d_out, h_out):
+            h.copy_(d, non_blocking=True)
+        e1.record(stream)
+        stream.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(e0.elapsed_time(e1))
+    return per, clocks.summary(), float(np.mean(e2e_ms)), h2d, d2h
+
+
+def barrier():
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float) -> float:
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+    return x
+
+
+def cpu_baseline(wl, budget_s: float = 15.0):
+    """The float64 oracle on a bounded sample: whole query tokens of the workload,
+    taken in order until about budget_s seconds of CPU work."""
+    from oracle import mla as omla
+    v = wl.view(0)
+    t0 = time.perf_counter()
+    done = 0
+    while done < wl.T and time.perf_counter() - t0 < budget_s:
+        omla.run_layer(v, wl.latent, wl.index_cache, tokens=[done])
+        done += 1
+    dt = time.perf_counter() - t0
+    return dict(value=done / dt, unit="queries/s", cores=os.cpu_count(), kind="oracle",
+                sample=f"{done} of {wl.T} query tokens of {wl.name} (one full layer each: "
+                       f"indexer over the whole context, top-k, sparse MLA) in {dt:.1f} s")
+
+
+def config_of(wl, args, n_gpus):
+    return {"workload": wl.name, "requests": wl.B, "query_tokens": wl.T, "mla_heads": wl.num_heads,
+            "indexer_heads": 64, "indexer_dim": 128, "topk": wl.topk, "page_tokens": 64,
+            "ctx_tokens_total": int(wl.ctx_len.sum()), "ctx_min": int(wl.ctx_len.min()),
+            "ctx_max": int(wl.ctx_len.max()), "ssmax": bool(wl.ssmax),
+            "rope_dim": wl.layers[0].rope_dim, "latent_cache": "fp8_ds_mla (656 B/token)",
+            "l2": "flushed by a 256 MiB write before every step", "parallelism": f"replicas x{n_gpus}"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="batched_decode", choices=sorted(synth.SUITE))
+    args = ap.parse_args()
+    world, rank, local = dist_env()
+    metric = "sparse-MLA decode queries/s (indexer + top-2048 + sparse MLA, one layer)"
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        wl = synth.SUITE[args.workload](seed=0)
+        vals = []
+        for _ in range(args.warmup + args.steps):
+            cb = cpu_baseline(wl, budget_s=max(1.0, 60.0 / (args.warmup + args.steps)))
+            vals.append(cb["value"])
+        v = float(np.mean(vals[args.warmup:]))
+        cb["value"] = v
+        print(json.dumps({"impl": "reference", "metric": metric, "value": v, "unit": "queries/s",
+                          "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                          "dtype": "f64", "data": "synthetic", "config": config_of(wl, args, 1),
+                          "cpu_baseline": cb,
+                          "e2e": {"value": v, "unit": "queries/s", "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}))
+        return
+
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    wl = synth.SUITE[args.workload](seed=0)
+    units = workload_units(wl)
+    per, clocks, e2e_ms, h2d, d2h = time_ours(args, wl, rank)
+    ms_step = max_over_ranks(float(per[:, 3].mean()))
+    ms_idx = max_over_ranks(float(per[:, 0].mean()))
+    ms_topk = max_over_ranks(float(per[:, 1].mean()))
+    ms_mla = max_over_ranks(float(per[:, 2].mean()))
+    e2e_ms = max_over_ranks(e2e_ms)
+    peak, peak_kind = peaks()
+    cb = cpu_baseline(wl) if rank == 0 and world == 1 else None
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    qps = world * wl.T / (ms_step / 1e3)
+    idx_gbs = units["indexer_bytes"] / (ms_idx / 1e3) / 1e9
+    line = {
+        "metric": metric, "value": qps, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3/f16 products, f32 accumulate", "data": "synthetic",
+        "config": config_of(wl, args, world),
+        "gathered_tokens_per_s": world * units["gathered"] / (ms_step / 1e3),
+        "stage_ms": {"indexer": ms_idx, "topk": ms_topk, "sparse_mla_and_merge": ms_mla},
+        "indexer_hbm_gbs": idx_gbs, "indexer_frac_of_8000_gbs": idx_gbs / 8000.0,
+        "mla_hbm_gbs": units["mla_bytes"] / (ms_mla / 1e3) / 1e9,
+        "mla_tflops": units["mla_flops"] / (ms_mla / 1e3) / 1e12,
+        "roofline": {"kernel": "indexer scores", "bound": "hbm", "achieved": idx_gbs, "peak": peak,
+                     "unit": "GB/s", "frac": idx_gbs / peak, "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": units["indexer_bytes"],
+                     "traffic": INDEXER_NCU_TRAFFIC_BYTES},
+        "clocks": clocks,
+        "e2e": {"value": world * wl.T / (e2e_ms / 1e3), "unit": "queries/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "entry_point": "sml_run_layer"},
+        "gpu_launches": args.steps * 4,
+        "cpu_baseline": cb,
+    }
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

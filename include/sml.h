@@ -1,0 +1,204 @@
+/*
+ * sml.h -- C ABI of libsml.so, the sparse-MLA decode step of a DeepSeek-style
+ * sparse attention layer (Mistral Large 4 as served by vLLM) on one NVIDIA
+ * B200 (sm_100a):
+ *
+ *   sml_indexer_scores     DSA indexer: FP8 q.k per indexer head, ReLU,
+ *                          head-weighted sum, over a paged FP8 indexer cache
+ *   sml_topk               exact per-query top-k over those scores
+ *   sml_sparse_mla_decode  absorbed-query MLA over only the selected tokens of
+ *                          a paged fp8_ds_mla latent cache (split over the
+ *                          selected keys, then a log-sum-exp merge)
+ *   sml_run_layer          the three in a row, or only the attention for a
+ *                          shared-indexer layer that reuses a prior top-k
+ *
+ * Sources: vLLM blog "vLLM 首日支持 Mistral Large 4：1T 参数 MoE 多模态模型",
+ * highlights list (MLA with KV LoRA rank 512 and RoPE dim 64; a DSA indexer
+ * picks the top 2048 keys per query; default fp8_ds_mla latent cache) and
+ * section "实现细节 / 模型架构" (sparse MLA over the fp8_ds_mla latent cache plus
+ * an indexer over an FP8 indexer cache; shared-indexer layers reuse the top-k
+ * of the preceding indexer layer; the indexer has its own SSMax; NoPE layers
+ * are MLA with RoPE dim 0 over the same kernels and cache layout; 47,136 B of
+ * KV per token).  The pages print no formula, layout or API; where they are
+ * silent this header states the reading it implements.
+ *
+ * Conventions for every entry point
+ *   - All array pointers are DEVICE pointers on the current CUDA device unless
+ *     a comment says "host".  The caller owns every buffer; the library
+ *     allocates nothing and frees nothing.
+ *   - Work is enqueued on `stream` (a cudaStream_t, NULL = legacy default
+ *     stream) and returns without waiting.  Only sml_read_device_status
+ *     synchronises (that stream).
+ *   - Return value: SML_OK, or a negative SML_ERR_* code.  On an error nothing
+ *     has been enqueued, and sml_last_error() (per host thread) lists every
+ *     check that failed, not only the first.
+ *   - Checks that need device data (context lengths, block-table entries,
+ *     selected indices) run inside the kernels: a bad value sets a bit in a
+ *     sticky status word in the workspace and the access is skipped (masked);
+ *     kernels never trap.  Read it with sml_read_device_status.
+ *   - Supported shapes (anything else returns SML_ERR_UNSUPPORTED): page size
+ *     64 tokens; num_heads in {16, 32, 64, 128}; 1 <= topk <= 2048;
+ *     rope_dim in {0, 64}; 64 indexer heads of dim 128.
+ *
+ * Notation: B requests; T query tokens in total; request r owns query tokens
+ * [cu_q[r], cu_q[r+1]) (Q_r = cu_q[r+1] - cu_q[r] >= 1) and L_r = ctx_len[r]
+ * cached tokens, its own query tokens included (L_r >= Q_r).  Query j (0-based)
+ * of request r sees positions [0, n_t) with n_t = L_r - Q_r + j + 1 (causal
+ * within the request).  Logical position s of request r lives in physical
+ * page block_table[r * max_pages + s / 64], row s % 64.
+ */
+#ifndef SML_H_
+#define SML_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes --------------------------------------------------------- */
+#define SML_OK 0
+#define SML_ERR_INVALID_ARG (-1)  /* a NULL pointer, negative size, inconsistent sizes */
+#define SML_ERR_UNSUPPORTED (-2)  /* a shape or option outside the supported set */
+#define SML_ERR_WORKSPACE (-3)    /* workspace NULL, misaligned or smaller than sml_workspace_size */
+#define SML_ERR_CUDA (-4)         /* a CUDA runtime call failed (launch, attribute) */
+#define SML_ERR_DEVICE_FAULT (-5) /* returned by sml_read_device_status: a device check failed */
+#define SML_ERR_TIMEOUT (-6)      /* returned by sml_read_device_status: a bounded wait gave up */
+
+/* Bits of the device status word (see sml_read_device_status). */
+#define SML_FAULT_PAGE 0x1        /* a block-table entry outside [0, num_pages) */
+#define SML_FAULT_INDEX 0x2       /* a selected position outside [0, n_t) */
+#define SML_FAULT_LENGTHS 0x4     /* cu_q / ctx_len inconsistent with the problem */
+#define SML_FAULT_TOPK_LEN 0x8    /* a top-k length outside [0, min(topk, n_t)] */
+#define SML_FAULT_TIMEOUT 0x10    /* an mbarrier or flag wait exceeded its poll limit */
+
+/* ---- fixed sizes (readings of the pages' byte counts) --------------------- */
+#define SML_PAGE_TOKENS 64
+#define SML_LATENT_DIM 512          /* KV LoRA rank */
+#define SML_ROPE_DIM 64
+/* fp8_ds_mla row, 656 B: [512 x e4m3 latent][4 x fp32 scale, one per 128
+ * elements][64 x bf16 RoPE key]; a page is 64 rows back to back. */
+#define SML_LATENT_ROW_BYTES 656
+#define SML_LATENT_PAGE_BYTES (SML_PAGE_TOKENS * SML_LATENT_ROW_BYTES)
+/* indexer page: [64 x 128 B e4m3 keys][64 x fp32 per-token scale], 132 B/token */
+#define SML_INDEX_HEADS 64
+#define SML_INDEX_DIM 128
+#define SML_INDEX_PAGE_BYTES (SML_PAGE_TOKENS * (SML_INDEX_DIM + 4))
+#define SML_MAX_TOPK 2048
+
+/* Workspace stages for sml_workspace_size. */
+#define SML_STAGE_INDEXER 1
+#define SML_STAGE_TOPK 2
+#define SML_STAGE_MLA 3
+#define SML_STAGE_LAYER 4
+
+/* One batch of query tokens.  Host struct; the pointers in it are device
+ * pointers.  Every entry point validates it. */
+typedef struct sml_problem {
+  int32_t num_requests;        /* B >= 1 */
+  int32_t num_tokens;          /* T = cu_q[B] >= 1 */
+  int32_t num_heads;           /* H, MLA query heads: 16, 32, 64 or 128 */
+  int32_t topk;                /* K, 1..2048 */
+  int32_t rope_dim;            /* 64 (RoPE layer) or 0 (NoPE layer) */
+  int32_t max_pages;           /* row stride of block_table, >= ceil(L_r / 64) */
+  int32_t max_ctx;             /* >= every L_r; row stride of the score matrix */
+  int32_t ssmax;               /* 0 = off; 1 = scale logits by s * ln(n_t) */
+  float sm_scale;              /* softmax scale sigma of the MLA logits */
+  float ssmax_s;               /* SSMax s of the MLA logits */
+  float ssmax_s_index;         /* SSMax s of the indexer scores */
+  const int32_t* cu_q;         /* [B + 1], cu_q[0] = 0, non-decreasing */
+  const int32_t* ctx_len;      /* [B], L_r */
+  const int32_t* block_table;  /* [B * max_pages], physical page ids */
+} sml_problem;
+
+/* A paged cache pool: num_pages pages starting at base (256-B aligned). */
+typedef struct sml_cache {
+  const void* base;
+  int64_t num_pages;
+} sml_cache;
+
+/* Bytes of workspace the given stage needs for this problem (0 on invalid
+ * arguments; see sml_last_error).  SML_STAGE_LAYER covers sml_run_layer,
+ * including the score matrix it keeps internally.  A workspace must be
+ * 256-B aligned and initialised once with sml_workspace_init; after that it may
+ * be reused by any later call whose size fits, on the same stream. */
+size_t sml_workspace_size(const sml_problem* p, int stage);
+
+/* Zero the workspace header (device status word and the per-row arrival
+ * counters of the two-level top-k).  Call once after allocating a workspace. */
+int sml_workspace_init(void* workspace, size_t ws_bytes, void* stream);
+
+/* DSA indexer scores.
+ *   I[t, s] = c_t * sq_t * sk_s * sum_h w[t, h] * ReLU(sum_d e4m3(q8[t,h,d]) * e4m3(k8[s,d]))
+ * for s < n_t, with c_t = ssmax_s_index * ln(n_t) when ssmax, else 1.
+ * (Reading: the pages name the indexer "FP8 q.k per indexer head, ReLU and a
+ * head-weighted sum" only; head weights are per query token and head, and
+ * both FP8 scales are positive so they commute with the ReLU.)
+ *   iq8       [T, 64, 128] e4m3 codes of the indexer query
+ *   iq_scale  [T] fp32 per-token query scale sq_t (> 0)
+ *   iw        [T, 64] fp32 head weights
+ *   index_cache  pool of SML_INDEX_PAGE_BYTES pages
+ *   scores    [T, max_ctx] fp32 out; entries s >= n_t are not written
+ * FP8 products are exact; sums accumulate in fp32. */
+int sml_indexer_scores(const sml_problem* p, const void* iq8, const float* iq_scale, const float* iw,
+                       sml_cache index_cache, float* scores, void* workspace, size_t ws_bytes,
+                       void* stream);
+
+/* Exact top-k per query token over scores[t, 0:n_t) (blog section "ROCm
+ * 实现细节", persistent decode paragraph: the selection is an exact
+ * top-2048).  Order: larger score first; -0.0 == +0.0; a NaN ranks below every
+ * number; equal scores go to the lower position.
+ *   scores   [T, max_ctx] fp32 (row stride max_ctx), read for s < n_t only
+ *   idx      [T, topk] int32 out: the selected positions in ASCENDING order,
+ *            then -1 padding
+ *   idx_len  [T] int32 out: min(topk, n_t) */
+int sml_topk(const sml_problem* p, const float* scores, int32_t* idx, int32_t* idx_len,
+             void* workspace, size_t ws_bytes, void* stream);
+
+/* Absorbed-query sparse MLA over the selected positions.  For token t, head h,
+ * selected set S_t = idx[t, 0:idx_len[t]):
+ *   z_i = sm_scale * c_t * (q[t,h,0:512] . c_hat_i + q[t,h,512:576] . k_pe_i)
+ *   out[t,h,:] = sum_i softmax(z)_i * c_hat_i,  lse[t,h] = ln sum_i exp(z_i)
+ * with c_hat_i = e4m3 latent * its block scale, c_t = ssmax_s * ln(n_t) when
+ * ssmax, else 1.  rope_dim = 0 (NoPE) drops the k_pe term.
+ *   q        [T, H, 512 + rope_dim] bf16
+ *   latent   pool of SML_LATENT_PAGE_BYTES pages
+ *   idx      [T, topk] int32 logical positions (any order; -1 padding ignored)
+ *   idx_len  [T] int32 number of valid entries at the front of each idx row
+ *   out      [T, H, 512] fp32;  lse [T, H] fp32 (natural log; -inf if empty)
+ * Products run on tensor cores in fp16 (dequantised latent, probabilities)
+ * with fp32 accumulation; softmax in fp32. */
+int sml_sparse_mla_decode(const sml_problem* p, const void* q, sml_cache latent,
+                          const int32_t* idx, const int32_t* idx_len, float* out, float* lse,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/* One layer.  If reuse_idx is NULL: indexer scores (kept in the workspace),
+ * top-k into idx_out / len_out, then sparse MLA over them.  If reuse_idx is not
+ * NULL (a shared-indexer layer): sparse MLA over reuse_idx / reuse_len only;
+ * iq8, iq_scale, iw, index_cache, idx_out and len_out may then be NULL. */
+int sml_run_layer(const sml_problem* p, const void* q, const void* iq8, const float* iq_scale,
+                  const float* iw, sml_cache latent, sml_cache index_cache,
+                  const int32_t* reuse_idx, const int32_t* reuse_len, int32_t* idx_out,
+                  int32_t* len_out, float* out, float* lse, void* workspace, size_t ws_bytes,
+                  void* stream);
+
+/* Synchronise `stream`, then return SML_OK, SML_ERR_DEVICE_FAULT or
+ * SML_ERR_TIMEOUT from the workspace's sticky status word (its SML_FAULT_*
+ * bits go to *bits when bits is a host pointer, else ignored).  clear != 0
+ * resets the word. */
+int sml_read_device_status(void* workspace, int clear, int32_t* bits, void* stream);
+
+/* Static text of a status code. */
+const char* sml_status_string(int code);
+
+/* Message of the last failed call on this host thread ("" if none). */
+const char* sml_last_error(void);
+
+/* Library version, e.g. "sml 0.1.0 sm_100a". */
+const char* sml_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SML_H_ */

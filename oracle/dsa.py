@@ -58,10 +58,14 @@ def ssmax_factor(enabled: bool, s: float, n: int) -> float:
     return s * math.log(n) if enabled else 1.0
 
 
-def indexer_scores_row(q8_t, q_scale_t, w_t, index_cache, bt_row, n, c_t, positions=None):
+def indexer_scores_row(q8_t, q_scale_t, w_t, index_cache, bt_row, n, c_t, positions=None,
+                       with_magnitude=False):
     """Scores of one query token against positions (default: all of 0..n-1).
 
     q8_t: [64, 128] uint8 e4m3 codes; q_scale_t: scalar; w_t: [64] head weights.
+    With ``with_magnitude`` also returns the size of the summed terms,
+    c_t * sum_h |w_h| * ReLU(q_h . k_s), against which a rounding error in the
+    weighted sum is measured.
     """
     if positions is None:
         positions = np.arange(n)
@@ -69,14 +73,17 @@ def indexer_scores_row(q8_t, q_scale_t, w_t, index_cache, bt_row, n, c_t, positi
     q = F.decode_e4m3(q8_t) * float(q_scale_t)                     # [64, 128]
     w = np.asarray(w_t, dtype=np.float64)                          # [64]
     out = np.empty(len(positions), dtype=np.float64)
+    mag = np.empty(len(positions), dtype=np.float64)
     chunk = 1 << 15
     for a in range(0, len(positions), chunk):
         pos = positions[a:a + chunk]
         pages, rows = F.physical(bt_row, pos)
         k = F.indexer_keys(index_cache, pages, rows)                # [m, 128]
-        dots = q @ k.T                                              # [64, m]
-        out[a:a + chunk] = c_t * (w[:, None] * np.maximum(dots, 0.0)).sum(axis=0)
-    return out
+        relu = np.maximum(q @ k.T, 0.0)                             # [64, m]
+        out[a:a + chunk] = c_t * (w[:, None] * relu).sum(axis=0)
+        if with_magnitude:
+            mag[a:a + chunk] = abs(c_t) * (np.abs(w)[:, None] * relu).sum(axis=0)
+    return (out, mag) if with_magnitude else out
 
 
 def indexer_scores(wl, q8, q_scale, w, index_cache, tokens=None):

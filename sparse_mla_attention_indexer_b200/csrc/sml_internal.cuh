@@ -1,0 +1,95 @@
+// Internal declarations shared by the libsml.so translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sml.h"
+
+namespace sml {
+
+// ---- workspace -----------------------------------------------------------------
+// Every stage's workspace starts with a 256-B header whose first word is the
+// sticky device status (SML_FAULT_* bits), then the per-row arrival counters of
+// the two-level top-k.  Regions are 256-B aligned.
+struct WsHeader {
+  int32_t status;
+  int32_t pad[63];
+};
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Top-k: one CTA selects over a chunk of up to kTopkChunk positions held in
+// shared memory; longer rows are cut into chunks whose candidates the last
+// arriving CTA of the row merges.
+constexpr int kTopkChunk = 32768;
+constexpr int kTopkThreads = 1024;
+
+struct TopkWs {
+  int32_t* counters;   // [T] arrival counters, zero between calls
+  uint32_t* cand_key;  // [T, chunks, K]
+  int32_t* cand_idx;   // [T, chunks, K]
+  int chunks;          // ceil(max_ctx / kTopkChunk)
+};
+
+struct MlaWs {
+  float* part_out;     // [T, H, S, 512]
+  float* part_lse;     // [T, H, S]
+  int splits;          // S
+  int keys_per_split;  // multiple of 64
+};
+
+// Region sizes, in bytes (host).
+size_t topk_region_bytes(const sml_problem& p);
+size_t mla_region_bytes(const sml_problem& p);
+int mla_splits(const sml_problem& p, int* keys_per_split);
+
+// ---- device helpers ---------------------------------------------------------------
+__device__ __forceinline__ void raise_fault(int32_t* status, int bits) {
+  if (status) atomicOr(status, bits);
+}
+
+// Request owning query token t (cu_q non-decreasing, cu_q[0] = 0).
+__device__ __forceinline__ int request_of(const int32_t* __restrict__ cu_q, int B, int t) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu_q + mid) <= t) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Query range, context length and visible length of request r, checked against
+// the problem: 0 <= q0, Q >= 1, q0 + Q <= T, Q <= L <= max_ctx and
+// ceil(L / 64) <= max_pages.  Anything else is SML_FAULT_LENGTHS and the
+// request is skipped, so no index derived from it leaves its buffer.
+struct Req {
+  int q0, Q, L;
+  bool ok;
+};
+
+__device__ __forceinline__ Req load_request(const int32_t* __restrict__ cu_q,
+                                            const int32_t* __restrict__ ctx_len, int r, int T,
+                                            int max_ctx, int max_pages) {
+  Req q;
+  q.q0 = __ldg(cu_q + r);
+  q.Q = __ldg(cu_q + r + 1) - q.q0;
+  q.L = __ldg(ctx_len + r);
+  q.ok = q.q0 >= 0 && q.Q >= 1 && q.q0 <= T - q.Q && q.L >= q.Q && q.L <= max_ctx &&
+         (q.L + SML_PAGE_TOKENS - 1) / SML_PAGE_TOKENS <= max_pages;
+  return q;
+}
+
+// ---- launchers (one per kernel family; all enqueue on `stream`) --------------------
+cudaError_t launch_indexer(const sml_problem& p, const uint8_t* iq8, const float* iq_scale,
+                           const float* iw, const uint8_t* index_base, int64_t index_pages,
+                           float* scores, int32_t* status, cudaStream_t stream);
+cudaError_t launch_topk(const sml_problem& p, const float* scores, int32_t* idx, int32_t* idx_len,
+                        const TopkWs& ws, int32_t* status, cudaStream_t stream);
+cudaError_t launch_sparse_mla(const sml_problem& p, const uint16_t* q, const uint8_t* latent_base,
+                              int64_t latent_pages, const int32_t* idx, const int32_t* idx_len,
+                              float* out, float* lse, const MlaWs& ws, int32_t* status,
+                              cudaStream_t stream);
+
+}  // namespace sml

@@ -1,0 +1,210 @@
+"""ctypes binding of libsml.so (declared in ``include/sml.h``).
+
+Argument marshalling only: every entry point takes torch tensors (device
+memory) or plain ints, passes their addresses and sizes to the C ABI and raises
+``SmlError`` on a non-zero status.  Every step of the computation runs in the
+library's CUDA kernels; if ``libsml.so`` is missing the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsml.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "sml.h")
+
+SML_OK = 0
+SML_ERR_INVALID_ARG = -1
+SML_ERR_UNSUPPORTED = -2
+SML_ERR_WORKSPACE = -3
+SML_ERR_CUDA = -4
+SML_ERR_DEVICE_FAULT = -5
+SML_ERR_TIMEOUT = -6
+
+SML_FAULT_PAGE = 0x1
+SML_FAULT_INDEX = 0x2
+SML_FAULT_LENGTHS = 0x4
+SML_FAULT_TOPK_LEN = 0x8
+SML_FAULT_TIMEOUT = 0x10
+
+SML_STAGE_INDEXER = 1
+SML_STAGE_TOPK = 2
+SML_STAGE_MLA = 3
+SML_STAGE_LAYER = 4
+
+PAGE_TOKENS = 64
+LATENT_PAGE_BYTES = 64 * 656
+INDEX_PAGE_BYTES = 64 * 132
+
+
+class SmlError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"[{code}] {msg}")
+        self.code = code
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [
+        ("num_requests", ctypes.c_int32),
+        ("num_tokens", ctypes.c_int32),
+        ("num_heads", ctypes.c_int32),
+        ("topk", ctypes.c_int32),
+        ("rope_dim", ctypes.c_int32),
+        ("max_pages", ctypes.c_int32),
+        ("max_ctx", ctypes.c_int32),
+        ("ssmax", ctypes.c_int32),
+        ("sm_scale", ctypes.c_float),
+        ("ssmax_s", ctypes.c_float),
+        ("ssmax_s_index", ctypes.c_float),
+        ("cu_q", ctypes.c_void_p),
+        ("ctx_len", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p),
+    ]
+
+
+class Cache(ctypes.Structure):
+    _fields_ = [("base", ctypes.c_void_p), ("num_pages", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libsml.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libsml.so is not built ({LIB_PATH}); run "
+                               "`python -m sparse_mla_attention_indexer_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        pp = ctypes.POINTER(Problem)
+        L.sml_workspace_size.argtypes = [pp, i32]
+        L.sml_workspace_size.restype = sz
+        L.sml_workspace_init.argtypes = [vp, sz, vp]
+        L.sml_indexer_scores.argtypes = [pp, vp, vp, vp, Cache, vp, vp, sz, vp]
+        L.sml_topk.argtypes = [pp, vp, vp, vp, vp, sz, vp]
+        L.sml_sparse_mla_decode.argtypes = [pp, vp, Cache, vp, vp, vp, vp, vp, sz, vp]
+        L.sml_run_layer.argtypes = [pp, vp, vp, vp, vp, Cache, Cache, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sml_read_device_status.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_int32), vp]
+        L.sml_status_string.argtypes = [i32]
+        for name in ("sml_status_string", "sml_last_error", "sml_version"):
+            getattr(L, name).restype = ctypes.c_char_p
+        for name in ("sml_workspace_init", "sml_indexer_scores", "sml_topk", "sml_sparse_mla_decode",
+                     "sml_run_layer", "sml_read_device_status"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def declared_entry_points(header: str = HEADER):
+    """Names of the functions declared in include/sml.h."""
+    text = open(header, encoding="utf-8").read()
+    return sorted(set(re.findall(r"^[A-Za-z_][\w \*]*?\b(sml_\w+)\s*\(", text, flags=re.M)))
+
+
+def _p(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _s(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(code: int):
+    if code != SML_OK:
+        raise SmlError(code, lib().sml_last_error().decode())
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+def make_problem(*, num_heads, topk, rope_dim, cu_q, ctx_len, block_table, max_ctx=None,
+                 ssmax=False, sm_scale, ssmax_s=0.4, ssmax_s_index=0.4, num_tokens=None) -> Problem:
+    """Problem struct for device tensors cu_q [B+1], ctx_len [B], block_table [B, max_pages] (int32)."""
+    B = ctx_len.numel()
+    return Problem(num_requests=B,
+                   num_tokens=int(num_tokens) if num_tokens is not None else int(cu_q[-1]),
+                   num_heads=num_heads, topk=topk, rope_dim=rope_dim,
+                   max_pages=block_table.shape[1],
+                   max_ctx=int(max_ctx) if max_ctx is not None else int(ctx_len.max()),
+                   ssmax=int(bool(ssmax)), sm_scale=sm_scale, ssmax_s=ssmax_s,
+                   ssmax_s_index=ssmax_s_index, cu_q=_p(cu_q), ctx_len=_p(ctx_len),
+                   block_table=_p(block_table))
+
+
+def cache(pool, page_bytes: int) -> Cache:
+    """Cache descriptor of a uint8 pool tensor (or None for an absent cache)."""
+    if pool is None:
+        return Cache(None, 0)
+    return Cache(_p(pool), _nbytes(pool) // page_bytes)
+
+
+def sml_workspace_size(problem: Problem, stage: int) -> int:
+    n = lib().sml_workspace_size(ctypes.byref(problem), stage)
+    if n == 0:
+        raise SmlError(SML_ERR_INVALID_ARG, lib().sml_last_error().decode())
+    return n
+
+
+def sml_workspace_init(workspace, stream=None):
+    _check(lib().sml_workspace_init(_p(workspace), _nbytes(workspace), _s(stream)))
+
+
+def sml_indexer_scores(problem, iq8, iq_scale, iw, index_cache, scores, workspace, stream=None):
+    _check(lib().sml_indexer_scores(ctypes.byref(problem), _p(iq8), _p(iq_scale), _p(iw),
+                                    cache(index_cache, INDEX_PAGE_BYTES), _p(scores), _p(workspace),
+                                    _nbytes(workspace), _s(stream)))
+
+
+def sml_topk(problem, scores, idx, idx_len, workspace, stream=None):
+    _check(lib().sml_topk(ctypes.byref(problem), _p(scores), _p(idx), _p(idx_len), _p(workspace),
+                          _nbytes(workspace), _s(stream)))
+
+
+def sml_sparse_mla_decode(problem, q, latent, idx, idx_len, out, lse, workspace, stream=None):
+    _check(lib().sml_sparse_mla_decode(ctypes.byref(problem), _p(q), cache(latent, LATENT_PAGE_BYTES),
+                                       _p(idx), _p(idx_len), _p(out), _p(lse), _p(workspace),
+                                       _nbytes(workspace), _s(stream)))
+
+
+def sml_run_layer(problem, q, iq8, iq_scale, iw, latent, index_cache, reuse_idx, reuse_len,
+                  idx_out, len_out, out, lse, workspace, stream=None):
+    _check(lib().sml_run_layer(ctypes.byref(problem), _p(q), _p(iq8), _p(iq_scale), _p(iw),
+                               cache(latent, LATENT_PAGE_BYTES), cache(index_cache, INDEX_PAGE_BYTES),
+                               _p(reuse_idx), _p(reuse_len), _p(idx_out), _p(len_out), _p(out),
+                               _p(lse), _p(workspace), _nbytes(workspace), _s(stream)))
+
+
+def sml_read_device_status(workspace, clear: bool = True, stream=None):
+    """(status code, SML_FAULT_* bits); synchronises the stream."""
+    bits = ctypes.c_int32(0)
+    code = lib().sml_read_device_status(_p(workspace), int(clear), ctypes.byref(bits), _s(stream))
+    if code in (SML_ERR_INVALID_ARG, SML_ERR_WORKSPACE, SML_ERR_CUDA):
+        _check(code)
+    return code, bits.value
+
+
+def sml_status_string(code: int) -> str:
+    return lib().sml_status_string(code).decode()
+
+
+def sml_last_error() -> str:
+    return lib().sml_last_error().decode()
+
+
+def sml_version() -> str:
+    return lib().sml_version().decode()

@@ -1,0 +1,75 @@
+"""The C ABI on the host: the library builds for sm_100a, loads, exports every
+entry point declared in include/sml.h, and rejects bad arguments before any
+CUDA call (so these run without a GPU)."""
+import ctypes
+
+import pytest
+
+from sparse_mla_attention_indexer_b200 import build as sml_build
+from sparse_mla_attention_indexer_b200 import sml
+
+
+@pytest.fixture(scope="module")
+def L():
+    sml_build.build()
+    return sml.lib()
+
+
+def test_every_declared_entry_point_is_exported(L):
+    names = sml.declared_entry_points()
+    assert {"sml_indexer_scores", "sml_topk", "sml_sparse_mla_decode", "sml_run_layer"} <= set(names)
+    for name in names:
+        assert hasattr(L, name), name
+    assert sml.sml_version().startswith("sml ")
+
+
+def _problem(**kw):
+    base = dict(num_requests=2, num_tokens=3, num_heads=16, topk=2048, rope_dim=64, max_pages=4,
+                max_ctx=256, ssmax=0, sm_scale=0.04, ssmax_s=0.4, ssmax_s_index=0.4,
+                cu_q=0x1000, ctx_len=0x2000, block_table=0x3000)
+    base.update(kw)
+    return sml.Problem(**base)
+
+
+def test_workspace_size_grows_with_stage_and_is_aligned(L):
+    p = _problem()
+    sizes = {s: sml.sml_workspace_size(p, s) for s in (1, 2, 3, 4)}
+    assert all(v % 256 == 0 and v > 0 for v in sizes.values())
+    assert sizes[4] >= sizes[2] and sizes[4] >= sizes[3]
+    # the layer keeps its own score matrix: T * max_ctx floats
+    assert sizes[4] >= 3 * 256 * 4
+
+
+def test_invalid_problem_lists_every_reason(L):
+    p = _problem(num_heads=24, topk=4096, rope_dim=32, sm_scale=float("nan"), cu_q=0)
+    assert L.sml_workspace_size(ctypes.byref(p), 4) == 0
+    msg = sml.sml_last_error()
+    for part in ("num_heads", "topk", "rope_dim", "sm_scale", "cu_q is NULL"):
+        assert part in msg, msg
+
+
+def test_entry_points_reject_null_and_misaligned_without_cuda(L):
+    p = _problem()
+    ws_small = 256
+    code = L.sml_indexer_scores(ctypes.byref(p), None, None, None, sml.Cache(None, 0), None,
+                                0x100, ws_small, None)
+    assert code == sml.SML_ERR_INVALID_ARG
+    msg = sml.sml_last_error()
+    assert "iq8" in msg and "index_cache.base" in msg and "scores" in msg
+    code = L.sml_topk(ctypes.byref(p), 0x1000, 0x2000, 0x3000, 0x100, 8, None)
+    assert code == sml.SML_ERR_WORKSPACE and "needs" in sml.sml_last_error()
+    code = L.sml_sparse_mla_decode(ctypes.byref(p), 0x1001, sml.Cache(0x1000, 4), 0x10, 0x10,
+                                   0x1000, 0x1000, 0x100, 1 << 30, None)
+    assert code == sml.SML_ERR_INVALID_ARG and "q NULL or not 16-B aligned" in sml.sml_last_error()
+    code = L.sml_run_layer(ctypes.byref(p), 0x1000, None, None, None, sml.Cache(0x1000, 4),
+                           sml.Cache(None, 0), 0x1000, None, None, None, 0x1000, 0x1000, 0x100,
+                           1 << 30, None)
+    assert code == sml.SML_ERR_INVALID_ARG and "reuse_len" in sml.sml_last_error()
+
+
+def test_unsupported_only_when_nothing_is_invalid(L):
+    p = _problem(num_heads=8)
+    assert L.sml_workspace_size(ctypes.byref(p), 1) == 0
+    code = L.sml_topk(ctypes.byref(p), 0x1000, 0x2000, 0x3000, 0x100, 1 << 30, None)
+    assert code == sml.SML_ERR_UNSUPPORTED
+    assert sml.sml_status_string(code) == "unsupported shape or option"
