@@ -132,9 +132,10 @@ int sml_workspace_init(void* workspace, size_t ws_bytes, void* stream);
 /* DSA indexer scores.
  *   I[t, s] = c_t * sq_t * sk_s * sum_h w[t, h] * ReLU(sum_d e4m3(q8[t,h,d]) * e4m3(k8[s,d]))
  * for s < n_t, with c_t = ssmax_s_index * ln(n_t) when ssmax, else 1.
- * (Reading: the pages name the indexer "FP8 q.k per indexer head, ReLU and a
- * head-weighted sum" only; head weights are per query token and head, and
- * both FP8 scales are positive so they commute with the ReLU.)
+ * (Reading: the pages print no formula for the indexer; this is the
+ * DeepSeek-style indexer -- an FP8 dot product per indexer head, a ReLU and a
+ * weighted sum over heads -- with head weights per query token and head; both
+ * FP8 scales are positive, so they commute with the ReLU.)
  *   iq8       [T, 64, 128] e4m3 codes of the indexer query
  *   iq_scale  [T] fp32 per-token query scale sq_t (> 0)
  *   iw        [T, 64] fp32 head weights
@@ -182,6 +183,30 @@ int sml_run_layer(const sml_problem* p, const void* q, const void* iq8, const fl
                   const int32_t* reuse_idx, const int32_t* reuse_len, int32_t* idx_out,
                   int32_t* len_out, float* out, float* lse, void* workspace, size_t ws_bytes,
                   void* stream);
+
+/* Sparse MLA decode for callers that cannot allocate device memory: same
+ * arguments, checks and results as sml_sparse_mla_decode, but no workspace.
+ * (The pages have no counterpart; this is an interface convenience.)
+ * Some callers cannot pass a workspace: a serving engine that has handed all
+ * spare HBM to its KV-cache pool at start-up, a host runtime that forbids
+ * cudaMalloc on its hot path because it synchronises the device, or a plugin
+ * with no handle on its host's allocator.  This entry point keeps its split
+ * partials in a scratch array built into libsml.so instead: 16 MiB held on
+ * every GPU that loads the library, until the process exits.  It allocates and
+ * frees nothing.
+ *   - A problem whose partials (T x H x splits x 2,052 B) exceed 16 MiB returns
+ *     SML_ERR_UNSUPPORTED; use sml_sparse_mla_decode for it.
+ *   - The first call on a device looks up the scratch array's device address
+ *     (once per device); make that first call before any stream capture.
+ *   - Every call on a device shares the one scratch array and it keeps the last
+ *     call's contents (nothing in it needs to start at zero).  Calls that can
+ *     overlap on the GPU (different streams, or several host threads) race on
+ *     it: serialise them.
+ *   - There is no workspace, so there is no device status word: out-of-range
+ *     pages or positions are still masked, but not reported. */
+int sml_sparse_mla_decode_noalloc(const sml_problem* p, const void* q, sml_cache latent,
+                                  const int32_t* idx, const int32_t* idx_len, float* out, float* lse,
+                                  void* stream);
 
 /* Synchronise `stream`, then return SML_OK, SML_ERR_DEVICE_FAULT or
  * SML_ERR_TIMEOUT from the workspace's sticky status word (its SML_FAULT_*

@@ -16,6 +16,8 @@ namespace sml {
 
 static thread_local std::string g_last_error;
 
+void set_last_error(const std::string& msg) { g_last_error = msg; }
+
 namespace {
 
 struct Checker {

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <string>
+
 #include "sml.h"
 
 namespace sml {
@@ -39,6 +41,9 @@ struct MlaWs {
   int splits;          // S
   int keys_per_split;  // multiple of 64
 };
+
+// Message returned by sml_last_error() on this host thread.
+void set_last_error(const std::string& msg);
 
 // Region sizes, in bytes (host).
 size_t topk_region_bytes(const sml_problem& p);

@@ -89,13 +89,14 @@ def lib() -> ctypes.CDLL:
         L.sml_indexer_scores.argtypes = [pp, vp, vp, vp, Cache, vp, vp, sz, vp]
         L.sml_topk.argtypes = [pp, vp, vp, vp, vp, sz, vp]
         L.sml_sparse_mla_decode.argtypes = [pp, vp, Cache, vp, vp, vp, vp, vp, sz, vp]
+        L.sml_sparse_mla_decode_noalloc.argtypes = [pp, vp, Cache, vp, vp, vp, vp, vp]
         L.sml_run_layer.argtypes = [pp, vp, vp, vp, vp, Cache, Cache, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sml_read_device_status.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_int32), vp]
         L.sml_status_string.argtypes = [i32]
         for name in ("sml_status_string", "sml_last_error", "sml_version"):
             getattr(L, name).restype = ctypes.c_char_p
         for name in ("sml_workspace_init", "sml_indexer_scores", "sml_topk", "sml_sparse_mla_decode",
-                     "sml_run_layer", "sml_read_device_status"):
+                     "sml_sparse_mla_decode_noalloc", "sml_run_layer", "sml_read_device_status"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -179,6 +180,13 @@ def sml_sparse_mla_decode(problem, q, latent, idx, idx_len, out, lse, workspace,
     _check(lib().sml_sparse_mla_decode(ctypes.byref(problem), _p(q), cache(latent, LATENT_PAGE_BYTES),
                                        _p(idx), _p(idx_len), _p(out), _p(lse), _p(workspace),
                                        _nbytes(workspace), _s(stream)))
+
+
+def sml_sparse_mla_decode_noalloc(problem, q, latent, idx, idx_len, out, lse, stream=None):
+    """Sparse MLA decode without a workspace (scratch built into the library)."""
+    _check(lib().sml_sparse_mla_decode_noalloc(ctypes.byref(problem), _p(q),
+                                               cache(latent, LATENT_PAGE_BYTES), _p(idx),
+                                               _p(idx_len), _p(out), _p(lse), _s(stream)))
 
 
 def sml_run_layer(problem, q, iq8, iq_scale, iw, latent, index_cache, reuse_idx, reuse_len,
