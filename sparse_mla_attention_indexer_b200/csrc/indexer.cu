@@ -1,4 +1,4 @@
-// DSA indexer scores over a paged FP8 indexer cache.
+// DSA indexer scores over a paged FP8 indexer cache, on the sm_100a tensor cores.
 //
 // vLLM blog "vLLM 首日支持 Mistral Large 4", section "实现细节 / 模型架构":
 // the sparse indexer reads an FP8 indexer cache and has its own SSMax; section
@@ -6,110 +6,364 @@
 // token t against cached token s < n_t:
 //   I[t, s] = c_t * sq_t * sk_s * sum_h w[t, h] * ReLU(q8[t, h, :] . k8[s, :])
 //
-// One CTA scores one 64-token page of one request for up to kQChunk of its
-// query tokens.  FP8 codes are widened exactly to fp32; each product of two
-// E4M3 values is exact in fp32 and the sums accumulate in fp32.
-#include <cuda_fp8.h>
+// Design (one persistent CTA per SM, warp-specialised):
+//   * a work item is (request, query group of <= 4 tokens, 128-token tile);
+//     items are enumerated on the device from cu_q / ctx_len and split evenly
+//     over the CTAs, so the host never reads device data;
+//   * warp 0 moves the tile's two 64-token key pages into shared memory with
+//     3-D TMA loads (128-B swizzle) over the paged pool, and the pages'
+//     per-token scales with plain bulk copies, into a 6-stage ring;
+//   * warp 1 issues tcgen05.mma kind::f8f6f4: D[128 tokens, 64 x Qg] =
+//     K[128, 128] . Q[64 x Qg, 128]^T, E4M3 x E4M3 with fp32 accumulation in
+//     TMEM (two 256-column accumulators, so MMA and epilogue overlap);
+//   * warps 2-5 (one thread per token row) read D from TMEM, apply ReLU, the
+//     head weights and sq * sk * c_t, and store the scores of visible positions.
+// Every wait is bounded; a wait that gives up sets SML_FAULT_TIMEOUT and the
+// CTA winds down (no trap).
+#include <cudaTypedefs.h>
+#include <math.h>
 
+#include "ptx.cuh"
 #include "sml_internal.cuh"
 
 namespace sml {
 namespace {
 
-constexpr int kQChunk = 16;
-constexpr int kThreads = 256;
-constexpr int kPad = 129;  // row pitch in floats: conflict-free column reads
+constexpr int kTile = 128;       // tokens per tile = MMA M
+constexpr int kStages = 6;
+constexpr int kGroup = 4;        // query tokens per group: N = 64 * Qg <= 256
+constexpr int kAccCols = 256;
+constexpr int kThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kPageKeyBytes = SML_PAGE_TOKENS * SML_INDEX_DIM;   // 8,192
+constexpr int kQRowsBytes = SML_INDEX_HEADS * SML_INDEX_DIM;      // 8,192 per query token
 
-__device__ __forceinline__ void e4m3x16_to_f32(uint4 v, float* dst) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] & 0xffffu), __NV_E4M3);
-    const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] >> 16), __NV_E4M3);
-    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
-    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
-    dst[4 * i + 0] = a.x;
-    dst[4 * i + 1] = a.y;
-    dst[4 * i + 2] = b.x;
-    dst[4 * i + 3] = b.y;
-  }
-}
+struct __align__(1024) Smem {
+  uint8_t keys[kStages][2 * kPageKeyBytes];      // [stage][128 rows x 128 B], SW128
+  uint8_t q[2][kGroup * kQRowsBytes];            // [buffer][256 rows x 128 B], SW128
+  float ksc[kStages][kTile];
+  float w[kGroup * SML_INDEX_HEADS];             // epilogue: head weights of the group
+  float qf[kGroup];                              // epilogue: sq_t * c_t per query
+  uint64_t full[kStages], empty[kStages];
+  uint64_t qfull[2], qempty[2];
+  uint64_t accfull[2], accempty[2];
+  uint64_t drain;
+  int valid[kStages];                            // bit p: page p of the tile was loaded
+  uint32_t tmem_base;
+  int abort;
+  int range[2];
+};
 
-__global__ void __launch_bounds__(kThreads)
-indexer_page_kernel(int B, int T, int max_pages, int max_ctx, int ssmax, float s_index,
-                    const int32_t* __restrict__ cu_q, const int32_t* __restrict__ ctx_len,
-                    const int32_t* __restrict__ block_table, const uint8_t* __restrict__ iq8,
-                    const float* __restrict__ iq_scale, const float* __restrict__ iw,
-                    const uint8_t* __restrict__ index_base, int64_t index_pages,
-                    float* __restrict__ scores, int32_t* status) {
-  extern __shared__ float dsm[];
-  float (*ks)[kPad] = reinterpret_cast<float (*)[kPad]>(dsm);                      // [64][kPad]
-  float (*qs)[kPad] = reinterpret_cast<float (*)[kPad]>(dsm + SML_PAGE_TOKENS * kPad);
-  __shared__ float ksc[SML_PAGE_TOKENS];
-  __shared__ float wsh[SML_INDEX_HEADS];
-  __shared__ float part[4][SML_PAGE_TOKENS];
-  const int tid = threadIdx.x;
-  const int pg = blockIdx.x, r = blockIdx.y;
-  const Req rq = load_request(cu_q, ctx_len, r, T, max_ctx, max_pages);
-  const int q0 = rq.q0, Q = rq.Q, L = rq.L;
-  if (!rq.ok) {
-    if (pg == 0 && blockIdx.z == 0 && tid == 0) raise_fault(status, SML_FAULT_LENGTHS);
-    return;
-  }
-  if (pg * SML_PAGE_TOKENS >= L) return;
-  const int jb = blockIdx.z * kQChunk;
-  if (jb >= Q) return;
-  const int je = min(Q, jb + kQChunk);
-  const int phys = __ldg(block_table + (size_t)r * max_pages + pg);
-  if (phys < 0 || phys >= index_pages) {
-    if (tid == 0) raise_fault(status, SML_FAULT_PAGE);
-    return;
-  }
-  const uint8_t* page = index_base + (size_t)phys * SML_INDEX_PAGE_BYTES;
-  for (int v = tid; v < SML_PAGE_TOKENS * SML_INDEX_DIM / 16; v += kThreads) {
-    float tmp[16];
-    e4m3x16_to_f32(__ldg(reinterpret_cast<const uint4*>(page) + v), tmp);
-    const int row = v / 8, col = (v % 8) * 16;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) ks[row][col + i] = tmp[i];
-  }
-  if (tid < SML_PAGE_TOKENS)
-    ksc[tid] = __ldg(reinterpret_cast<const float*>(page + SML_PAGE_TOKENS * SML_INDEX_DIM) + tid);
+struct Params {
+  int B, T, max_ctx, max_pages, ssmax;
+  float s_index;
+  const int32_t* cu_q;
+  const int32_t* ctx_len;
+  const int32_t* block_table;
+  const float* iq_scale;
+  const float* iw;
+  const uint8_t* index_base;
+  int64_t index_pages;
+  float* scores;
+  int32_t* status;
+};
 
-  const int tok = tid & 63, hg = tid >> 6;
-  for (int j = jb; j < je; ++j) {
-    const int n = L - Q + j + 1;
-    if (pg * SML_PAGE_TOKENS >= n) continue;  // uniform: page not visible to query j
-    const int t = q0 + j;
-    __syncthreads();
-    const uint8_t* qrow = iq8 + (size_t)t * SML_INDEX_HEADS * SML_INDEX_DIM;
-    for (int v = tid; v < SML_INDEX_HEADS * SML_INDEX_DIM / 16; v += kThreads) {
-      float tmp[16];
-      e4m3x16_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow) + v), tmp);
-      const int row = v / 8, col = (v % 8) * 16;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) qs[row][col + i] = tmp[i];
-    }
-    if (tid < SML_INDEX_HEADS) wsh[tid] = __ldg(iw + (size_t)t * SML_INDEX_HEADS + tid);
-    __syncthreads();
-    float acc = 0.f;
-    for (int h = hg * 16; h < hg * 16 + 16; ++h) {
-      float dot = 0.f;
-#pragma unroll 8
-      for (int d = 0; d < SML_INDEX_DIM; ++d) dot = fmaf(qs[h][d], ks[tok][d], dot);
-      acc = fmaf(wsh[h], fmaxf(dot, 0.f), acc);
-    }
-    part[hg][tok] = acc;
-    __syncthreads();
-    if (tid < SML_PAGE_TOKENS) {
-      const int s = pg * SML_PAGE_TOKENS + tid;
-      if (s < n) {
-        const float c = ssmax ? s_index * logf((float)n) : 1.f;
-        const float sum = (part[0][tid] + part[1][tid]) + (part[2][tid] + part[3][tid]);
-        scores[(size_t)t * max_ctx + s] = sum * __ldg(iq_scale + t) * ksc[tid] * c;
+// Walks the work items (request r, query group g, tile) in order.
+struct Walker {
+  const Params* P;
+  int r, g, tile, ngroups, ntiles;
+  Req rq;
+
+  __device__ void load_req() {
+    rq = load_request(P->cu_q, P->ctx_len, r, P->T, P->max_ctx, P->max_pages);
+    ngroups = rq.ok ? (rq.Q + kGroup - 1) / kGroup : 0;
+  }
+  __device__ int group_tiles() const {
+    const int last = min(rq.Q, kGroup * g + kGroup);   // the group's queries: [4g, last)
+    const int n_last = rq.L - rq.Q + last;             // visible length of its last query
+    return (n_last + kTile - 1) / kTile;
+  }
+  __device__ int qg() const { return min(kGroup, rq.Q - kGroup * g); }
+  // Position on item `index` (r == B past the end).
+  __device__ void seek(int index) {
+    for (r = 0; r < P->B; ++r) {
+      load_req();
+      for (g = 0; g < ngroups; ++g) {
+        ntiles = group_tiles();
+        if (index < ntiles) {
+          tile = index;
+          return;
+        }
+        index -= ntiles;
       }
     }
   }
+  __device__ void advance() {
+    if (++tile < ntiles) return;
+    tile = 0;
+    if (++g < ngroups) {
+      ntiles = group_tiles();
+      return;
+    }
+    g = 0;
+    for (++r; r < P->B; ++r) {
+      load_req();
+      if (ngroups > 0) {
+        ntiles = group_tiles();
+        return;
+      }
+    }
+  }
+};
+
+__device__ int count_items(const Params& P, bool report) {
+  int total = 0;
+  Walker w{&P};
+  for (w.r = 0; w.r < P.B; ++w.r) {
+    w.load_req();
+    if (!w.rq.ok && report) raise_fault(P.status, SML_FAULT_LENGTHS);
+    for (w.g = 0; w.g < w.ngroups; ++w.g) total += w.group_tiles();
+  }
+  return total;
+}
+
+// Warp-uniform bounded wait: every lane polls, the warp agrees on the result.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort) {
+  const bool ok = ptx::mbar_wait(bar, parity, abort);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                  const Params P) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      ptx::mbar_init(&S.full[i], 1);
+      ptx::mbar_init(&S.empty[i], 1 + 4);   // MMA commit + one arrive per epilogue warp
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&S.qfull[i], 1);
+      ptx::mbar_init(&S.qempty[i], 1);
+      ptx::mbar_init(&S.accfull[i], 1);
+      ptx::mbar_init(&S.accempty[i], 4);
+    }
+    ptx::mbar_init(&S.drain, 1);
+    S.abort = 0;
+    const int total = count_items(P, blockIdx.x == 0);
+    const long long G = gridDim.x;
+    S.range[0] = (int)((long long)total * blockIdx.x / G);
+    S.range[1] = (int)((long long)total * (blockIdx.x + 1) / G);
+    ptx::fence_mbar_init();
+    ptx::prefetch_tensormap(&kmap);
+    ptx::prefetch_tensormap(&qmap);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&S.tmem_base, 2 * kAccCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const int beg = S.range[0], end = S.range[1];
+  volatile int* abort = &S.abort;
+
+  if (warp == 0) {
+    // ---------------- TMA producer (one lane) ----------------
+    if (lane == 0 && beg < end) {
+      Walker w{&P};
+      w.seek(beg);
+      int stage = 0;
+      uint32_t phase = 0;
+      int qcount = 0, last_r = -1, last_g = -1;
+      for (int it = beg; it < end; ++it, w.advance()) {
+        if (w.r != last_r || w.g != last_g) {
+          const int qb = qcount & 1;
+          if (!ptx::mbar_wait(&S.qempty[qb], ((qcount >> 1) & 1) ^ 1, abort)) { *abort = 1; break; }
+          const int qg = w.qg();
+          ptx::mbar_arrive_expect_tx(&S.qfull[qb], qg * kQRowsBytes);
+          for (int j = 0; j < qg; ++j)
+            ptx::tma_load_2d(&S.q[qb][j * kQRowsBytes], &qmap, &S.qfull[qb], 0,
+                             (w.rq.q0 + kGroup * w.g + j) * SML_INDEX_HEADS);
+          ++qcount;
+          last_r = w.r;
+          last_g = w.g;
+        }
+        if (!ptx::mbar_wait(&S.empty[stage], phase ^ 1, abort)) { *abort = 1; break; }
+        int valid = 0;
+        uint32_t bytes = 0;
+        int phys[2];
+        for (int pg = 0; pg < 2; ++pg) {
+          const int lp = w.tile * 2 + pg;
+          phys[pg] = -1;
+          if (lp * SML_PAGE_TOKENS < w.rq.L) {
+            const int ph = __ldg(P.block_table + (size_t)w.r * P.max_pages + lp);
+            if (ph >= 0 && ph < P.index_pages) {
+              phys[pg] = ph;
+              valid |= 1 << pg;
+              bytes += kPageKeyBytes + SML_PAGE_TOKENS * 4;
+            } else {
+              raise_fault(P.status, SML_FAULT_PAGE);
+            }
+          }
+        }
+        S.valid[stage] = valid;
+        ptx::mbar_arrive_expect_tx(&S.full[stage], bytes);
+        for (int pg = 0; pg < 2; ++pg) {
+          if (phys[pg] < 0) continue;
+          ptx::tma_load_3d(&S.keys[stage][pg * kPageKeyBytes], &kmap, &S.full[stage], 0, 0, phys[pg]);
+          ptx::bulk_load(&S.ksc[stage][pg * SML_PAGE_TOKENS],
+                         P.index_base + (size_t)phys[pg] * SML_INDEX_PAGE_BYTES + kPageKeyBytes,
+                         SML_PAGE_TOKENS * 4, &S.full[stage]);
+        }
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (*abort) {
+        // Let copies already issued land before the CTA's shared memory goes away.
+        for (int i = 0; i < kStages; ++i) ptx::mbar_wait(&S.full[i], phase ^ (i >= stage ? 1u : 0u), nullptr, 1u << 16);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (one lane) ----------------
+    if (lane == 0 && beg < end) {
+      Walker w{&P};
+      w.seek(beg);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, accphase = 0;
+      int qcount = 0, last_r = -1, last_g = -1, qb = 0;
+      for (int it = beg; it < end; ++it, w.advance()) {
+        if (w.r != last_r || w.g != last_g) {
+          if (qcount > 0) ptx::mma_commit(&S.qempty[qb]);   // previous group's queries free once read
+          qb = qcount & 1;
+          if (!ptx::mbar_wait(&S.qfull[qb], (qcount >> 1) & 1, abort)) { *abort = 1; break; }
+          ++qcount;
+          last_r = w.r;
+          last_g = w.g;
+        }
+        if (!ptx::mbar_wait(&S.accempty[acc], accphase ^ 1, abort)) { *abort = 1; break; }
+        if (!ptx::mbar_wait(&S.full[stage], phase, abort)) { *abort = 1; break; }
+        ptx::tc_fence_after();
+        const uint32_t idesc = ptx::idesc_m128(SML_INDEX_HEADS * w.qg(), 0);
+        const uint32_t d = S.tmem_base + acc * kAccCols;
+        const uint32_t a0 = ptx::smem_u32(S.keys[stage]);
+        const uint32_t b0 = ptx::smem_u32(S.q[qb]);
+#pragma unroll
+        for (int k = 0; k < SML_INDEX_DIM / 32; ++k)
+          ptx::mma_f8f6f4_ss(d, ptx::sdesc_sw128(a0 + 32 * k), ptx::sdesc_sw128(b0 + 32 * k), idesc, k > 0);
+        ptx::mma_commit(&S.empty[stage]);
+        ptx::mma_commit(&S.accfull[acc]);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+        if (++acc == 2) {
+          acc = 0;
+          accphase ^= 1;
+        }
+      }
+    }
+    if (lane == 0) {
+      // Every MMA this thread issued has finished before TMEM is released.
+      ptx::mma_commit(&S.drain);
+      ptx::mbar_wait(&S.drain, 0, nullptr, 1u << 20);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue: warps 2..5, one thread per token row ----------------
+    const int quarter = warp & 3;               // TMEM lanes 32 * quarter .. + 31
+    const int row = quarter * 32 + lane;
+    const int et = threadIdx.x - 64;            // 0..127
+    Walker w{&P};
+    if (beg < end) w.seek(beg);
+    int stage = 0, acc = 0;
+    uint32_t phase = 0, accphase = 0;
+    int last_r = -1, last_g = -1;
+    for (int it = beg; it < end; ++it, w.advance()) {
+      const int qg = w.qg();
+      const int j0 = kGroup * w.g;
+      if (w.r != last_r || w.g != last_g) {
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        for (int i = et; i < qg * SML_INDEX_HEADS; i += 128)
+          S.w[i] = __ldg(P.iw + (size_t)(w.rq.q0 + j0) * SML_INDEX_HEADS + i);
+        if (et < qg) {
+          const int n = w.rq.L - w.rq.Q + j0 + et + 1;
+          const float c = P.ssmax ? P.s_index * logf((float)n) : 1.f;
+          S.qf[et] = __ldg(P.iq_scale + w.rq.q0 + j0 + et) * c;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        last_r = w.r;
+        last_g = w.g;
+      }
+      if (!warp_wait(&S.accfull[acc], accphase, abort)) { *abort = 1; break; }
+      if (!warp_wait(&S.full[stage], phase, abort)) { *abort = 1; break; }
+      ptx::tc_fence_after();
+      const float sk = S.ksc[stage][row];
+      const bool row_ok = (S.valid[stage] >> (row >> 6)) & 1;
+      const int s = w.tile * kTile + row;
+      const uint32_t tbase = S.tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * kAccCols;
+      for (int j = 0; j < qg; ++j) {
+        float sum = 0.f;
+#pragma unroll
+        for (int c = 0; c < SML_INDEX_HEADS / 32; ++c) {
+          uint32_t v[32];
+          ptx::tmem_ld32(tbase + j * SML_INDEX_HEADS + c * 32, v);
+          ptx::tmem_wait_ld();
+          const float* wj = S.w + j * SML_INDEX_HEADS + c * 32;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sum = fmaf(wj[i], fmaxf(__uint_as_float(v[i]), 0.f), sum);
+        }
+        const int n = w.rq.L - w.rq.Q + j0 + j + 1;
+        if (row_ok && s < n) P.scores[(size_t)(w.rq.q0 + j0 + j) * P.max_ctx + s] = sum * S.qf[j] * sk;
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        ptx::mbar_arrive(&S.accempty[acc]);
+        ptx::mbar_arrive(&S.empty[stage]);
+      }
+      if (++stage == kStages) {
+        stage = 0;
+        phase ^= 1;
+      }
+      if (++acc == 2) {
+        acc = 0;
+        accphase ^= 1;
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && S.abort) raise_fault(P.status, SML_FAULT_TIMEOUT);
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(S.tmem_base, 2 * kAccCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
 }
 
 }  // namespace
@@ -117,16 +371,51 @@ indexer_page_kernel(int B, int T, int max_pages, int max_ctx, int ssmax, float s
 cudaError_t launch_indexer(const sml_problem& p, const uint8_t* iq8, const float* iq_scale,
                            const float* iw, const uint8_t* index_base, int64_t index_pages,
                            float* scores, int32_t* status, cudaStream_t stream) {
-  // Query chunks: enough for the request with the most query tokens (<= T).
-  const int qchunks = (p.num_tokens - p.num_requests + 1 + kQChunk - 1) / kQChunk;
-  dim3 grid(p.max_pages, p.num_requests, qchunks);
-  const size_t smem = (size_t)(SML_PAGE_TOKENS + SML_INDEX_HEADS) * kPad * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(indexer_page_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap kmap, qmap;
+  {
+    // The pool as [pages][64 rows][128 B]: one box = the 64 keys of one page.
+    cuuint64_t dims[3] = {SML_INDEX_DIM, SML_PAGE_TOKENS, (cuuint64_t)index_pages};
+    cuuint64_t strides[2] = {SML_INDEX_DIM, SML_INDEX_PAGE_BYTES};
+    cuuint32_t box[3] = {SML_INDEX_DIM, SML_PAGE_TOKENS, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(index_base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    // Indexer queries as [T * 64 rows][128 B]: one box = the 64 heads of a token.
+    cuuint64_t dims[2] = {SML_INDEX_DIM, (cuuint64_t)p.num_tokens * SML_INDEX_HEADS};
+    cuuint64_t strides[1] = {SML_INDEX_DIM};
+    cuuint32_t box[2] = {SML_INDEX_DIM, SML_INDEX_HEADS};
+    cuuint32_t estr[2] = {1, 1};
+    if (enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(iq8), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  Params P;
+  P.B = p.num_requests;
+  P.T = p.num_tokens;
+  P.max_ctx = p.max_ctx;
+  P.max_pages = p.max_pages;
+  P.ssmax = p.ssmax;
+  P.s_index = p.ssmax_s_index;
+  P.cu_q = p.cu_q;
+  P.ctx_len = p.ctx_len;
+  P.block_table = p.block_table;
+  P.iq_scale = iq_scale;
+  P.iw = iw;
+  P.index_base = index_base;
+  P.index_pages = index_pages;
+  P.scores = scores;
+  P.status = status;
+  const size_t smem = sizeof(Smem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  indexer_page_kernel<<<grid, kThreads, smem, stream>>>(
-      p.num_requests, p.num_tokens, p.max_pages, p.max_ctx, p.ssmax, p.ssmax_s_index, p.cu_q, p.ctx_len,
-      p.block_table, iq8, iq_scale, iw, index_base, index_pages, scores, status);
+  indexer_tc_kernel<<<num_sms(), kThreads, smem, stream>>>(kmap, qmap, P);
   return cudaGetLastError();
 }
 
