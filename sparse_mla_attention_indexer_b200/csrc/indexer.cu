@@ -8,11 +8,12 @@
 //
 // Design (one persistent CTA per SM, warp-specialised):
 //   * a work item is (request, query group of <= 4 tokens, 128-token tile);
-//     items are enumerated on the device from cu_q / ctx_len and split evenly
-//     over the CTAs, so the host never reads device data;
+//     items are counted on the device from cu_q / ctx_len (one round of
+//     parallel loads per 192 requests) and split evenly over the CTAs, so the
+//     host never reads device data;
 //   * warp 0 moves the tile's two 64-token key pages into shared memory with
 //     3-D TMA loads (128-B swizzle) over the paged pool, and the pages'
-//     per-token scales with plain bulk copies, into a 6-stage ring;
+//     per-token scales with plain bulk copies, into a 9-stage ring;
 //   * warp 1 issues tcgen05.mma kind::f8f6f4: D[128 tokens, 64 x Qg] =
 //     K[128, 128] . Q[64 x Qg, 128]^T, E4M3 x E4M3 with fp32 accumulation in
 //     TMEM (two 256-column accumulators, so MMA and epilogue overlap);
@@ -30,7 +31,7 @@ namespace sml {
 namespace {
 
 constexpr int kTile = 128;       // tokens per tile = MMA M
-constexpr int kStages = 6;
+constexpr int kStages = 9;
 constexpr int kGroup = 4;        // query tokens per group: N = 64 * Qg <= 256
 constexpr int kAccCols = 256;
 constexpr int kThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
@@ -50,7 +51,8 @@ struct __align__(1024) Smem {
   int valid[kStages];                            // bit p: page p of the tile was loaded
   uint32_t tmem_base;
   int abort;
-  int range[2];
+  int sched[4];   // beg, end, first request, offset in it
+  int red[kThreads / 32];
 };
 
 struct Params {
@@ -83,19 +85,22 @@ struct Walker {
     return (n_last + kTile - 1) / kTile;
   }
   __device__ int qg() const { return min(kGroup, rq.Q - kGroup * g); }
-  // Position on item `index` (r == B past the end).
-  __device__ void seek(int index) {
-    for (r = 0; r < P->B; ++r) {
-      load_req();
-      for (g = 0; g < ngroups; ++g) {
-        ntiles = group_tiles();
-        if (index < ntiles) {
-          tile = index;
-          return;
-        }
-        index -= ntiles;
-      }
+  // Position on item `off` of request r0 (which has more than `off` items).
+  __device__ void start(int r0, int off) {
+    r = r0;
+    load_req();
+    for (g = 0; g < ngroups; ++g) {
+      ntiles = group_tiles();
+      if (off < ntiles) break;
+      off -= ntiles;
     }
+    tile = off;
+  }
+  // Items of the current request.
+  __device__ int request_items() {
+    int total = 0;
+    for (g = 0; g < ngroups; ++g) total += group_tiles();
+    return total;
   }
   __device__ void advance() {
     if (++tile < ntiles) return;
@@ -115,15 +120,84 @@ struct Walker {
   }
 };
 
-__device__ int count_items(const Params& P, bool report) {
-  int total = 0;
-  Walker w{&P};
-  for (w.r = 0; w.r < P.B; ++w.r) {
-    w.load_req();
-    if (!w.rq.ok && report) raise_fault(P.status, SML_FAULT_LENGTHS);
-    for (w.g = 0; w.g < w.ngroups; ++w.g) total += w.group_tiles();
+// Block-wide sum of one int per thread (all kThreads threads call it).
+__device__ __forceinline__ int block_sum(int v, int* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  int s = 0;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) s += red[w];
+  return s;
+}
+
+// Block-wide inclusive scan of one int per thread; *sum gets the block total.
+__device__ __forceinline__ int block_scan(int v, int* red, int* sum) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
   }
-  return total;
+  __syncthreads();
+  if (lane == 31) red[warp] = v;
+  __syncthreads();
+  int before = 0, s = 0;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) {
+    before += w < warp ? red[w] : 0;
+    s += red[w];
+  }
+  *sum = s;
+  return v + before;
+}
+
+// This CTA's share of the work items and where it starts (request, offset),
+// with every thread loading one request at a time: a round of parallel loads
+// per kThreads requests instead of one dependent load chain per request.
+__device__ void schedule(const Params& P, int* red, int* out /* beg, end, r0, off0 */) {
+  int total = 0;
+  for (int base = 0; base < P.B; base += kThreads) {
+    Walker w{&P};
+    w.r = base + threadIdx.x;
+    int cnt = 0;
+    if (w.r < P.B) {
+      w.load_req();
+      if (!w.rq.ok && blockIdx.x == 0) raise_fault(P.status, SML_FAULT_LENGTHS);
+      cnt = w.request_items();
+    }
+    total += block_sum(cnt, red);
+  }
+  const long long G = gridDim.x;
+  const int beg = (int)((long long)total * blockIdx.x / G);
+  const int end = (int)((long long)total * (blockIdx.x + 1) / G);
+  if (threadIdx.x == 0) {
+    out[0] = beg;
+    out[1] = end;
+    out[2] = P.B;
+    out[3] = 0;
+  }
+  if (beg >= end) return;
+  int acc = 0;
+  for (int base = 0; base < P.B && acc <= beg; base += kThreads) {
+    Walker w{&P};
+    w.r = base + threadIdx.x;
+    int cnt = 0;
+    if (w.r < P.B) {
+      w.load_req();
+      cnt = w.request_items();
+    }
+    int sum;
+    const int incl = block_scan(cnt, red, &sum);
+    if (cnt > 0 && beg >= acc + incl - cnt && beg < acc + incl) {
+      out[2] = w.r;
+      out[3] = beg - (acc + incl - cnt);
+    }
+    acc += sum;
+  }
 }
 
 // Warp-uniform bounded wait: every lane polls, the warp agrees on the result.
@@ -152,10 +226,6 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     }
     ptx::mbar_init(&S.drain, 1);
     S.abort = 0;
-    const int total = count_items(P, blockIdx.x == 0);
-    const long long G = gridDim.x;
-    S.range[0] = (int)((long long)total * blockIdx.x / G);
-    S.range[1] = (int)((long long)total * (blockIdx.x + 1) / G);
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&kmap);
     ptx::prefetch_tensormap(&qmap);
@@ -164,17 +234,18 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     ptx::tmem_alloc(&S.tmem_base, 2 * kAccCols);
     ptx::tmem_relinquish();
   }
+  schedule(P, S.red, S.sched);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  const int beg = S.range[0], end = S.range[1];
+  const int beg = S.sched[0], end = S.sched[1];
   volatile int* abort = &S.abort;
 
   if (warp == 0) {
     // ---------------- TMA producer (one lane) ----------------
     if (lane == 0 && beg < end) {
       Walker w{&P};
-      w.seek(beg);
+      w.start(S.sched[2], S.sched[3]);
       int stage = 0;
       uint32_t phase = 0;
       int qcount = 0, last_r = -1, last_g = -1;
@@ -233,7 +304,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     // ---------------- MMA issuer (one lane) ----------------
     if (lane == 0 && beg < end) {
       Walker w{&P};
-      w.seek(beg);
+      w.start(S.sched[2], S.sched[3]);
       int stage = 0, acc = 0;
       uint32_t phase = 0, accphase = 0;
       int qcount = 0, last_r = -1, last_g = -1, qb = 0;
@@ -280,7 +351,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     const int row = quarter * 32 + lane;
     const int et = threadIdx.x - 64;            // 0..127
     Walker w{&P};
-    if (beg < end) w.seek(beg);
+    if (beg < end) w.start(S.sched[2], S.sched[3]);
     int stage = 0, acc = 0;
     uint32_t phase = 0, accphase = 0;
     int last_r = -1, last_g = -1;

@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
   const int Dq = SML_LATENT_DIM + P.rope_dim;
 
   // ---- this split's key range (uniform across the CTA) ----
-  const int r = request_of(P.cu_q, P.B, t);
+  const int r = request_of_warp(P.cu_q, P.B, t);
   const Req rq = load_request(P.cu_q, P.ctx_len, r, P.T, P.max_ctx, P.max_pages);
   const bool req_ok = rq.ok && t >= rq.q0 && t - rq.q0 < rq.Q;
   const int n = req_ok ? rq.L - rq.Q + (t - rq.q0) + 1 : 0;
@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
   const int nchunks = ntiles * (kKT / kChunk);
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(&S.q_ready, kConvWarps);
+    ptx::mbar_init(&S.q_ready, 4);
     ptx::mbar_init(&S.rows_ready, kConvWarps);
     ptx::mbar_init(&S.e_full, kConvWarps);
     ptx::mbar_init(&S.s_full, 1);
@@ -198,44 +198,38 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
     constexpr int kCT = kConvWarps * 32;
     constexpr int kRowsPerWarp = kChunk / kConvWarps;
     const int cw = warp - 6, ct = threadIdx.x - 6 * 32;
-    // Pool rows of the split's keys.
-    for (int k = ct; k < kMaxSplit; k += kCT) {
+    // Pool rows of the split's keys: all position loads first, then all
+    // block-table loads, so each thread waits for two latencies, not eight.
+    constexpr int kPer = kMaxSplit / kCT;
+    int pos[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int k = ct + j * kCT;
+      pos[j] = k < nkeys ? __ldg(P.idx + (size_t)t * P.K + kb + k) : -1;
+    }
+    int ph[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int k = ct + j * kCT;
+      const bool in = k < nkeys && pos[j] >= 0 && pos[j] < n;
+      if (k < nkeys && !in) raise_fault(P.status, SML_FAULT_INDEX);
+      ph[j] = in ? __ldg(P.block_table + (size_t)r * P.max_pages + pos[j] / SML_PAGE_TOKENS) : -1;
+      if (!in) pos[j] = -1;
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int k = ct + j * kCT;
       int32_t id = -1;
-      if (k < nkeys) {
-        const int pos = __ldg(P.idx + (size_t)t * P.K + kb + k);
-        if (pos >= 0 && pos < n) {
-          const int ph = __ldg(P.block_table + (size_t)r * P.max_pages + pos / SML_PAGE_TOKENS);
-          if (ph >= 0 && ph < P.latent_pages)
-            id = ph * SML_PAGE_TOKENS + pos % SML_PAGE_TOKENS;
-          else
-            raise_fault(P.status, SML_FAULT_PAGE);
-        } else {
-          raise_fault(P.status, SML_FAULT_INDEX);
-        }
+      if (pos[j] >= 0) {
+        if (ph[j] >= 0 && ph[j] < P.latent_pages)
+          id = ph[j] * SML_PAGE_TOKENS + pos[j] % SML_PAGE_TOKENS;
+        else
+          raise_fault(P.status, SML_FAULT_PAGE);
       }
       S.rowid[k] = id;
     }
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(&S.rows_ready);
-    // Query heads of this group: nope bf16 -> fp16, RoPE part copied (bf16).
-    const uint16_t* qbase = P.q + ((size_t)t * P.H + hg * kHC) * Dq;
-    for (int e = ct; e < kHC * (Dq / 8); e += kCT) {
-      const int h = e / (Dq / 8), c8 = e % (Dq / 8);    // 8 elements = one 16-B chunk
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(qbase + (size_t)h * Dq) + c8);
-      if (c8 < 64) {
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t o[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          o[i] = pack_half2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
-        st_shared_v4(sw128(ptx::smem_u32(S.q[c8 >> 3]), h, c8 & 7), o[0], o[1], o[2], o[3]);
-      } else {
-        st_shared_v4(sw128(ptx::smem_u32(S.qpe), h, c8 - 64), v.x, v.y, v.z, v.w);
-      }
-    }
-    ptx::fence_proxy_async();
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(&S.q_ready);
 
     int chunk = 0;
     for (int tile = 0; tile < ntiles; ++tile) {
@@ -359,6 +353,28 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
   } else {
     // ================= softmax: warps 0-3, thread = key row / latent dim =================
     const int row = warp * 32 + lane;
+    {
+      // Query heads of this group, while the other warps resolve the key rows:
+      // nope bf16 -> fp16 (exact in fp16's normal range), RoPE part copied as bf16.
+      const uint16_t* qbase = P.q + ((size_t)t * P.H + hg * kHC) * Dq;
+      for (int e = row; e < kHC * (Dq / 8); e += 128) {
+        const int h = e / (Dq / 8), c8 = e % (Dq / 8);    // 8 elements = one 16-B chunk
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(qbase + (size_t)h * Dq) + c8);
+        if (c8 < 64) {
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            o[i] = pack_half2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+          st_shared_v4(sw128(ptx::smem_u32(S.q[c8 >> 3]), h, c8 & 7), o[0], o[1], o[2], o[3]);
+        } else {
+          st_shared_v4(sw128(ptx::smem_u32(S.qpe), h, c8 - 64), v.x, v.y, v.z, v.w);
+        }
+      }
+      ptx::fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&S.q_ready);
+    }
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const float zscale = P.sm_scale * (P.ssmax ? P.ssmax_s * logf((float)max(n, 1)) : 1.f);
     float m[kHC];
@@ -547,11 +563,12 @@ lse_merge_kernel(int H, MlaWs ws, float* __restrict__ out, float* __restrict__ l
 }  // namespace
 
 int mla_splits(const sml_problem& p, int* keys_per_split) {
-  // Splits of whole 128-key tiles, at most 512 keys: enough CTAs to fill the
-  // GPU about twice, no more.
+  // Splits of whole 128-key tiles, at most 512 keys: about one CTA per SM for
+  // the whole problem, so the per-CTA set-up is paid once per SM and the
+  // gather of a tile overlaps the math of the one before.
   const int tiles = (p.topk + kKT - 1) / kKT;
   const int ctas = p.num_tokens * (p.num_heads / kHC);
-  int tps = (int)(((long long)ctas * tiles + 2 * 148 - 1) / (2 * 148));
+  int tps = (int)(((long long)ctas * tiles + 148 - 1) / 148);
   tps = tps < 1 ? 1 : (tps > kMaxSplit / kKT ? kMaxSplit / kKT : tps);
   if (tps > tiles) tps = tiles;
   const int kps = tps * kKT;

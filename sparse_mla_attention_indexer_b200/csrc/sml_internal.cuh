@@ -25,7 +25,7 @@ inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // Top-k: one CTA selects over a chunk of up to kTopkChunk positions held in
 // shared memory; longer rows are cut into chunks whose candidates the last
 // arriving CTA of the row merges.
-constexpr int kTopkChunk = 32768;
+constexpr int kTopkChunk = 16384;
 constexpr int kTopkThreads = 1024;
 
 struct TopkWs {
@@ -61,6 +61,24 @@ __device__ __forceinline__ int request_of(const int32_t* __restrict__ cu_q, int 
   while (lo < hi) {
     int mid = (lo + hi + 1) >> 1;
     if (__ldg(cu_q + mid) <= t) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// The same lookup by one full warp: a 32-way search, one round of parallel
+// loads for B <= 32 (log32(B) rounds in general) instead of log2(B) dependent
+// loads.  Every lane returns the same request.
+__device__ __forceinline__ int request_of_warp(const int32_t* __restrict__ cu_q, int B, int t) {
+  const int lane = threadIdx.x & 31;
+  int lo = 0, hi = B;   // answer in [lo, hi)
+  while (hi - lo > 1) {
+    const int step = (hi - lo + 31) / 32;
+    const int j = lo + lane * step;
+    const bool le = j < hi && __ldg(cu_q + j) <= t;
+    const unsigned mask = __ballot_sync(0xffffffffu, le);
+    const int last = mask ? 31 - __clz(mask) : 0;
+    lo = lo + last * step;
+    hi = min(hi, lo + step);
   }
   return lo;
 }

@@ -1,17 +1,23 @@
-// Exact per-row top-k by radix select in shared memory.
+// Exact per-row top-k over the indexer scores.
 //
 // The pages (vLLM blog on Mistral Large 4, section "ROCm 实现细节", paragraph on
 // the persistent fused decode) require an exact top-2048; the DCP paragraph of
 // section "长上下文" mentions the radix select that vLLM's candidate exchange
-// replaced.  This is a single-GPU radix select written for sm_100a:
+// replaced.  This is a single-GPU select written for sm_100a:
 //
 //  * scores become order-preserving 32-bit keys (-0 -> +0, NaN lowest);
-//  * three histogram passes over 11 / 11 / 10 key bits find the k-th largest
-//    key tau and how many keys equal to tau are taken;
-//  * a final pass in position order emits every key > tau and the lowest
-//    positions among keys == tau, so the output is in ascending position
-//    order and ties go to the lower position by construction;
-//  * a row longer than one chunk (32,768 positions) is cut into chunks, each
+//  * one pass histograms the values into 2,048 buckets linear in value between
+//    the row's finite min and max (-inf / NaN in the lowest bucket, +inf in the
+//    highest), which spreads the bins for shared-memory atomics and finds the
+//    bucket that holds the k-th largest value;
+//  * only that bucket's keys (a handful, typically) go through an exact radix
+//    select (11 / 11 / 10 key bits) to find the k-th largest key tau and how
+//    many keys equal to tau are taken; a row whose threshold bucket is huge
+//    (heavy ties) runs the radix select over all its keys instead;
+//  * a last pass in position order, one warp per contiguous range, emits every
+//    key > tau and the lowest positions among keys == tau: the output is in
+//    ascending position order and ties go to the lower position;
+//  * rows longer than one chunk (16,384 positions) are cut into chunks, each
 //    selected by its own CTA into a candidate list; the last CTA of the row to
 //    finish (an arrival counter, no waiting) selects again over the
 //    concatenated candidates.  The global top-k is a subset of the union of
@@ -21,6 +27,9 @@
 namespace sml {
 namespace {
 
+constexpr int kBuckets = 2048;
+constexpr int kCandCap = 4096;
+
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t b = __float_as_uint(f);
   if ((b & 0x7fffffffu) > 0x7f800000u) return 0u;  // NaN ranks below -inf
@@ -28,9 +37,17 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// Inverse of order_key (NaN comes back as a NaN).
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 struct SelectShared {
-  int hist[2048];
-  int warp_tot[32];
+  int hist[kBuckets];
+  uint32_t cand[kCandCap];
+  int warp_a[32], warp_b[32];
+  float red_lo[32], red_hi[32];
+  int ncand;
   int bcast[2];
 };
 
@@ -60,16 +77,36 @@ __device__ __forceinline__ int block_scan_incl(int v, int* warp_tot, int* total)
   return v;
 }
 
-// Select the k largest of n keys (key_at(i), i in [0, n)); call emit(pos, i)
-// for each selected i, pos = its rank in ascending i order.  All threads of the
-// block must call it.  Requires blockDim.x == kTopkThreads.
-template <typename KeyAt, typename Emit>
-__device__ void select_topk(int n, int k, KeyAt key_at, Emit emit, SelectShared& sh) {
-  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
-  if (n <= k) {
-    for (int i = tid; i < n; i += nt) emit(i, i);
-    return;
+// Over the histogram sh.hist[0, nb): the bin holding the `need`-th largest
+// element, and how many elements lie in the bins above it.
+__device__ __forceinline__ void find_bin(int nb, int need, SelectShared& sh, int* bin, int* above_out) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int bpt = nb / nt;   // nb is a multiple of nt
+  int local = 0;
+  for (int j = 0; j < bpt; ++j) local += sh.hist[nb - 1 - (tid * bpt + j)];
+  int total;
+  const int incl = block_scan_incl(local, sh.warp_a, &total);
+  int above = incl - local;
+  for (int j = 0; j < bpt; ++j) {
+    const int b = nb - 1 - (tid * bpt + j);
+    const int h = sh.hist[b];
+    if (above < need && need <= above + h) {
+      sh.bcast[0] = b;
+      sh.bcast[1] = above;
+    }
+    above += h;
   }
+  __syncthreads();
+  *bin = sh.bcast[0];
+  *above_out = sh.bcast[1];
+  __syncthreads();
+}
+
+// Radix select over n keys: the k-th largest key tau (1 <= k <= n) and how
+// many keys equal to tau belong to the top k (*take).
+template <typename KeyAt>
+__device__ void radix_threshold(int n, int k, KeyAt key_at, SelectShared& sh, uint32_t* tau, int* take) {
+  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
   uint32_t prefix = 0, pmask = 0;
   int remaining = k;
   const int shifts[3] = {21, 10, 0};
@@ -90,47 +127,129 @@ __device__ void select_topk(int n, int k, KeyAt key_at, Emit emit, SelectShared&
       if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], __popc(peers));
     }
     __syncthreads();
-    // Bins in descending order, nb / nt consecutive bins per thread.
-    const int bpt = nb / nt;
-    int local = 0;
-    for (int j = 0; j < bpt; ++j) local += sh.hist[nb - 1 - (tid * bpt + j)];
-    int total;
-    const int incl = block_scan_incl(local, sh.warp_tot, &total);
-    int above = incl - local;  // keys in bins higher than this thread's bins
-    for (int j = 0; j < bpt; ++j) {
-      const int b = nb - 1 - (tid * bpt + j);
-      const int h = sh.hist[b];
-      if (above < remaining && remaining <= above + h) {
-        sh.bcast[0] = b;
-        sh.bcast[1] = above;
-      }
-      above += h;
-    }
-    __syncthreads();
-    const int b = sh.bcast[0];
-    remaining -= sh.bcast[1];
+    int b, above;
+    find_bin(nb, remaining, sh, &b, &above);
+    remaining -= above;
     prefix |= (uint32_t)b << shift;
     pmask |= (uint32_t)(nb - 1) << shift;
-    __syncthreads();
   }
-  const uint32_t tau = prefix;
-  int gt_run = 0, eq_run = 0;
-  for (int base = 0; base < n; base += nt) {
-    const int i = base + tid;
-    const uint32_t key = i < n ? key_at(i) : 0u;
-    const int gt = (i < n) && key > tau;
-    const int eq = (i < n) && key == tau;
-    const int packed = (gt << 16) | eq;
-    int total;
-    const int incl = block_scan_incl(packed, sh.warp_tot, &total);
-    const int excl = incl - packed;
-    const int gt_before = gt_run + (excl >> 16);
-    const int eq_before = eq_run + (excl & 0xffff);
-    if (gt || (eq && eq_before < remaining)) emit(gt_before + min(eq_before, remaining), i);
-    gt_run += total >> 16;
-    eq_run += total & 0xffff;
-    if (gt_run + min(eq_run, remaining) >= k) break;  // uniform across the block
+  *tau = prefix;
+  *take = remaining;
+}
+
+// Select the k largest of n keys (key_at(i), i in [0, n)); call emit(pos, i)
+// for each selected i, pos = its rank in ascending i order.  All threads of the
+// block call it; blockDim.x == kTopkThreads.
+template <typename KeyAt, typename Emit>
+__device__ void select_topk(int n, int k, KeyAt key_at, Emit emit, SelectShared& sh) {
+  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  if (n <= k) {
+    for (int i = tid; i < n; i += nt) emit(i, i);
+    return;
   }
+  // 1. finite range of the values
+  float lo = INFINITY, hi = -INFINITY;
+  for (int i = tid; i < n; i += nt) {
+    const float v = key_value(key_at(i));
+    if (isfinite(v)) {
+      lo = fminf(lo, v);
+      hi = fmaxf(hi, v);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    sh.red_lo[warp] = lo;
+    sh.red_hi[warp] = hi;
+  }
+  for (int b = tid; b < kBuckets; b += nt) sh.hist[b] = 0;
+  if (tid == 0) sh.ncand = 0;
+  __syncthreads();
+  lo = INFINITY;
+  hi = -INFINITY;
+  for (int w = 0; w < nt / 32; ++w) {
+    lo = fminf(lo, sh.red_lo[w]);
+    hi = fmaxf(hi, sh.red_hi[w]);
+  }
+  // 2. value-linear buckets: 0 = NaN / -inf, 1 .. kBuckets-2 finite, top = +inf.
+  // A range too wide for fp32 gives scale 0: every finite value in bucket 1.
+  const float width = hi - lo;
+  const float scale = (hi > lo && width < INFINITY) ? (float)(kBuckets - 3) / width : 0.f;
+  auto bucket = [&](uint32_t key) -> int {
+    const float v = key_value(key);
+    if (!(v > -INFINITY)) return 0;                               // NaN or -inf
+    if (v == INFINITY) return kBuckets - 1;
+    const float x = fminf(fmaxf((v - lo) * scale, 0.f), (float)(kBuckets - 3));   // monotone in v
+    return 1 + (int)x;
+  };
+  for (int i = tid; i < n; i += nt) atomicAdd(&sh.hist[bucket(key_at(i))], 1);
+  __syncthreads();
+  int bk, above;
+  find_bin(kBuckets, k, sh, &bk, &above);
+  // 3. the keys of the threshold bucket
+  for (int i = tid; i < n; i += nt) {
+    const uint32_t key = key_at(i);
+    if (bucket(key) == bk) {
+      const int slot = atomicAdd(&sh.ncand, 1);
+      if (slot < kCandCap) sh.cand[slot] = key;
+    }
+  }
+  __syncthreads();
+  const int nc = sh.ncand;
+  uint32_t tau;
+  int take;
+  if (nc <= kCandCap) {
+    radix_threshold(nc, k - above, [&](int i) { return sh.cand[i]; }, sh, &tau, &take);
+  } else {
+    radix_threshold(n, k, key_at, sh, &tau, &take);   // heavy ties: over every key
+  }
+  // 4. emission in position order; warp w owns a contiguous range
+  const int nw = nt / 32;
+  const int seg = ((n + nw - 1) / nw + 31) & ~31;
+  const int beg = min(n, warp * seg), end = min(n, beg + seg);
+  int cgt = 0, ceq = 0;
+  for (int i0 = beg; i0 < end; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t key = i < end ? key_at(i) : 0u;
+    cgt += __popc(__ballot_sync(0xffffffffu, i < end && key > tau));
+    ceq += __popc(__ballot_sync(0xffffffffu, i < end && key == tau));
+  }
+  if (lane == 0) {
+    sh.warp_a[warp] = cgt;
+    sh.warp_b[warp] = ceq;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int a = sh.warp_a[lane], b = sh.warp_b[lane];
+    const int a0 = a, b0 = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, a, o), y = __shfl_up_sync(0xffffffffu, b, o);
+      if (lane >= o) {
+        a += x;
+        b += y;
+      }
+    }
+    sh.warp_a[lane] = a - a0;   // exclusive prefix over the warps
+    sh.warp_b[lane] = b - b0;
+  }
+  __syncthreads();
+  int g = sh.warp_a[warp], e = sh.warp_b[warp];
+  const unsigned below = (1u << lane) - 1u;
+  for (int i0 = beg; i0 < end; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t key = i < end ? key_at(i) : 0u;
+    const bool gt = i < end && key > tau, eq = i < end && key == tau;
+    const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+    const int gb = g + __popc(bg & below), eb = e + __popc(be & below);
+    if (gt || (eq && eb < take)) emit(gb + min(eb, take), i);
+    g += __popc(bg);
+    e += __popc(be);
+  }
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(kTopkThreads, 1)
@@ -143,7 +262,7 @@ topk_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32_t* __re
   __shared__ int is_last;
   const int tid = threadIdx.x, nt = blockDim.x;
   const int t = blockIdx.y, c = blockIdx.x;
-  const int r = request_of(cu_q, B, t);
+  const int r = request_of_warp(cu_q, B, t);
   const Req rq = load_request(cu_q, ctx_len, r, T, max_ctx, max_pages);
   const int q0 = rq.q0, Q = rq.Q, L = rq.L;
   int32_t* out = idx + (size_t)t * K;
@@ -220,8 +339,8 @@ cudaError_t launch_topk(const sml_problem& p, const float* scores, int32_t* idx,
   if (e != cudaSuccess) return e;
   dim3 grid(ws.chunks, p.num_tokens);
   topk_kernel<<<grid, kTopkThreads, smem, stream>>>(p.num_requests, p.num_tokens, p.topk,
-                                                    p.max_ctx, p.max_pages, p.cu_q,
-                                                    p.ctx_len, scores, idx, idx_len, ws, status);
+                                                    p.max_ctx, p.max_pages, p.cu_q, p.ctx_len,
+                                                    scores, idx, idx_len, ws, status);
   return cudaGetLastError();
 }
 
