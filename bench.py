@@ -8,10 +8,12 @@ One step = one layer's sparse attention over one batch: the default workload is
 64 indexer heads of dim 128, top-2048, 64-token pages over a permuted shared
 pool (one TP8 rank of batched decode).  Inputs are seeded synthetic data.
 
-Timing: W untimed warm-up steps; then K steps, each preceded by a 256 MiB write
-that flushes L2, each timed on its stream with CUDA events around the three
-stage calls (events between them give per-kernel times); a barrier and a device
-synchronize bracket the timed region; the max over ranks is taken.  Under
+Timing: the step (the three stage calls, with a CUDA event before, between and
+after them) is captured once into a CUDA graph.  W untimed warm-up replays;
+then K replays, each preceded by a 256 MiB write that flushes L2, each timed on
+the device by its events (the events between stages give per-kernel times); a
+barrier and a device synchronize bracket the timed region; the max over ranks
+is taken.  Under
 torchrun each rank runs its own batch on its own GPU (independent requests:
 weak scaling, no data-path collective).
 
@@ -21,6 +23,7 @@ oracle on a bounded sample of the same workload instead.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import subprocess
@@ -152,39 +155,57 @@ def time_ours(args, wl, rank):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
-    def step():
-        sml.sml_indexer_scores(p, lay.iq8, lay.iq_scale, lay.iw, dw.index_cache, scores, ws, stream)
-        ev[1].record(stream)
-        sml.sml_topk(p, scores, idx, ln, ws, stream)
-        ev[2].record(stream)
-        sml.sml_sparse_mla_decode(p, lay.q, dw.latent, idx, ln, out, lse, ws, stream)
+    # One step = the three stage calls, captured once into a CUDA graph with an
+    # event between stages, so the device timeline has no host gaps in it.
+    # Events recorded during capture become timing event nodes only with the
+    # runtime's "external" record flag.
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    cudart = ctypes.CDLL("libcudart.so.12")
+    cudart.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
 
+    def record(e, st, capturing):
+        if capturing:
+            rc = cudart.cudaEventRecordWithFlags(ctypes.c_void_p(e.cuda_event), ctypes.c_void_p(st.cuda_stream), 1)
+            if rc != 0:
+                raise RuntimeError(f"cudaEventRecordWithFlags failed: {rc}")
+        else:
+            e.record(st)
+
+    def step(st, capturing=False):
+        record(ev[0], st, capturing)
+        sml.sml_indexer_scores(p, lay.iq8, lay.iq_scale, lay.iw, dw.index_cache, scores, ws, st)
+        record(ev[1], st, capturing)
+        sml.sml_topk(p, scores, idx, ln, ws, st)
+        record(ev[2], st, capturing)
+        sml.sml_sparse_mla_decode(p, lay.q, dw.latent, idx, ln, out, lse, ws, st)
+        record(ev[3], st, capturing)
+
+    step(stream)                       # first calls outside capture (per-device set-up, events created)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(torch.cuda.current_stream(), capturing=True)
     for _ in range(args.warmup):
         flush.fill_(1)
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        ev[0].record(stream)
-        step()
-        ev[3].record(stream)
+        graph.replay()
     torch.cuda.synchronize()
     code, bits = sml.sml_read_device_status(ws)
     if code != sml.SML_OK:
         raise RuntimeError(f"device status {code} bits {bits:#x}")
 
-    events = []
+    rows = []
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clocks:
         for _ in range(args.steps):
             flush.fill_(1)
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-            ev[0].record(stream)
-            step()
-            ev[3].record(stream)
-            events.append(ev)
-        torch.cuda.synchronize()
+            graph.replay()
+            torch.cuda.synchronize()
+            rows.append([ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]), ev[2].elapsed_time(ev[3]),
+                         ev[0].elapsed_time(ev[3])])
         barrier()
-    per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]),
-                     e[0].elapsed_time(e[3])] for e in events])
+    per = np.array(rows)
+    del graph
     code, bits = sml.sml_read_device_status(ws)
     if code != sml.SML_OK:
         raise RuntimeError(f"device status {code} bits {bits:#x}")

@@ -16,9 +16,11 @@
 //     per-token scales with plain bulk copies, into a 9-stage ring;
 //   * warp 1 issues tcgen05.mma kind::f8f6f4: D[128 tokens, 64 x Qg] =
 //     K[128, 128] . Q[64 x Qg, 128]^T, E4M3 x E4M3 with fp32 accumulation in
-//     TMEM (two 256-column accumulators, so MMA and epilogue overlap);
-//   * warps 2-5 (one thread per token row) read D from TMEM, apply ReLU, the
-//     head weights and sq * sk * c_t, and store the scores of visible positions.
+//     TMEM (eight 64-column accumulators for one-query groups, else two of
+//     256, so MMA and epilogue overlap);
+//   * two epilogue warpgroups (one thread per token row, alternate items)
+//     read D from TMEM, apply ReLU, the head weights and sq * sk * c_t, and
+//     store the scores of visible positions.
 // Every wait is bounded; a wait that gives up sets SML_FAULT_TIMEOUT and the
 // CTA winds down (no trap).
 #include <cudaTypedefs.h>
@@ -31,28 +33,47 @@ namespace sml {
 namespace {
 
 constexpr int kTile = 128;       // tokens per tile = MMA M
-constexpr int kStages = 9;
-constexpr int kGroup = 4;        // query tokens per group: N = 64 * Qg <= 256
-constexpr int kAccCols = 256;
-constexpr int kThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kPageKeyBytes = SML_PAGE_TOKENS * SML_INDEX_DIM;   // 8,192
 constexpr int kQRowsBytes = SML_INDEX_HEADS * SML_INDEX_DIM;      // 8,192 per query token
 
+// Two shapes of the same kernel:
+//   general: 9-stage ring, query groups of up to 4 tokens (N <= 256), two
+//            256-column accumulators, two epilogue warpgroups, one CTA per SM;
+//   decode (every request has one query token): 5-stage ring, one-token groups
+//            (N = 64), four 64-column accumulators, one epilogue warpgroup, and
+//            half the shared memory and TMEM, so two CTAs share each SM and
+//            keep twice the loads in flight.
+template <int kStages_, int kGroup_, int kAccBufs_, int kEpiGroups_, int kCtasPerSm_>
+struct Cfg {
+  static constexpr int kStages = kStages_;
+  static constexpr int kGroup = kGroup_;          // query tokens per group: N = 64 * Qg
+  static constexpr int kAccBufs = kAccBufs_;
+  static constexpr int kAccCols = 64 * kGroup_;
+  static constexpr int kTmemCols = kAccBufs_ * 64 * kGroup_;
+  static constexpr int kEpiGroups = kEpiGroups_;  // epilogue warpgroups, taking alternate items
+  static constexpr int kThreads = 64 + 128 * kEpiGroups_;   // warp 0 TMA, warp 1 MMA, then the epilogue
+  static constexpr int kCtasPerSm = kCtasPerSm_;
+};
+using CfgGeneral = Cfg<9, 4, 2, 2, 1>;
+using CfgDecode = Cfg<5, 1, 4, 1, 2>;
+
+template <class C>
 struct __align__(1024) Smem {
+  static constexpr int kStages = C::kStages, kGroup = C::kGroup, kEpiGroups = C::kEpiGroups;
   uint8_t keys[kStages][2 * kPageKeyBytes];      // [stage][128 rows x 128 B], SW128
   uint8_t q[2][kGroup * kQRowsBytes];            // [buffer][256 rows x 128 B], SW128
   float ksc[kStages][kTile];
-  float w[kGroup * SML_INDEX_HEADS];             // epilogue: head weights of the group
-  float qf[kGroup];                              // epilogue: sq_t * c_t per query
+  float w[kEpiGroups][kGroup * SML_INDEX_HEADS]; // per epilogue warpgroup: head weights of the group
+  float qf[kEpiGroups][kGroup];                  // per epilogue warpgroup: sq_t * c_t per query
   uint64_t full[kStages], empty[kStages];
   uint64_t qfull[2], qempty[2];
-  uint64_t accfull[2], accempty[2];
+  uint64_t accfull[C::kAccBufs], accempty[C::kAccBufs];
   uint64_t drain;
   int valid[kStages];                            // bit p: page p of the tile was loaded
   uint32_t tmem_base;
   int abort;
   int sched[4];   // beg, end, first request, offset in it
-  int red[kThreads / 32];
+  int red[C::kThreads / 32];
 };
 
 struct Params {
@@ -70,6 +91,7 @@ struct Params {
 };
 
 // Walks the work items (request r, query group g, tile) in order.
+template <int kGroup>
 struct Walker {
   const Params* P;
   int r, g, tile, ngroups, ntiles;
@@ -121,6 +143,7 @@ struct Walker {
 };
 
 // Block-wide sum of one int per thread (all kThreads threads call it).
+template <int kThreads>
 __device__ __forceinline__ int block_sum(int v, int* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -135,6 +158,7 @@ __device__ __forceinline__ int block_sum(int v, int* red) {
 }
 
 // Block-wide inclusive scan of one int per thread; *sum gets the block total.
+template <int kThreads>
 __device__ __forceinline__ int block_scan(int v, int* red, int* sum) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -158,10 +182,11 @@ __device__ __forceinline__ int block_scan(int v, int* red, int* sum) {
 // This CTA's share of the work items and where it starts (request, offset),
 // with every thread loading one request at a time: a round of parallel loads
 // per kThreads requests instead of one dependent load chain per request.
+template <int kThreads, int kGroup>
 __device__ void schedule(const Params& P, int* red, int* out /* beg, end, r0, off0 */) {
   int total = 0;
   for (int base = 0; base < P.B; base += kThreads) {
-    Walker w{&P};
+    Walker<kGroup> w{&P};
     w.r = base + threadIdx.x;
     int cnt = 0;
     if (w.r < P.B) {
@@ -169,7 +194,7 @@ __device__ void schedule(const Params& P, int* red, int* out /* beg, end, r0, of
       if (!w.rq.ok && blockIdx.x == 0) raise_fault(P.status, SML_FAULT_LENGTHS);
       cnt = w.request_items();
     }
-    total += block_sum(cnt, red);
+    total += block_sum<kThreads>(cnt, red);
   }
   const long long G = gridDim.x;
   const int beg = (int)((long long)total * blockIdx.x / G);
@@ -183,7 +208,7 @@ __device__ void schedule(const Params& P, int* red, int* out /* beg, end, r0, of
   if (beg >= end) return;
   int acc = 0;
   for (int base = 0; base < P.B && acc <= beg; base += kThreads) {
-    Walker w{&P};
+    Walker<kGroup> w{&P};
     w.r = base + threadIdx.x;
     int cnt = 0;
     if (w.r < P.B) {
@@ -191,7 +216,7 @@ __device__ void schedule(const Params& P, int* red, int* out /* beg, end, r0, of
       cnt = w.request_items();
     }
     int sum;
-    const int incl = block_scan(cnt, red, &sum);
+    const int incl = block_scan<kThreads>(cnt, red, &sum);
     if (cnt > 0 && beg >= acc + incl - cnt && beg < acc + incl) {
       out[2] = w.r;
       out[3] = beg - (acc + incl - cnt);
@@ -206,11 +231,14 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, ok);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                   const Params P) {
+  constexpr int kStages = C::kStages, kGroup = C::kGroup, kAccBufs = C::kAccBufs, kTmemCols = C::kTmemCols;
+  constexpr int kEpiGroups = C::kEpiGroups, kThreads = C::kThreads;
   extern __shared__ uint8_t smem_raw[];
-  Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem<C>& S = *reinterpret_cast<Smem<C>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -221,8 +249,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&S.qfull[i], 1);
       ptx::mbar_init(&S.qempty[i], 1);
+    }
+    for (int i = 0; i < kAccBufs; ++i) {
       ptx::mbar_init(&S.accfull[i], 1);
-      ptx::mbar_init(&S.accempty[i], 4);
+      ptx::mbar_init(&S.accempty[i], 4);   // the owning warpgroup's 4 warps
     }
     ptx::mbar_init(&S.drain, 1);
     S.abort = 0;
@@ -231,10 +261,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     ptx::prefetch_tensormap(&qmap);
   }
   if (warp == 1) {
-    ptx::tmem_alloc(&S.tmem_base, 2 * kAccCols);
+    ptx::tmem_alloc(&S.tmem_base, kTmemCols);
     ptx::tmem_relinquish();
   }
-  schedule(P, S.red, S.sched);
+  schedule<kThreads, kGroup>(P, S.red, S.sched);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -244,7 +274,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
   if (warp == 0) {
     // ---------------- TMA producer (one lane) ----------------
     if (lane == 0 && beg < end) {
-      Walker w{&P};
+      Walker<kGroup> w{&P};
       w.start(S.sched[2], S.sched[3]);
       int stage = 0;
       uint32_t phase = 0;
@@ -303,7 +333,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
   } else if (warp == 1) {
     // ---------------- MMA issuer (one lane) ----------------
     if (lane == 0 && beg < end) {
-      Walker w{&P};
+      Walker<kGroup> w{&P};
       w.start(S.sched[2], S.sched[3]);
       int stage = 0, acc = 0;
       uint32_t phase = 0, accphase = 0;
@@ -321,7 +351,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         if (!ptx::mbar_wait(&S.full[stage], phase, abort)) { *abort = 1; break; }
         ptx::tc_fence_after();
         const uint32_t idesc = ptx::idesc_m128(SML_INDEX_HEADS * w.qg(), 0);
-        const uint32_t d = S.tmem_base + acc * kAccCols;
+        const uint32_t d = S.tmem_base + acc * C::kAccCols;
         const uint32_t a0 = ptx::smem_u32(S.keys[stage]);
         const uint32_t b0 = ptx::smem_u32(S.q[qb]);
 #pragma unroll
@@ -333,7 +363,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
           stage = 0;
           phase ^= 1;
         }
-        if (++acc == 2) {
+        if (++acc == kAccBufs) {
           acc = 0;
           accphase ^= 1;
         }
@@ -346,28 +376,36 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue: warps 2..5, one thread per token row ----------------
+    // ---------------- epilogue: kEpiGroups warpgroups, one thread per token row ----------------
+    // Warpgroup eg takes the items with ordinal (it - beg) = eg mod kEpiGroups.
+    const int eg = (warp - 2) >> 2;
     const int quarter = warp & 3;               // TMEM lanes 32 * quarter .. + 31
     const int row = quarter * 32 + lane;
-    const int et = threadIdx.x - 64;            // 0..127
-    Walker w{&P};
+    const int et = threadIdx.x - 64 - 128 * eg; // 0..127 within the warpgroup
+    float* wsm = S.w[eg];
+    float* qfs = S.qf[eg];
+    Walker<kGroup> w{&P};
     if (beg < end) w.start(S.sched[2], S.sched[3]);
-    int stage = 0, acc = 0;
-    uint32_t phase = 0, accphase = 0;
     int last_r = -1, last_g = -1;
     for (int it = beg; it < end; ++it, w.advance()) {
+      const int j_it = it - beg;
+      if (j_it % kEpiGroups != eg) continue;
+      const int stage = j_it % kStages, acc = j_it % kAccBufs;
+      const uint32_t phase = (j_it / kStages) & 1, accphase = (j_it / kAccBufs) & 1;
       const int qg = w.qg();
       const int j0 = kGroup * w.g;
       if (w.r != last_r || w.g != last_g) {
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (eg == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
+        else asm volatile("bar.sync 2, 128;" ::: "memory");
         for (int i = et; i < qg * SML_INDEX_HEADS; i += 128)
-          S.w[i] = __ldg(P.iw + (size_t)(w.rq.q0 + j0) * SML_INDEX_HEADS + i);
+          wsm[i] = __ldg(P.iw + (size_t)(w.rq.q0 + j0) * SML_INDEX_HEADS + i);
         if (et < qg) {
           const int n = w.rq.L - w.rq.Q + j0 + et + 1;
           const float c = P.ssmax ? P.s_index * logf((float)n) : 1.f;
-          S.qf[et] = __ldg(P.iq_scale + w.rq.q0 + j0 + et) * c;
+          qfs[et] = __ldg(P.iq_scale + w.rq.q0 + j0 + et) * c;
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (eg == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
+        else asm volatile("bar.sync 2, 128;" ::: "memory");
         last_r = w.r;
         last_g = w.g;
       }
@@ -377,34 +415,27 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
       const float sk = S.ksc[stage][row];
       const bool row_ok = (S.valid[stage] >> (row >> 6)) & 1;
       const int s = w.tile * kTile + row;
-      const uint32_t tbase = S.tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * kAccCols;
+      const uint32_t tbase = S.tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * C::kAccCols;
       for (int j = 0; j < qg; ++j) {
-        float sum = 0.f;
+        uint32_t v0[32], v1[32];
+        ptx::tmem_ld32(tbase + j * SML_INDEX_HEADS, v0);
+        ptx::tmem_ld32(tbase + j * SML_INDEX_HEADS + 32, v1);
+        ptx::tmem_wait_ld();
+        const float* wj = wsm + j * SML_INDEX_HEADS;
+        float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int c = 0; c < SML_INDEX_HEADS / 32; ++c) {
-          uint32_t v[32];
-          ptx::tmem_ld32(tbase + j * SML_INDEX_HEADS + c * 32, v);
-          ptx::tmem_wait_ld();
-          const float* wj = S.w + j * SML_INDEX_HEADS + c * 32;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) sum = fmaf(wj[i], fmaxf(__uint_as_float(v[i]), 0.f), sum);
+        for (int i = 0; i < 32; ++i) {
+          s0 = fmaf(wj[i], fmaxf(__uint_as_float(v0[i]), 0.f), s0);
+          s1 = fmaf(wj[32 + i], fmaxf(__uint_as_float(v1[i]), 0.f), s1);
         }
         const int n = w.rq.L - w.rq.Q + j0 + j + 1;
-        if (row_ok && s < n) P.scores[(size_t)(w.rq.q0 + j0 + j) * P.max_ctx + s] = sum * S.qf[j] * sk;
+        if (row_ok && s < n) P.scores[(size_t)(w.rq.q0 + j0 + j) * P.max_ctx + s] = (s0 + s1) * qfs[j] * sk;
       }
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         ptx::mbar_arrive(&S.accempty[acc]);
         ptx::mbar_arrive(&S.empty[stage]);
-      }
-      if (++stage == kStages) {
-        stage = 0;
-        phase ^= 1;
-      }
-      if (++acc == 2) {
-        acc = 0;
-        accphase ^= 1;
       }
     }
   }
@@ -414,7 +445,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
   if (threadIdx.x == 0 && S.abort) raise_fault(P.status, SML_FAULT_TIMEOUT);
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(S.tmem_base, 2 * kAccCols);
+    ptx::tmem_dealloc(S.tmem_base, kTmemCols);
   }
 }
 
@@ -435,6 +466,15 @@ int num_sms() {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   return n > 0 ? n : 148;
+}
+
+template <class C>
+cudaError_t launch_cfg(const CUtensorMap& kmap, const CUtensorMap& qmap, const Params& P, cudaStream_t stream) {
+  const size_t smem = sizeof(Smem<C>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  indexer_tc_kernel<C><<<num_sms() * C::kCtasPerSm, C::kThreads, smem, stream>>>(kmap, qmap, P);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -483,11 +523,9 @@ cudaError_t launch_indexer(const sml_problem& p, const uint8_t* iq8, const float
   P.index_pages = index_pages;
   P.scores = scores;
   P.status = status;
-  const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  indexer_tc_kernel<<<num_sms(), kThreads, smem, stream>>>(kmap, qmap, P);
-  return cudaGetLastError();
+  // When every request has one query token (T == B) every group is one token.
+  if (p.num_tokens == p.num_requests) return launch_cfg<CfgDecode>(kmap, qmap, P, stream);
+  return launch_cfg<CfgGeneral>(kmap, qmap, P, stream);
 }
 
 }  // namespace sml

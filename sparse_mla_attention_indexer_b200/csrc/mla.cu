@@ -8,24 +8,32 @@
 // their LSE).  For token t, head h over the selected set S_t:
 //   z_i = sm_scale * c_t * (q_nope . c_hat_i + q_pe . k_pe_i)
 //   out = sum_i softmax(z)_i c_hat_i,   lse = ln sum_i exp(z_i)
+// with c_hat_i = e4m3 latent x its 128-element block scale.
 //
 // One CTA = (query token, group of 16 heads, split of up to 512 selected keys),
-// processed in tiles of 128 keys, with the keys as the MMA M dimension and the
-// heads as N (16 heads would waste 3/4 of an M >= 64 tile the other way round):
-//   * warp 5 gathers the selected 656-B rows with one bulk copy per row into a
-//     4-slot ring of 16-row chunks;
-//   * warps 6-9 dequantise each row (E4M3 x its block scale -> fp16; the bf16
-//     RoPE key is copied as is) into a 128-B-swizzled tile C [128 keys x 576];
-//   * warp 4 issues tcgen05.mma kind::f16: S^T[128 x 16] = C . Q^T (nope in
-//     fp16, RoPE part in bf16, one fp32 accumulator), then after the softmax
-//     O_b^T[128 dims x 16] += C_b^T . P^T for the four 128-dim blocks b -- the
-//     same shared tile read K-major for QK^T and MN-major for PV;
-//   * warps 0-3 (one thread per key) run the softmax on S^T: column maxima
-//     through shared memory, a lazily raised running max (O in TMEM is
-//     rescaled only when a head's max grows by more than 8, so P stays below
-//     e^8 in fp16), P in fp16, per-thread partial row sums; at the end they read
-//     O^T back (one thread per latent dim) and write the split's normalised
-//     output and LSE.
+// in tiles of 128 keys; keys are the MMA M dimension and the 16 heads N (an
+// MMA costs at least ~45 cycles whatever its N, and 16 heads as M would waste
+// 3/4 of the smallest M).
+//   * warp 11 gathers the selected 656-B rows, one bulk copy per row, into a
+//     ring of 16-row chunks that holds a whole tile;
+//   * warps 4-5 copy each row's E4M3 latent and bf16 RoPE key into
+//     128-B-swizzled MMA tiles (and the block scales aside);
+//   * warps 6-9 (one thread per latent dim) write V^T into TMEM as fp16
+//     (E4M3 -> fp16 is exact): the A operand of the PV MMA;
+//   * warp 10 issues tcgen05.mma: S_b^T = C_b . Q_b^T per 128-dim block b with
+//     kind::f8f6f4 straight from the E4M3 tile (the bf16 query split exactly
+//     into two E4M3 terms sharing a power-of-two scale per head, so both
+//     accumulate into one fp32 accumulator), the RoPE part with kind::f16
+//     (bf16), and after the softmax O_b^T += V_b^T . P'_b^T;
+//   * warps 0-3 (one thread per key) run the softmax on S^T: z = sm_scale c_t
+//     (sum_b scale_b s_h S_b + S_pe) in fp32, column maxima through shared
+//     memory, a lazily raised running max (O rescaled in TMEM only when a
+//     head's max grows by more than 8), P'_b = fp16(p x scale_b) and per-block
+//     row sums of exactly those weights divided by the scale (so a dominant
+//     key's rounding cancels in the normalisation); at the end they read O^T
+//     back (one thread per latent dim) and write the split's output and LSE.
+// The E4M3 tile is free again as soon as QK^T has read it, so the next tile is
+// staged while this one's softmax and PV run.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -41,23 +49,31 @@ constexpr int kHC = 16;          // heads per CTA (MMA N)
 constexpr int kKT = 128;         // keys per tile (MMA M)
 constexpr int kMaxSplit = 512;   // keys per split (4 tiles)
 constexpr int kChunk = 16;       // rows per gather chunk
-constexpr int kRing = 4;         // gather ring slots
-constexpr int kConvWarps = 4;
-constexpr int kThreads = (6 + kConvWarps) * 32;   // warps 0-3 softmax, 4 MMA, 5 gather, 6.. dequantise
+constexpr int kRing = kKT / kChunk;   // ring slots: one whole tile
+constexpr int kThreads = 384;    // warps 0-3 softmax, 4-5 stage, 6-9 V^T, 10 MMA, 11 gather
+constexpr int kStageWarps = 2;
 constexpr float kLazyRescale = 8.f;   // nats
 
+// TMEM columns
+constexpr uint32_t kColVT = 0;      // V_b^T, fp16 pairs: 64 columns per block b (lanes = dims)
+constexpr uint32_t kColS = 256;     // S_b^T (lanes = keys): 16 columns per block b
+constexpr uint32_t kColSpe = 320;   // S_pe^T
+constexpr uint32_t kColO = 384;     // O_b^T (lanes = dims of block b): 16 columns per block
+constexpr uint32_t kColL = 448;     // per-key row-sum partials of block b (lanes = keys)
+
 struct __align__(1024) Smem {
-  uint8_t c[8][kKT * 128];       // latent sub-tile d: dims [64d, 64d + 64), fp16 E4M3 values, [128 keys x 128 B], SW128
-  uint8_t pe[kKT * 128];         // RoPE key bf16 [128 keys x 64], SW128
-  uint8_t q[8][kHC * 128];       // q nope fp16 sub-tiles [16 heads x 64], SW128
-  uint8_t qpe[kHC * 128];        // q RoPE bf16 [16 heads x 64], SW128
-  uint8_t p[4][kKT * kHC * 2];   // P'_b fp16, MN-major 8x8 core matrices [key/8][head/8][key%8][head%8];
-                                 // p[2..3] double as the softmax exchange buffer
+  uint8_t lat[4][kKT * 128];     // [block b][128 keys x 128 B] E4M3, SW128
+  uint8_t pe[kKT * 128];         // [128 keys x 64 bf16], SW128
+  uint8_t qhi[4][kHC * 128];     // query nope, high E4M3 term [block][16 heads x 128 B], SW128
+  uint8_t qlo[4][kHC * 128];     // low E4M3 term
+  uint8_t qpe[kHC * 128];        // query RoPE bf16 [16 heads x 64], SW128
+  uint8_t p[4][kKT * kHC * 2];   // P'_b fp16, MN-major 8x8 core matrices; p[2..3] double as the exchange buffer
   uint8_t raw[kRing][kChunk * SML_LATENT_ROW_BYTES];
-  float sc[kKT][4];              // block scales of the tile's keys
+  float sc[kKT][4];              // [key][block] scales of the staged tile
+  float qs[kHC];                 // power-of-two query scale per head
   float hstat[kHC];              // per-head tile max / row sum
   int32_t rowid[kMaxSplit];      // pool row (page * 64 + row) of each key, -1 = masked
-  uint64_t q_ready, rows_ready, e_full, s_full, p_full, pv_done, drain;
+  uint64_t q_ready, rows_ready, e_full, e_free, s_full, p_full, vt_full, pv_done, drain;
   uint64_t raw_full[kRing], raw_empty[kRing];
   uint32_t tmem_base;
   int abort;
@@ -87,15 +103,20 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
-  const __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-// Two E4M3 codes (low byte first) -> two fp16 values (exact).
+// Two E4M3 codes (low byte first) -> two fp16 values (exact), packed.
 __device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t two) {
   const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
   return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+// Round two floats to E4M3 (nearest even, saturating); the codes, low byte = a.
+__device__ __forceinline__ uint32_t f2_to_e4m3x2(float a, float b) {
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort) {
@@ -103,14 +124,14 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, ok);
 }
 
-// Softmax exchange: [128 keys][16] floats in the P'_2 / P'_3 buffers, columns
-// XOR-swizzled by key to spread banks.
+// Softmax exchange buffer: [128 keys][16] floats in P'_2 / P'_3, columns
+// XOR-swizzled by key.
 __device__ __forceinline__ float* xbuf(Smem& S, int key, int col) {
   return reinterpret_cast<float*>(S.p[2]) + key * kHC + (col ^ (key & 15));
 }
 
-// Sum (or max) over the 128 keys of 16 per-key values, one call per 16 columns;
-// every softmax thread gets the 16 results in S.hstat.  Threads: warps 0-3.
+// Sum (or max) over the 128 keys of 16 per-key values (warps 0-3); every
+// softmax thread reads the 16 results from S.hstat afterwards.
 template <bool kMax>
 __device__ __forceinline__ void column_reduce(Smem& S, int row, const float (&v)[kHC]) {
 #pragma unroll
@@ -137,7 +158,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, hg = blockIdx.y, t = blockIdx.z;
-  const int Dq = SML_LATENT_DIM + P.rope_dim;
 
   // ---- this split's key range (uniform across the CTA) ----
   const int r = request_of_warp(P.cu_q, P.B, t);
@@ -163,108 +183,93 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
   }
   const int nkeys = ke - kb;
   const int ntiles = (nkeys + kKT - 1) / kKT;
-  const int nchunks = ntiles * (kKT / kChunk);
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&S.q_ready, 4);
-    ptx::mbar_init(&S.rows_ready, kConvWarps);
-    ptx::mbar_init(&S.e_full, kConvWarps);
+    ptx::mbar_init(&S.rows_ready, kStageWarps);
+    ptx::mbar_init(&S.e_full, kStageWarps);
+    ptx::mbar_init(&S.e_free, 1 + 4);     // QK done + softmax warps read the scales
     ptx::mbar_init(&S.s_full, 1);
     ptx::mbar_init(&S.p_full, 4);
+    ptx::mbar_init(&S.vt_full, 4);
     ptx::mbar_init(&S.pv_done, 1);
     ptx::mbar_init(&S.drain, 1);
     for (int i = 0; i < kRing; ++i) {
       ptx::mbar_init(&S.raw_full[i], 1);
-      ptx::mbar_init(&S.raw_empty[i], kConvWarps);
+      ptx::mbar_init(&S.raw_empty[i], kStageWarps + 4);   // stage warps + V^T warps
     }
     S.abort = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 4) {
-    ptx::tmem_alloc(&S.tmem_base, 256);
+  if (warp == 10) {
+    ptx::tmem_alloc(&S.tmem_base, 512);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   volatile int* abort = &S.abort;
-  // TMEM columns: S_b^T (b = 0..3, lanes = keys) at 16 b; S_pe^T at 64;
-  // O_b^T (lanes = dims of block b) at 128 + 16 b; per-key row-sum partials
-  // of block b (lanes = keys) at 192 + 16 b.
-  const uint32_t tS = S.tmem_base, tO = S.tmem_base + 128, tL = S.tmem_base + 192;
+  const uint32_t T0 = S.tmem_base;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
 
-  if (warp >= 6) {
-    // ================= dequantise (kConvWarps warps) =================
-    constexpr int kCT = kConvWarps * 32;
-    constexpr int kRowsPerWarp = kChunk / kConvWarps;
-    const int cw = warp - 6, ct = threadIdx.x - 6 * 32;
-    // Pool rows of the split's keys: all position loads first, then all
-    // block-table loads, so each thread waits for two latencies, not eight.
-    constexpr int kPer = kMaxSplit / kCT;
-    int pos[kPer];
+  if (warp >= 4 && warp < 4 + kStageWarps) {
+    // ================= stage warps: row offsets, then rows -> swizzled tiles =================
+    constexpr int kST = 32 * kStageWarps;
+    const int ct = threadIdx.x - 128;   // 0 .. kST - 1
+    {
+      // Pool rows of the split's keys: all position loads, then all block-table loads.
+      constexpr int kPer = kMaxSplit / kST;
+      int pos[kPer], ph[kPer];
 #pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      const int k = ct + j * kCT;
-      pos[j] = k < nkeys ? __ldg(P.idx + (size_t)t * P.K + kb + k) : -1;
-    }
-    int ph[kPer];
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      const int k = ct + j * kCT;
-      const bool in = k < nkeys && pos[j] >= 0 && pos[j] < n;
-      if (k < nkeys && !in) raise_fault(P.status, SML_FAULT_INDEX);
-      ph[j] = in ? __ldg(P.block_table + (size_t)r * P.max_pages + pos[j] / SML_PAGE_TOKENS) : -1;
-      if (!in) pos[j] = -1;
-    }
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      const int k = ct + j * kCT;
-      int32_t id = -1;
-      if (pos[j] >= 0) {
-        if (ph[j] >= 0 && ph[j] < P.latent_pages)
-          id = ph[j] * SML_PAGE_TOKENS + pos[j] % SML_PAGE_TOKENS;
-        else
-          raise_fault(P.status, SML_FAULT_PAGE);
+      for (int j = 0; j < kPer; ++j) {
+        const int k = ct + j * kST;
+        pos[j] = k < nkeys ? __ldg(P.idx + (size_t)t * P.K + kb + k) : -1;
       }
-      S.rowid[k] = id;
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int k = ct + j * kST;
+        const bool in = k < nkeys && pos[j] >= 0 && pos[j] < n;
+        if (k < nkeys && !in) raise_fault(P.status, SML_FAULT_INDEX);
+        ph[j] = in ? __ldg(P.block_table + (size_t)r * P.max_pages + pos[j] / SML_PAGE_TOKENS) : -1;
+        if (!in) pos[j] = -1;
+      }
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        int32_t id = -1;
+        if (pos[j] >= 0) {
+          if (ph[j] >= 0 && ph[j] < P.latent_pages)
+            id = ph[j] * SML_PAGE_TOKENS + pos[j] % SML_PAGE_TOKENS;
+          else
+            raise_fault(P.status, SML_FAULT_PAGE);
+        }
+        S.rowid[ct + j * kST] = id;
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&S.rows_ready);
     }
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(&S.rows_ready);
-
+    // Rows -> tiles: stage warp w takes rows kRowsPerWarp w .. of each chunk.
+    constexpr int kRowsPerWarp = kChunk / kStageWarps;
+    const int sw = warp - 4;
     int chunk = 0;
     for (int tile = 0; tile < ntiles; ++tile) {
-      if (tile > 0 && !warp_wait(&S.pv_done, (tile - 1) & 1, abort)) { *abort = 1; break; }
+      if (tile > 0 && !warp_wait(&S.e_free, (tile - 1) & 1, abort)) { *abort = 1; break; }
       bool ok = true;
-      for (int cc = 0; cc < kKT / kChunk; ++cc, ++chunk) {
+      for (int cc = 0; cc < kRing; ++cc, ++chunk) {
         const int slot = chunk % kRing;
         if (!warp_wait(&S.raw_full[slot], (chunk / kRing) & 1, abort)) { ok = false; break; }
+#pragma unroll
         for (int rr = 0; rr < kRowsPerWarp; ++rr) {
-          const int j = cw * kRowsPerWarp + rr;      // row within the chunk
-          const int row = cc * kChunk + j;           // row within the tile
+          const int j = kRowsPerWarp * sw + rr; // row within the chunk
+          const int row = cc * kChunk + j;      // row within the tile
           const bool valid = S.rowid[tile * kKT + row] >= 0;
           const uint8_t* src = S.raw[slot] + j * SML_LATENT_ROW_BYTES;
-          // latent: lane l holds dims [16 l, 16 l + 16) as exact fp16 E4M3 values
-          uint32_t o[8];
-          if (valid) {
-            const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * lane);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              o[2 * i] = e4m3x2_to_h2(w[i] & 0xffffu);
-              o[2 * i + 1] = e4m3x2_to_h2(w[i] >> 16);
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = 0u;
-          }
-          const int d = lane >> 2, ch = (lane & 3) * 2;
-          const uint32_t tb = ptx::smem_u32(S.c[d]);
-          st_shared_v4(sw128(tb, row, ch), o[0], o[1], o[2], o[3]);
-          st_shared_v4(sw128(tb, row, ch + 1), o[4], o[5], o[6], o[7]);
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (valid) v = *reinterpret_cast<const uint4*>(src + 16 * lane);
+          st_shared_v4(sw128(ptx::smem_u32(S.lat[lane >> 3]), row, lane & 7), v.x, v.y, v.z, v.w);
           if (lane < 8) {
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (valid && P.rope_dim) v = *reinterpret_cast<const uint4*>(src + SML_LATENT_DIM + 16 + 16 * lane);
-            st_shared_v4(sw128(ptx::smem_u32(S.pe), row, lane), v.x, v.y, v.z, v.w);
+            uint4 e = make_uint4(0u, 0u, 0u, 0u);
+            if (valid && P.rope_dim) e = *reinterpret_cast<const uint4*>(src + SML_LATENT_DIM + 16 + 16 * lane);
+            st_shared_v4(sw128(ptx::smem_u32(S.pe), row, lane), e.x, e.y, e.z, e.w);
           } else if (lane < 12) {
             S.sc[row][lane - 8] = valid ? reinterpret_cast<const float*>(src + SML_LATENT_DIM)[lane - 8] : 1.f;
           }
@@ -277,10 +282,46 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&S.e_full);
     }
-  } else if (warp == 5) {
+  } else if (warp >= 4 + kStageWarps && warp < 8 + kStageWarps) {
+    // ================= V^T warps: one thread per latent dim of every block =================
+    const int d = (warp & 3) * 32 + lane;   // = TMEM lane (a warp reaches lanes 32 (warp % 4) ..)
+    int chunk = 0;
+    for (int tile = 0; tile < ntiles; ++tile) {
+      if (tile > 0 && !warp_wait(&S.pv_done, (tile - 1) & 1, abort)) { *abort = 1; break; }
+      ptx::tc_fence_after();
+      bool ok = true;
+      for (int cc = 0; cc < kRing; ++cc, ++chunk) {
+        const int slot = chunk % kRing;
+        if (!warp_wait(&S.raw_full[slot], (chunk / kRing) & 1, abort)) { ok = false; break; }
+        const uint8_t* src = S.raw[slot];
+        uint32_t vb[4][8];
+#pragma unroll
+        for (int jp = 0; jp < kChunk / 2; ++jp) {   // key pairs of the chunk
+          const int k0 = cc * kChunk + 2 * jp;
+          const bool v0 = S.rowid[tile * kKT + k0] >= 0, v1 = S.rowid[tile * kKT + k0 + 1] >= 0;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const uint32_t lo8 = v0 ? src[(2 * jp) * SML_LATENT_ROW_BYTES + 128 * b + d] : 0u;
+            const uint32_t hi8 = v1 ? src[(2 * jp + 1) * SML_LATENT_ROW_BYTES + 128 * b + d] : 0u;
+            vb[b][jp] = e4m3x2_to_h2(lo8 | (hi8 << 8));
+          }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&S.raw_empty[slot]);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) ptx::tmem_st8(T0 + kColVT + 64 * b + 8 * cc + lane_off, vb[b]);
+      }
+      if (!ok) { *abort = 1; break; }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&S.vt_full);
+    }
+  } else if (warp == 11) {
     // ================= gather: one bulk copy per selected row =================
     if (lane == 0) {
       bool ok = ptx::mbar_wait(&S.rows_ready, 0, abort);
+      const int nchunks = ntiles * kRing;
       int chunk = 0;
       for (; ok && chunk < nchunks; ++chunk) {
         const int slot = chunk % kRing;
@@ -303,45 +344,44 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
       }
     }
     __syncwarp();
-  } else if (warp == 4) {
+  } else if (warp == 10) {
     // ================= MMA issuer =================
     if (lane == 0) {
       bool ok = ptx::mbar_wait(&S.q_ready, 0, abort);
-      const uint32_t id_qk = ptx::idesc_f16(kHC, 0, 0, 0);   // f16, K-major A and B
-      const uint32_t id_pe = ptx::idesc_f16(kHC, 1, 0, 0);   // bf16
-      const uint32_t id_pv = ptx::idesc_f16(kHC, 0, 1, 1);   // f16, MN-major A (C_b^T) and B (P'_b^T)
+      const uint32_t id_qk = ptx::idesc_m128(kHC, 0);         // E4M3 x E4M3, K-major
+      const uint32_t id_pe = ptx::idesc_f16(kHC, 1, 0, 0);    // bf16
+      const uint32_t id_pv = ptx::idesc_f16(kHC, 0, 0, 1);    // f16; A (TMEM) K-major, B MN-major
       for (int tile = 0; ok && tile < ntiles; ++tile) {
         if (!ptx::mbar_wait(&S.e_full, tile & 1, abort)) { ok = false; break; }
         ptx::tc_fence_after();
-        // S_b^T = C_b . Q_b^T, one accumulator per 128-dim scale block b
-        // (2 sub-tiles x 4 steps of 16 dims each) ...
-        for (int d = 0; d < 8; ++d) {
-          const uint32_t a = ptx::smem_u32(S.c[d]), b = ptx::smem_u32(S.q[d]);
+        // S_b^T = C_b . (Qhi_b + Qlo_b)^T: four accumulators, 32 dims per step, interleaved
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            ptx::mma_f16_ss(tS + 16 * (d >> 1), ptx::sdesc(a + 32 * k, 16, 1024, 2),
-                            ptx::sdesc(b + 32 * k, 16, 1024, 2), id_qk, ((d & 1) | k) != 0);
-        }
-        // ... and the RoPE part (bf16) in its own accumulator.
-        if (P.rope_dim) {
-          const uint32_t a = ptx::smem_u32(S.pe), b = ptx::smem_u32(S.qpe);
+        for (int k = 0; k < 4; ++k) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            ptx::mma_f16_ss(tS + 64, ptx::sdesc(a + 32 * k, 16, 1024, 2), ptx::sdesc(b + 32 * k, 16, 1024, 2), id_pe,
-                            k != 0);
+          for (int b = 0; b < 4; ++b) {
+            const uint64_t a = ptx::sdesc_sw128(ptx::smem_u32(S.lat[b]) + 32 * k);
+            ptx::mma_f8f6f4_ss(T0 + kColS + 16 * b, a, ptx::sdesc_sw128(ptx::smem_u32(S.qhi[b]) + 32 * k), id_qk, k > 0);
+            ptx::mma_f8f6f4_ss(T0 + kColS + 16 * b, a, ptx::sdesc_sw128(ptx::smem_u32(S.qlo[b]) + 32 * k), id_qk, 1);
+          }
+          if (P.rope_dim)
+            ptx::mma_f16_ss(T0 + kColSpe, ptx::sdesc_sw128(ptx::smem_u32(S.pe) + 32 * k),
+                            ptx::sdesc_sw128(ptx::smem_u32(S.qpe) + 32 * k), id_pe, k > 0);
         }
         ptx::mma_commit(&S.s_full);
-        if (!ptx::mbar_wait(&S.p_full, tile & 1, abort)) { ok = false; break; }
+        ptx::mma_commit(&S.e_free);
+        if (!ptx::mbar_wait(&S.p_full, tile & 1, abort) || !ptx::mbar_wait(&S.vt_full, tile & 1, abort)) {
+          ok = false;
+          break;
+        }
         ptx::tc_fence_after();
-        // O_b^T += C_b^T . P'_b^T: A = dims [128 b, 128 b + 128) of the tile read MN-major
-        // (64-dim blocks 16 KB apart, 8-key groups 1 KB apart); B = P'_b^T, MN-major core
-        // matrices (8-head blocks 128 B apart, 8-key groups 256 B apart).
-        for (int b = 0; b < 4; ++b) {
-          const uint32_t a = ptx::smem_u32(S.c[2 * b]), pb = ptx::smem_u32(S.p[b]);
+        // O_b^T += V_b^T . P'_b^T: A = V_b^T in TMEM (16 keys = 8 columns per step);
+        // B = P'_b^T, MN-major core matrices (8-head blocks 128 B apart, 8-key groups 256 B apart).
 #pragma unroll
-          for (int k = 0; k < kKT / 16; ++k)
-            ptx::mma_f16_ss(tO + 16 * b, ptx::sdesc(a + 2048 * k, 16384, 1024, 2),
-                            ptx::sdesc(pb + 512 * k, 256, 128, 0), id_pv, (tile | k) != 0);
+        for (int k = 0; k < kKT / 16; ++k) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b)
+            ptx::mma_f16_ts(T0 + kColO + 16 * b, T0 + kColVT + 64 * b + 8 * k,
+                            ptx::sdesc(ptx::smem_u32(S.p[b]) + 512 * k, 256, 128, 0), id_pv, (tile | k) != 0);
         }
         ptx::mma_commit(&S.pv_done);
       }
@@ -354,46 +394,97 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
     // ================= softmax: warps 0-3, thread = key row / latent dim =================
     const int row = warp * 32 + lane;
     {
-      // Query heads of this group, while the other warps resolve the key rows:
-      // nope bf16 -> fp16 (exact in fp16's normal range), RoPE part copied as bf16.
-      const uint16_t* qbase = P.q + ((size_t)t * P.H + hg * kHC) * Dq;
-      for (int e = row; e < kHC * (Dq / 8); e += 128) {
-        const int h = e / (Dq / 8), c8 = e % (Dq / 8);    // 8 elements = one 16-B chunk
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(qbase + (size_t)h * Dq) + c8);
-        if (c8 < 64) {
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-          uint32_t o[4];
+      // Query of the 16 heads.  Nope part: q = s_h (hi + lo), hi and lo E4M3 and
+      // s_h a power of two >= amax_h / 448, so q / s_h, its rounding to hi and
+      // the residual lo are exact in fp32, and lo is exact in E4M3 (a bf16 has
+      // 8 significant bits, hi takes 4, the residual the other 4) down to
+      // E4M3's subnormal step.  RoPE part copied as bf16.
+      const int Dq = SML_LATENT_DIM + P.rope_dim;
+      const int h = row >> 3, part = row & 7;   // 8 threads per head, 64 nope dims each
+      const uint16_t* qh = P.q + ((size_t)t * P.H + hg * kHC + h) * Dq;
+      uint4 v[8];
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            o[i] = pack_half2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
-          st_shared_v4(sw128(ptx::smem_u32(S.q[c8 >> 3]), h, c8 & 7), o[0], o[1], o[2], o[3]);
-        } else {
-          st_shared_v4(sw128(ptx::smem_u32(S.qpe), h, c8 - 64), v.x, v.y, v.z, v.w);
-        }
+      for (int i = 0; i < 8; ++i) v[i] = __ldg(reinterpret_cast<const uint4*>(qh + 64 * part) + i);
+      uint4 pv = make_uint4(0u, 0u, 0u, 0u);
+      if (P.rope_dim) pv = __ldg(reinterpret_cast<const uint4*>(qh + SML_LATENT_DIM) + part);   // 8 bf16
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[k] << 16)), fabsf(__uint_as_float(w[k] & 0xffff0000u))));
       }
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+      int e2 = 0;
+      if (amax > 0.f) frexpf(amax / 448.f, &e2);        // amax / 448 < 2^e2
+      const float qscale = ldexpf(1.f, e2), inv = ldexpf(1.f, -e2);
+      if (part == 0) S.qs[h] = qscale;
+      // dims [64 part, 64 part + 64) -> block part / 2, 16-B chunks 4 (part % 2) + c
+      const int b = part >> 1;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          // elements 16 c + 4 k .. + 3 of this thread's 64
+          const uint4 vv = v[2 * c + (k >> 1)];
+          const uint32_t wa = (k & 1) ? vv.z : vv.x, wb = (k & 1) ? vv.w : vv.y;
+          const float x0 = __uint_as_float(wa << 16) * inv, x1 = __uint_as_float(wa & 0xffff0000u) * inv;
+          const float x2 = __uint_as_float(wb << 16) * inv, x3 = __uint_as_float(wb & 0xffff0000u) * inv;
+          const uint32_t h01 = f2_to_e4m3x2(x0, x1), h23 = f2_to_e4m3x2(x2, x3);
+          const float2 r01 = e4m3x2_to_f2(h01), r23 = e4m3x2_to_f2(h23);
+          const uint32_t l01 = f2_to_e4m3x2(x0 - r01.x, x1 - r01.y), l23 = f2_to_e4m3x2(x2 - r23.x, x3 - r23.y);
+          hw[k] = (h01 & 0xffffu) | (h23 << 16);
+          lw[k] = (l01 & 0xffffu) | (l23 << 16);
+        }
+        const int chunk = 4 * (part & 1) + c;
+        st_shared_v4(sw128(ptx::smem_u32(S.qhi[b]), h, chunk), hw[0], hw[1], hw[2], hw[3]);
+        st_shared_v4(sw128(ptx::smem_u32(S.qlo[b]), h, chunk), lw[0], lw[1], lw[2], lw[3]);
+      }
+      st_shared_v4(sw128(ptx::smem_u32(S.qpe), h, part), pv.x, pv.y, pv.z, pv.w);
       ptx::fence_proxy_async();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&S.q_ready);
     }
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const float zscale = P.sm_scale * (P.ssmax ? P.ssmax_s * logf((float)max(n, 1)) : 1.f);
     float m[kHC];
 #pragma unroll
     for (int h = 0; h < kHC; ++h) m[h] = -INFINITY;
-    bool ok = true;
-    for (int tile = 0; tile < ntiles; ++tile) {
-      if (!warp_wait(&S.s_full, tile & 1, abort)) { ok = false; break; }
+    bool ok = warp_wait(&S.q_ready, 0, abort);   // S.qs
+    float qs[kHC];
+#pragma unroll
+    for (int h = 0; h < kHC; ++h) qs[h] = S.qs[h];
+    for (int tile = 0; ok && tile < ntiles; ++tile) {
+      if (!warp_wait(&S.e_full, tile & 1, abort) || !warp_wait(&S.s_full, tile & 1, abort)) {
+        ok = false;
+        break;
+      }
       ptx::tc_fence_after();
       const bool valid = S.rowid[tile * kKT + row] >= 0;
       float sc[4];
 #pragma unroll
       for (int b = 0; b < 4; ++b) sc[b] = S.sc[row][b];
-      // z = zscale * (sum_b scale_b * S_b + S_pe), fp32
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&S.e_free);   // scales read
+      // z = zscale * (sum_b scale_b * s_h * S_b + S_pe), fp32
       float z[kHC];
       {
         uint32_t v[16];
+        float acc[kHC];
+#pragma unroll
+        for (int h = 0; h < kHC; ++h) acc[h] = 0.f;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          ptx::tmem_ld16(T0 + kColS + 16 * b + lane_off, v);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < kHC; ++h) acc[h] = fmaf(sc[b], __uint_as_float(v[h]), acc[h]);
+        }
         if (P.rope_dim) {
-          ptx::tmem_ld16(tS + 64 + lane_off, v);
+          ptx::tmem_ld16(T0 + kColSpe + lane_off, v);
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int h = 0; h < kHC; ++h) z[h] = __uint_as_float(v[h]);
@@ -402,15 +493,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
           for (int h = 0; h < kHC; ++h) z[h] = 0.f;
         }
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          ptx::tmem_ld16(tS + 16 * b + lane_off, v);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < kHC; ++h) z[h] = fmaf(sc[b], __uint_as_float(v[h]), z[h]);
-        }
+        for (int h = 0; h < kHC; ++h) z[h] = valid ? fmaf(acc[h], qs[h], z[h]) * zscale : -INFINITY;
       }
-#pragma unroll
-      for (int h = 0; h < kHC; ++h) z[h] = valid ? z[h] * zscale : -INFINITY;
       column_reduce<true>(S, row, z);
       // lazily raised running max; rescale O and the row-sum partials when it moves
       float alpha[kHC];
@@ -429,30 +513,29 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
           uint32_t ov[16];
-          ptx::tmem_ld16(tO + 16 * b + lane_off, ov);    // this thread: latent dim 128 b + row
+          ptx::tmem_ld16(T0 + kColO + 16 * b + lane_off, ov);    // this thread: latent dim 128 b + row
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int h = 0; h < kHC; ++h) ov[h] = __float_as_uint(__uint_as_float(ov[h]) * alpha[h]);
-          ptx::tmem_st16(tO + 16 * b + lane_off, ov);
-          ptx::tmem_ld16(tL + 16 * b + lane_off, ov);    // this thread: key row's partials
+          ptx::tmem_st16(T0 + kColO + 16 * b + lane_off, ov);
+          ptx::tmem_ld16(T0 + kColL + 16 * b + lane_off, ov);    // this thread: key row's partials
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int h = 0; h < kHC; ++h) ov[h] = __float_as_uint(__uint_as_float(ov[h]) * alpha[h]);
-          ptx::tmem_st16(tL + 16 * b + lane_off, ov);
+          ptx::tmem_st16(T0 + kColL + 16 * b + lane_off, ov);
         }
         ptx::tmem_wait_st();
       }
       float p[kHC];
 #pragma unroll
       for (int h = 0; h < kHC; ++h) p[h] = z[h] == -INFINITY ? 0.f : expf(z[h] - m[h]);
-      // P'_b = fp16(p * scale_b); row-sum partial of block b += P'_b / scale_b, so a
-      // block's normalisation uses exactly the weights its MMA used.
+      // P'_b = fp16(p * scale_b); row-sum partial of block b += P'_b / scale_b
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
         uint32_t lv[16], pw[8];
         const float inv_sc = sc[b] > 0.f ? 1.f / sc[b] : 0.f;   // an all-zero block has scale 0
         if (tile > 0) {
-          ptx::tmem_ld16(tL + 16 * b + lane_off, lv);
+          ptx::tmem_ld16(T0 + kColL + 16 * b + lane_off, lv);
           ptx::tmem_wait_ld();
         } else {
 #pragma unroll
@@ -468,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
           lv[h + 1] = __float_as_uint(__uint_as_float(lv[h + 1]) + w1);
           pw[h >> 1] = *reinterpret_cast<const uint32_t*>(&ph);
         }
-        ptx::tmem_st16(tL + 16 * b + lane_off, lv);
+        ptx::tmem_st16(T0 + kColL + 16 * b + lane_off, lv);
         const uint32_t pb = ptx::smem_u32(S.p[b]) + (row >> 3) * 256 + (row & 7) * 16;
         st_shared_v4(pb, pw[0], pw[1], pw[2], pw[3]);          // heads 0-7
         st_shared_v4(pb + 128, pw[4], pw[5], pw[6], pw[7]);    // heads 8-15
@@ -487,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
       uint32_t lv[16];
-      ptx::tmem_ld16(tL + 16 * b + lane_off, lv);
+      ptx::tmem_ld16(T0 + kColL + 16 * b + lane_off, lv);
       ptx::tmem_wait_ld();
       float lf[kHC];
 #pragma unroll
@@ -501,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
         if (b == 0) lsum0[h] = ls;
       }
       uint32_t ov[16];
-      ptx::tmem_ld16(tO + 16 * b + lane_off, ov);
+      ptx::tmem_ld16(T0 + kColO + 16 * b + lane_off, ov);
       ptx::tmem_wait_ld();
       const int dim = 128 * b + row;
 #pragma unroll
@@ -523,9 +606,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
   ptx::tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && S.abort) raise_fault(P.status, SML_FAULT_TIMEOUT);
-  if (warp == 4) {
+  if (warp == 10) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(S.tmem_base, 256);
+    ptx::tmem_dealloc(S.tmem_base, 512);
   }
 }
 
@@ -565,7 +648,7 @@ lse_merge_kernel(int H, MlaWs ws, float* __restrict__ out, float* __restrict__ l
 int mla_splits(const sml_problem& p, int* keys_per_split) {
   // Splits of whole 128-key tiles, at most 512 keys: about one CTA per SM for
   // the whole problem, so the per-CTA set-up is paid once per SM and the
-  // gather of a tile overlaps the math of the one before.
+  // staging of a tile overlaps the math of the one before.
   const int tiles = (p.topk + kKT - 1) / kKT;
   const int ctas = p.num_tokens * (p.num_heads / kHC);
   int tps = (int)(((long long)ctas * tiles + 148 - 1) / 148);
@@ -580,6 +663,7 @@ cudaError_t launch_sparse_mla(const sml_problem& p, const uint16_t* q, const uin
                               int64_t latent_pages, const int32_t* idx, const int32_t* idx_len,
                               float* out, float* lse, const MlaWs& ws, int32_t* status,
                               cudaStream_t stream) {
+  if (latent_pages > (int64_t)(INT32_MAX / SML_PAGE_TOKENS)) return cudaErrorInvalidValue;
   Params P;
   P.B = p.num_requests;
   P.T = p.num_tokens;

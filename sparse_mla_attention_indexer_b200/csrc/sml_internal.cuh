@@ -26,7 +26,7 @@ inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // shared memory; longer rows are cut into chunks whose candidates the last
 // arriving CTA of the row merges.
 constexpr int kTopkChunk = 16384;
-constexpr int kTopkThreads = 1024;
+constexpr int kTopkThreads = 512;
 
 struct TopkWs {
   int32_t* counters;   // [T] arrival counters, zero between calls

@@ -6,10 +6,11 @@
 // replaced.  This is a single-GPU select written for sm_100a:
 //
 //  * scores become order-preserving 32-bit keys (-0 -> +0, NaN lowest);
-//  * one pass histograms the values into 2,048 buckets linear in value between
-//    the row's finite min and max (-inf / NaN in the lowest bucket, +inf in the
-//    highest), which spreads the bins for shared-memory atomics and finds the
-//    bucket that holds the k-th largest value;
+//  * a 1,024-key sample places a floor below the k-th largest value; one pass
+//    histograms the values at or above it into 2,048 buckets linear in value
+//    up to the row's maximum (so the shared-memory atomics touch about k values
+//    and spread over the bins) and finds the bucket that holds the k-th
+//    largest value; if the sample misjudged, the pass covers every value;
 //  * only that bucket's keys (a handful, typically) go through an exact radix
 //    select (11 / 11 / 10 key bits) to find the k-th largest key tau and how
 //    many keys equal to tau are taken; a row whose threshold bucket is huge
@@ -29,6 +30,8 @@ namespace {
 
 constexpr int kBuckets = 2048;
 constexpr int kCandCap = 4096;
+constexpr int kSmallCand = 256;   // threshold by direct rank counting up to this many candidates
+constexpr int kSample = 1024;     // keys sampled to place the histogram floor
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t b = __float_as_uint(f);
@@ -49,6 +52,8 @@ struct SelectShared {
   float red_lo[32], red_hi[32];
   int ncand;
   int bcast[2];
+  uint32_t bcast_tau;
+  float bcast_f;
 };
 
 // Inclusive block-wide scan of one int per thread; *total gets the block sum.
@@ -109,11 +114,10 @@ __device__ void radix_threshold(int n, int k, KeyAt key_at, SelectShared& sh, ui
   const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
   uint32_t prefix = 0, pmask = 0;
   int remaining = k;
-  const int shifts[3] = {21, 10, 0};
-  const int widths[3] = {11, 11, 10};
+#pragma unroll
   for (int pass = 0; pass < 3; ++pass) {
-    const int shift = shifts[pass];
-    const int nb = 1 << widths[pass];
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);   // 11 / 11 / 10 key bits
+    const int nb = pass == 2 ? 1024 : 2048;
     for (int b = tid; b < nb; b += nt) sh.hist[b] = 0;
     __syncthreads();
     for (int base = 0; base < n; base += nt) {
@@ -137,6 +141,35 @@ __device__ void radix_threshold(int n, int k, KeyAt key_at, SelectShared& sh, ui
   *take = remaining;
 }
 
+// Warp 0 only: over sh.hist[0, kBuckets), the bucket holding the `need`-th
+// largest element and the count above it, into sh.bcast.
+__device__ __forceinline__ void find_bucket_warp(int need, SelectShared& sh) {
+  const int lane = threadIdx.x & 31;
+  constexpr int kPer = kBuckets / 32;           // lane l owns buckets [top - kPer l, ...) descending
+  const int top = kBuckets - 1 - lane * kPer;
+  int local = 0;
+  for (int j = 0; j < kPer; ++j) local += sh.hist[top - j];
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int before = incl - local;
+  if (before < need && need <= incl) {
+    int above = before;
+    for (int j = 0; j < kPer; ++j) {
+      const int h = sh.hist[top - j];
+      if (need <= above + h) {
+        sh.bcast[0] = top - j;
+        sh.bcast[1] = above;
+        break;
+      }
+      above += h;
+    }
+  }
+}
+
 // Select the k largest of n keys (key_at(i), i in [0, n)); call emit(pos, i)
 // for each selected i, pos = its rank in ascending i order.  All threads of the
 // block call it; blockDim.x == kTopkThreads.
@@ -149,6 +182,7 @@ __device__ void select_topk(int n, int k, KeyAt key_at, Emit emit, SelectShared&
   }
   // 1. finite range of the values
   float lo = INFINITY, hi = -INFINITY;
+#pragma unroll 4
   for (int i = tid; i < n; i += nt) {
     const float v = key_value(key_at(i));
     if (isfinite(v)) {
@@ -174,22 +208,97 @@ __device__ void select_topk(int n, int k, KeyAt key_at, Emit emit, SelectShared&
     lo = fminf(lo, sh.red_lo[w]);
     hi = fmaxf(hi, sh.red_hi[w]);
   }
-  // 2. value-linear buckets: 0 = NaN / -inf, 1 .. kBuckets-2 finite, top = +inf.
-  // A range too wide for fp32 gives scale 0: every finite value in bucket 1.
+  // 2. A floor below which fewer than k values can lie above: a sample of
+  // kSample evenly spaced keys, histogrammed into 256 value bins, gives the bin
+  // holding its k * kSample / n-th largest key, plus a 4-sigma margin.  Only
+  // values at or above the floor go into the fine histogram, so its atomics
+  // touch about k values instead of n.  If the sample misjudged (fewer than k
+  // values at or above the floor) every value is histogrammed instead.
   const float width = hi - lo;
-  const float scale = (hi > lo && width < INFINITY) ? (float)(kBuckets - 3) / width : 0.f;
+  const bool finite_range = hi > lo && width < INFINITY;
+  float floor_v = -INFINITY;
+  if (finite_range && n > 2 * k) {
+    const int stride = n / kSample;
+    for (int b = tid; b < 256; b += nt) sh.hist[b] = 0;
+    __syncthreads();
+    const float cscale = 254.f / width;
+    for (int j = tid; j < kSample; j += nt) {
+      const float v = key_value(key_at(j * stride));
+      const int cb = !(v > -INFINITY) ? 0 : (v == INFINITY ? 255 : 1 + (int)fminf(fmaxf((v - lo) * cscale, 0.f), 253.f));
+      atomicAdd(&sh.hist[cb], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const float mu = (float)k * kSample / (float)n;
+      const int need_s = min(kSample, (int)ceilf(mu + 4.f * sqrtf(mu) + 4.f));
+      // 8 coarse bins per lane, descending
+      const int top = 255 - 8 * lane;
+      int local = 0;
+      for (int j = 0; j < 8; ++j) local += sh.hist[top - j];
+      int incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int above = incl - local;
+      if (above < need_s && need_s <= incl) {
+        for (int j = 0; j < 8; ++j) {
+          above += sh.hist[top - j];
+          if (need_s <= above) {
+            const int cb = top - j;   // coarse bin 1..254 covers [lo + (cb-1)/cscale, ...)
+            sh.bcast_f = cb <= 1 ? -INFINITY : lo + (float)(cb - 1) / cscale;
+            break;
+          }
+        }
+      }
+      if (lane == 0 && incl < need_s) sh.bcast_f = -INFINITY;   // unreachable: all samples counted
+    }
+    __syncthreads();
+    floor_v = sh.bcast_f;
+  }
+  // Fine buckets: 0 = NaN / -inf (full mode only), 1 .. kBuckets-2 finite, top = +inf;
+  // -1 = below the floor.
+  int full = !(floor_v > -INFINITY);
+  float base_v = full ? lo : floor_v;
+  float scale = finite_range && hi > base_v ? (float)(kBuckets - 3) / (hi - base_v) : 0.f;
   auto bucket = [&](uint32_t key) -> int {
     const float v = key_value(key);
-    if (!(v > -INFINITY)) return 0;                               // NaN or -inf
     if (v == INFINITY) return kBuckets - 1;
-    const float x = fminf(fmaxf((v - lo) * scale, 0.f), (float)(kBuckets - 3));   // monotone in v
+    if (!full && !(v >= base_v)) return -1;
+    if (!(v > -INFINITY)) return 0;                               // NaN or -inf
+    const float x = fminf(fmaxf((v - base_v) * scale, 0.f), (float)(kBuckets - 3));   // monotone in v
     return 1 + (int)x;
   };
-  for (int i = tid; i < n; i += nt) atomicAdd(&sh.hist[bucket(key_at(i))], 1);
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    for (int b = tid; b < kBuckets; b += nt) sh.hist[b] = 0;
+    __syncthreads();
+    int counted = 0;
+#pragma unroll 4
+    for (int i = tid; i < n; i += nt) {
+      const int b = bucket(key_at(i));
+      if (b >= 0) {
+        atomicAdd(&sh.hist[b], 1);
+        ++counted;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) counted += __shfl_xor_sync(0xffffffffu, counted, o);
+    if (lane == 0) sh.warp_a[warp] = counted;
+    __syncthreads();
+    int total = 0;
+    for (int w = 0; w < nt / 32; ++w) total += sh.warp_a[w];
+    if (full || total >= k) break;   // uniform across the block
+    full = 1;                        // the sample misjudged: histogram every value
+    base_v = lo;
+    scale = finite_range ? (float)(kBuckets - 3) / width : 0.f;
+    __syncthreads();
+  }
+  if (warp == 0) find_bucket_warp(k, sh);
   __syncthreads();
-  int bk, above;
-  find_bin(kBuckets, k, sh, &bk, &above);
+  const int bk = sh.bcast[0], above = sh.bcast[1];
   // 3. the keys of the threshold bucket
+#pragma unroll 4
   for (int i = tid; i < n; i += nt) {
     const uint32_t key = key_at(i);
     if (bucket(key) == bk) {
@@ -199,10 +308,30 @@ __device__ void select_topk(int n, int k, KeyAt key_at, Emit emit, SelectShared&
   }
   __syncthreads();
   const int nc = sh.ncand;
+  const int need = k - above;   // 1 <= need <= nc
   uint32_t tau;
   int take;
-  if (nc <= kCandCap) {
-    radix_threshold(nc, k - above, [&](int i) { return sh.cand[i]; }, sh, &tau, &take);
+  if (nc <= kSmallCand) {
+    // tau = the candidate with fewer than `need` candidates above it and at
+    // least `need` at or above it; every thread holding that key agrees.
+    if (tid < nc) {
+      const uint32_t key = sh.cand[tid];
+      int gt = 0, ge = 0;
+      for (int j = 0; j < nc; ++j) {
+        const uint32_t c = sh.cand[j];
+        gt += c > key;
+        ge += c >= key;
+      }
+      if (gt < need && need <= ge) {
+        sh.bcast_tau = key;
+        sh.bcast[1] = need - gt;
+      }
+    }
+    __syncthreads();
+    tau = sh.bcast_tau;
+    take = sh.bcast[1];
+  } else if (nc <= kCandCap) {
+    radix_threshold(nc, need, [&](int i) { return sh.cand[i]; }, sh, &tau, &take);
   } else {
     radix_threshold(n, k, key_at, sh, &tau, &take);   // heavy ties: over every key
   }
@@ -282,6 +411,7 @@ topk_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32_t* __re
   const int c0 = c * kTopkChunk;
   const int cn = min(kTopkChunk, n - c0);
   const float* row = scores + (size_t)t * max_ctx + c0;
+#pragma unroll 32
   for (int i = tid; i < cn; i += nt) skeys[i] = order_key(__ldcg(row + i));
   __syncthreads();
   auto smem_key = [&](int i) { return skeys[i]; };
@@ -316,6 +446,7 @@ topk_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32_t* __re
   const uint32_t* tk = ws.cand_key + row_base;
   const int32_t* ti = ws.cand_idx + row_base;
   if (total <= kTopkChunk) {
+#pragma unroll 16
     for (int i = tid; i < total; i += nt) skeys[i] = __ldcg(tk + i);
     __syncthreads();
     select_topk(total, K, smem_key, [&](int pos, int i) { out[pos] = __ldcg(ti + i); }, sh);
