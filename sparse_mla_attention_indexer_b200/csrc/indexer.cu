@@ -420,7 +420,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         uint32_t v0[32], v1[32];
         ptx::tmem_ld32(tbase + j * SML_INDEX_HEADS, v0);
         ptx::tmem_ld32(tbase + j * SML_INDEX_HEADS + 32, v1);
-        ptx::tmem_wait_ld();
+        ptx::tmem_wait_ld(v0, v1);
         const float* wj = wsm + j * SML_INDEX_HEADS;
         float s0 = 0.f, s1 = 0.f;
 #pragma unroll

@@ -11,29 +11,29 @@
 // with c_hat_i = e4m3 latent x its 128-element block scale.
 //
 // One CTA = (query token, group of 16 heads, split of up to 512 selected keys),
-// in tiles of 128 keys; keys are the MMA M dimension and the 16 heads N (an
-// MMA costs at least ~45 cycles whatever its N, and 16 heads as M would waste
-// 3/4 of the smallest M).
-//   * warp 11 gathers the selected 656-B rows, one bulk copy per row, into a
-//     ring of 16-row chunks that holds a whole tile;
-//   * warps 4-5 copy each row's E4M3 latent and bf16 RoPE key into
-//     128-B-swizzled MMA tiles (and the block scales aside);
-//   * warps 6-9 (one thread per latent dim) write V^T into TMEM as fp16
-//     (E4M3 -> fp16 is exact): the A operand of the PV MMA;
-//   * warp 10 issues tcgen05.mma: S_b^T = C_b . Q_b^T per 128-dim block b with
-//     kind::f8f6f4 straight from the E4M3 tile (the bf16 query split exactly
-//     into two E4M3 terms sharing a power-of-two scale per head, so both
-//     accumulate into one fp32 accumulator), the RoPE part with kind::f16
-//     (bf16), and after the softmax O_b^T += V_b^T . P'_b^T;
-//   * warps 0-3 (one thread per key) run the softmax on S^T: z = sm_scale c_t
-//     (sum_b scale_b s_h S_b + S_pe) in fp32, column maxima through shared
-//     memory, a lazily raised running max (O rescaled in TMEM only when a
-//     head's max grows by more than 8), P'_b = fp16(p x scale_b) and per-block
-//     row sums of exactly those weights divided by the scale (so a dominant
-//     key's rounding cancels in the normalisation); at the end they read O^T
-//     back (one thread per latent dim) and write the split's output and LSE.
-// The E4M3 tile is free again as soon as QK^T has read it, so the next tile is
-// staged while this one's softmax and PV run.
+// in tiles of 128 keys; keys are the MMA M dimension of QK^T and its K
+// dimension of PV, the 16 heads N (an MMA costs at least ~45 cycles whatever
+// its N, and 16 heads as M would waste 3/4 of the smallest M).  Both products
+// run on kind::f8f6f4 straight from the gathered E4M3 latent tile: nothing of
+// the latent is ever converted.
+//   * warps 4-14 gather the selected 656-B rows with 16-B asynchronous copies
+//     (one row per warp instruction) into 128-B-swizzled tiles: E4M3 latent,
+//     bf16 RoPE key, block scales aside; two tile buffers.  Random rows need
+//     many requests in flight per SM, hence many gather warps;
+//   * warp 15 issues the MMAs:
+//       S_b^T = C_b . [Qhi_b; Qlo_b]^T  (K-major; N = 32: both query terms),
+//       S_pe^T = K_pe . Q_pe^T          (kind::f16, bf16),
+//       O_b^T += C_b^T . [Bhi_b; Bmid_b; Blo_b]^T  (C_b^T read MN-major from
+//       the same tile; N = 48: the three weight terms);
+//     the next tile's QK^T follows this tile's PV;
+//   * warps 0-3 (one thread per key) run the softmax on S^T and build the
+//     weights B_b[i, h] = p_ih scale_ib / sigma_h as three E4M3 terms whose
+//     sum carries 12 significant bits (finer than fp16); sigma_h is a per-head
+//     power of two that keeps the terms in range, raised (and O rescaled,
+//     exactly) only when a tile would overflow; at the end they read O^T back
+//     (one thread per latent dim) and write the split's output and LSE.
+// The query is split exactly into two E4M3 terms sharing a power-of-two scale
+// per head; products of E4M3 values are exact and accumulate in fp32.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -45,36 +45,40 @@
 namespace sml {
 namespace {
 
-constexpr int kHC = 16;          // heads per CTA (MMA N)
-constexpr int kKT = 128;         // keys per tile (MMA M)
+constexpr int kHC = 16;          // heads per CTA
+constexpr int kKT = 128;         // keys per tile
 constexpr int kMaxSplit = 512;   // keys per split (4 tiles)
-constexpr int kChunk = 16;       // rows per gather chunk
-constexpr int kRing = kKT / kChunk;   // ring slots: one whole tile
-constexpr int kThreads = 384;    // warps 0-3 softmax, 4-5 stage, 6-9 V^T, 10 MMA, 11 gather
-constexpr int kStageWarps = 2;
+constexpr int kThreads = 512;    // warps 0-3 softmax, 4-14 gather, 15 MMA
+constexpr int kGatherWarps = 11;
+constexpr int kWarpMma = 15;
 constexpr float kLazyRescale = 8.f;   // nats
 
 // TMEM columns
-constexpr uint32_t kColVT = 0;      // V_b^T, fp16 pairs: 64 columns per block b (lanes = dims)
-constexpr uint32_t kColS = 256;     // S_b^T (lanes = keys): 16 columns per block b
-constexpr uint32_t kColSpe = 320;   // S_pe^T
-constexpr uint32_t kColO = 384;     // O_b^T (lanes = dims of block b): 16 columns per block
-constexpr uint32_t kColL = 448;     // per-key row-sum partials of block b (lanes = keys)
+constexpr uint32_t kColS = 0;       // S_b^T (lanes = keys): 32 columns per block b (hi | lo query term)
+constexpr uint32_t kColSpe = 128;   // S_pe^T
+constexpr uint32_t kColO = 256;     // O_b^T (lanes = dims of block b): 48 columns (hi | mid | lo) ...
+constexpr uint32_t kOStride = 64;   // ... at kColO + kOStride b
+constexpr int kPBytes = kKT * 3 * kHC;   // one block's weight terms: 128 keys x 48 E4M3
 
 struct __align__(1024) Smem {
-  uint8_t lat[4][kKT * 128];     // [block b][128 keys x 128 B] E4M3, SW128
-  uint8_t pe[kKT * 128];         // [128 keys x 64 bf16], SW128
-  uint8_t qhi[4][kHC * 128];     // query nope, high E4M3 term [block][16 heads x 128 B], SW128
-  uint8_t qlo[4][kHC * 128];     // low E4M3 term
+  uint8_t lat[2][4][kKT * 128];  // [buffer][block b][128 keys x 128 B] E4M3, SW128
+  uint8_t pe[2][kKT * 128];      // [buffer][128 keys x 64 bf16], SW128
+  uint8_t q8[4][2 * kHC * 128];  // [block] 32 rows x 128 B, SW128: rows 0-15 high term, 16-31 low term
   uint8_t qpe[kHC * 128];        // query RoPE bf16 [16 heads x 64], SW128
-  uint8_t p[4][kKT * kHC * 2];   // P'_b fp16, MN-major 8x8 core matrices; p[2..3] double as the exchange buffer
-  uint8_t raw[kRing][kChunk * SML_LATENT_ROW_BYTES];
-  float sc[kKT][4];              // [key][block] scales of the staged tile
+  uint8_t pb[4][kPBytes];        // weight terms of block b, MN-major 8-key x 16-B core matrices
+  float xch[kKT * kHC];          // softmax column-reduction exchange
+  float sc[2][kKT][4];           // [buffer][key][block] scales of the staged tile
   float qs[kHC];                 // power-of-two query scale per head
-  float hstat[kHC];              // per-head tile max / row sum
+  float hstat[kHC];              // per-head row sum (epilogue)
+  float hm[kHC];                 // per-head running max m_h
+  float hsig[kHC];               // per-head weight scale sigma_h (a power of two; 0 = not set yet)
+  float halpha[kHC];             // this tile's exp(m_old - m_new)
+  float hf[kHC];                 // this tile's rescale factor of O
+  float hinv[kHC];               // 1 / sigma_h (0 while unset)
+  float scw[2][4];               // per-warp max of the tile's scales (double-buffered by tile)
   int32_t rowid[kMaxSplit];      // pool row (page * 64 + row) of each key, -1 = masked
-  uint64_t q_ready, rows_ready, e_full, e_free, s_full, p_full, vt_full, pv_done, drain;
-  uint64_t raw_full[kRing], raw_empty[kRing];
+  uint64_t e_full[2], e_free[2];
+  uint64_t q_ready, s_full, s_free, p_full, pv_done, drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -94,7 +98,7 @@ struct Params {
   int32_t* status;
 };
 
-// Byte address of (row, 16-B chunk) in a 128-B-swizzled K-major tile.
+// Byte address of (row, 16-B chunk) in a 128-B-swizzled tile of 128-B rows.
 __device__ __forceinline__ uint32_t sw128(uint32_t base, int row, int chunk) {
   return base + (row >> 3) * 1024 + (row & 7) * 128 + ((chunk ^ (row & 7)) << 4);
 }
@@ -103,15 +107,9 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-// Two E4M3 codes (low byte first) -> two fp16 values (exact), packed.
-__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t two) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
-  return (uint32_t)h.x | ((uint32_t)h.y << 16);
-}
-
 // Round two floats to E4M3 (nearest even, saturating); the codes, low byte = a.
 __device__ __forceinline__ uint32_t f2_to_e4m3x2(float a, float b) {
-  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3) & 0xffffu;
 }
 
 __device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t two) {
@@ -119,19 +117,41 @@ __device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t two) {
   return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
+// x (two values) -> E4M3 codes of the nearest value and the exact residual.
+__device__ __forceinline__ uint32_t split_e4m3x2(float& x0, float& x1) {
+  const uint32_t c = f2_to_e4m3x2(x0, x1);
+  const float2 r = e4m3x2_to_f2(c);
+  x0 -= r.x;
+  x1 -= r.y;
+  return c;
+}
+
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort) {
   const bool ok = ptx::mbar_wait(bar, parity, abort);
   return __all_sync(0xffffffffu, ok);
 }
 
-// Softmax exchange buffer: [128 keys][16] floats in P'_2 / P'_3, columns
-// XOR-swizzled by key.
+// AND of a flag over the four softmax warps (named barrier 1): every wait
+// outcome is made uniform across them before the next named barrier, so a
+// timed-out wait ends all four together instead of leaving three behind.
+__device__ __forceinline__ bool softmax_all(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}"
+      : "=r"(r)
+      : "r"((uint32_t)ok)
+      : "memory");
+  return r != 0;
+}
+
+// Softmax exchange buffer: [128 keys][16] floats, columns XOR-swizzled by key.
 __device__ __forceinline__ float* xbuf(Smem& S, int key, int col) {
-  return reinterpret_cast<float*>(S.p[2]) + key * kHC + (col ^ (key & 15));
+  return S.xch + key * kHC + (col ^ (key & 15));
 }
 
 // Sum (or max) over the 128 keys of 16 per-key values (warps 0-3); every
-// softmax thread reads the 16 results from S.hstat afterwards.
+// softmax thread reads the 16 results from S.hstat afterwards.  Shared writes
+// made before the call are visible to all four warps after it.
 template <bool kMax>
 __device__ __forceinline__ void column_reduce(Smem& S, int row, const float (&v)[kHC]) {
 #pragma unroll
@@ -151,6 +171,64 @@ __device__ __forceinline__ void column_reduce(Smem& S, int row, const float (&v)
   }
   if (part == 0) S.hstat[hh] = acc;
   asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// Per-tile softmax statistics (warps 0-3).  Max over the 128 keys of z; then
+// the thread owning head h updates, for that head, the lazily raised running
+// max m_h and the weight scale sigma_h: the tile's weights are at most
+// exp(tmax_h - m_h) * SC (SC = largest block scale in the tile) and must stay
+// <= 448 sigma_h; sigma_h is reset to the next power of two >= U_h / 448
+// (U_h below) whenever U_h leaves [28, 448] sigma_h.  O holds
+// sum(weights / sigma), so both changes rescale it by
+// f_h = exp(m_old - m_new) * sigma_old / sigma_new (exact for the sigma
+// part).  Returns whether any f_h != 1.
+__device__ __forceinline__ bool tile_stats(Smem& S, int row, const float (&z)[kHC], int tile) {
+#pragma unroll
+  for (int h = 0; h < kHC; ++h) *xbuf(S, row, h) = z[h];
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  const int hh = row >> 3, part = row & 7;
+  float tm = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < kKT / 8; ++j) tm = fmaxf(tm, *xbuf(S, part + 8 * j, hh));
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, o));
+  uint32_t changed = 0;
+  if (part == 0) {
+    const float* w = S.scw[tile & 1];
+    const float SC = fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3]));
+    float m = S.hm[hh], sig = S.hsig[hh];
+    float alpha = 1.f;
+    if (tm > m + kLazyRescale || (m == -INFINITY && tm != -INFINITY)) {
+      alpha = m == -INFINITY ? 0.f : expf(m - tm);
+      m = tm;
+    }
+    // Weights that matter are ~SC (p ~ 1 against the running max) or, in a
+    // tile above the running max, up to exp(tmax - m) SC; sigma keeps the
+    // largest of them within [28, 448] sigma, so the dominant weights keep all
+    // 12 bits of the three-term split, and moves only when they leave it.
+    const float U = tm == -INFINITY ? 0.f : fmaxf(expf(tm - m), 1.f) * SC;
+    float beta = 1.f;
+    if (U > 0.f && (U > 448.f * sig || U < 28.f * sig)) {
+      int e = 0;
+      frexpf(U * (1.f / 448.f), &e);   // U / 448 < 2^e
+      const float ns = ldexpf(1.f, e);
+      beta = sig > 0.f ? sig / ns : 1.f;
+      sig = ns;
+    }
+    S.hm[hh] = m;
+    S.hsig[hh] = sig;
+    S.halpha[hh] = alpha;
+    S.hf[hh] = alpha * beta;
+    S.hinv[hh] = sig > 0.f ? 1.f / sig : 0.f;
+    changed = alpha * beta != 1.f;
+  }
+  uint32_t any;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}"
+      : "=r"(any)
+      : "r"(changed)
+      : "memory");
+  return any != 0;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params P) {
@@ -185,23 +263,20 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
   const int ntiles = (nkeys + kKT - 1) / kKT;
 
   if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&S.e_full[i], 32 * kGatherWarps);   // one arrival per gather thread, on completion of its copies
+      ptx::mbar_init(&S.e_free[i], 1);   // PV of the tile done (it is the tile's last reader)
+    }
     ptx::mbar_init(&S.q_ready, 4);
-    ptx::mbar_init(&S.rows_ready, kStageWarps);
-    ptx::mbar_init(&S.e_full, kStageWarps);
-    ptx::mbar_init(&S.e_free, 1 + 4);     // QK done + softmax warps read the scales
     ptx::mbar_init(&S.s_full, 1);
+    ptx::mbar_init(&S.s_free, 4);
     ptx::mbar_init(&S.p_full, 4);
-    ptx::mbar_init(&S.vt_full, 4);
     ptx::mbar_init(&S.pv_done, 1);
     ptx::mbar_init(&S.drain, 1);
-    for (int i = 0; i < kRing; ++i) {
-      ptx::mbar_init(&S.raw_full[i], 1);
-      ptx::mbar_init(&S.raw_empty[i], kStageWarps + 4);   // stage warps + V^T warps
-    }
     S.abort = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 10) {
+  if (warp == kWarpMma) {
     ptx::tmem_alloc(&S.tmem_base, 512);
     ptx::tmem_relinquish();
   }
@@ -212,178 +287,110 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
   const uint32_t T0 = S.tmem_base;
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
 
-  if (warp >= 4 && warp < 4 + kStageWarps) {
-    // ================= stage warps: row offsets, then rows -> swizzled tiles =================
-    constexpr int kST = 32 * kStageWarps;
-    const int ct = threadIdx.x - 128;   // 0 .. kST - 1
-    {
-      // Pool rows of the split's keys: all position loads, then all block-table loads.
-      constexpr int kPer = kMaxSplit / kST;
-      int pos[kPer], ph[kPer];
-#pragma unroll
-      for (int j = 0; j < kPer; ++j) {
-        const int k = ct + j * kST;
-        pos[j] = k < nkeys ? __ldg(P.idx + (size_t)t * P.K + kb + k) : -1;
-      }
-#pragma unroll
-      for (int j = 0; j < kPer; ++j) {
-        const int k = ct + j * kST;
-        const bool in = k < nkeys && pos[j] >= 0 && pos[j] < n;
-        if (k < nkeys && !in) raise_fault(P.status, SML_FAULT_INDEX);
-        ph[j] = in ? __ldg(P.block_table + (size_t)r * P.max_pages + pos[j] / SML_PAGE_TOKENS) : -1;
-        if (!in) pos[j] = -1;
-      }
-#pragma unroll
-      for (int j = 0; j < kPer; ++j) {
-        int32_t id = -1;
-        if (pos[j] >= 0) {
-          if (ph[j] >= 0 && ph[j] < P.latent_pages)
-            id = ph[j] * SML_PAGE_TOKENS + pos[j] % SML_PAGE_TOKENS;
+  if (warp >= 4 && warp < 4 + kGatherWarps) {
+    // ================= gather warps: row offsets, then rows -> swizzled tiles =================
+    constexpr int kGT = 32 * kGatherWarps;
+    const int ct = threadIdx.x - 128;   // 0 .. kGT - 1
+    // Pool rows of the split's keys.
+    for (int k = ct; k < kMaxSplit; k += kGT) {
+      int32_t id = -1;
+      if (k < nkeys) {
+        const int pos = __ldg(P.idx + (size_t)t * P.K + kb + k);
+        if (pos >= 0 && pos < n) {
+          const int ph = __ldg(P.block_table + (size_t)r * P.max_pages + pos / SML_PAGE_TOKENS);
+          if (ph >= 0 && ph < P.latent_pages)
+            id = ph * SML_PAGE_TOKENS + pos % SML_PAGE_TOKENS;
           else
             raise_fault(P.status, SML_FAULT_PAGE);
+        } else {
+          raise_fault(P.status, SML_FAULT_INDEX);
         }
-        S.rowid[ct + j * kST] = id;
       }
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&S.rows_ready);
+      S.rowid[k] = id;
     }
-    // Rows -> tiles: stage warp w takes rows kRowsPerWarp w .. of each chunk.
-    constexpr int kRowsPerWarp = kChunk / kStageWarps;
-    const int sw = warp - 4;
-    int chunk = 0;
+    asm volatile("bar.sync 2, %0;" ::"n"(kGT) : "memory");
+    // Rows -> tiles, one row per warp instruction: lane l copies latent chunk l
+    // (block l / 8, chunk l % 8), then lane 0 the four scales and lanes 1-8
+    // the RoPE key.  A masked row is zero-filled (nothing is read).  The
+    // tile's barrier completes when every gather thread's copies have landed,
+    // so the warps go straight on to the next tile: two tiles in flight.
+    const int gw = warp - 4;
+    bool ok = true;
     for (int tile = 0; tile < ntiles; ++tile) {
-      if (tile > 0 && !warp_wait(&S.e_free, (tile - 1) & 1, abort)) { *abort = 1; break; }
-      bool ok = true;
-      for (int cc = 0; cc < kRing; ++cc, ++chunk) {
-        const int slot = chunk % kRing;
-        if (!warp_wait(&S.raw_full[slot], (chunk / kRing) & 1, abort)) { ok = false; break; }
-#pragma unroll
-        for (int rr = 0; rr < kRowsPerWarp; ++rr) {
-          const int j = kRowsPerWarp * sw + rr; // row within the chunk
-          const int row = cc * kChunk + j;      // row within the tile
-          const bool valid = S.rowid[tile * kKT + row] >= 0;
-          const uint8_t* src = S.raw[slot] + j * SML_LATENT_ROW_BYTES;
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (valid) v = *reinterpret_cast<const uint4*>(src + 16 * lane);
-          st_shared_v4(sw128(ptx::smem_u32(S.lat[lane >> 3]), row, lane & 7), v.x, v.y, v.z, v.w);
-          if (lane < 8) {
-            uint4 e = make_uint4(0u, 0u, 0u, 0u);
-            if (valid && P.rope_dim) e = *reinterpret_cast<const uint4*>(src + SML_LATENT_DIM + 16 + 16 * lane);
-            st_shared_v4(sw128(ptx::smem_u32(S.pe), row, lane), e.x, e.y, e.z, e.w);
-          } else if (lane < 12) {
-            S.sc[row][lane - 8] = valid ? reinterpret_cast<const float*>(src + SML_LATENT_DIM)[lane - 8] : 1.f;
-          }
-        }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&S.raw_empty[slot]);
+      const int buf = tile & 1;
+      if (tile >= 2 && !warp_wait(&S.e_free[buf], ((tile >> 1) - 1) & 1, abort)) { ok = false; break; }
+      const uint32_t lat_l = ptx::smem_u32(S.lat[buf][lane >> 3]);
+      const uint32_t pe_b = ptx::smem_u32(S.pe[buf]);
+      const uint32_t sc_b = ptx::smem_u32(&S.sc[buf][0][0]);
+      for (int row = gw; row < kKT; row += kGatherWarps) {
+        const int32_t id = S.rowid[tile * kKT + row];
+        const uint8_t* src = id >= 0 ? P.latent + (size_t)id * SML_LATENT_ROW_BYTES : P.latent;
+        const uint32_t nb = id >= 0 ? 16u : 0u;
+        ptx::cp_async16(sw128(lat_l, row, lane & 7), src + 16 * lane, nb);
+        if (lane == 0)
+          ptx::cp_async16(sc_b + row * 16, src + SML_LATENT_DIM, nb);
+        else if (lane <= 8 && P.rope_dim)
+          ptx::cp_async16(sw128(pe_b, row, lane - 1), src + SML_LATENT_DIM + 16 * lane, nb);
       }
-      if (!ok) { *abort = 1; break; }
-      ptx::fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&S.e_full);
+      // every gather thread arrives once its own copies of this tile have landed
+      ptx::cp_async_arrive_noinc(&S.e_full[buf]);
     }
-  } else if (warp >= 4 + kStageWarps && warp < 8 + kStageWarps) {
-    // ================= V^T warps: one thread per latent dim of every block =================
-    const int d = (warp & 3) * 32 + lane;   // = TMEM lane (a warp reaches lanes 32 (warp % 4) ..)
-    int chunk = 0;
-    for (int tile = 0; tile < ntiles; ++tile) {
-      if (tile > 0 && !warp_wait(&S.pv_done, (tile - 1) & 1, abort)) { *abort = 1; break; }
-      ptx::tc_fence_after();
-      bool ok = true;
-      for (int cc = 0; cc < kRing; ++cc, ++chunk) {
-        const int slot = chunk % kRing;
-        if (!warp_wait(&S.raw_full[slot], (chunk / kRing) & 1, abort)) { ok = false; break; }
-        const uint8_t* src = S.raw[slot];
-        uint32_t vb[4][8];
-#pragma unroll
-        for (int jp = 0; jp < kChunk / 2; ++jp) {   // key pairs of the chunk
-          const int k0 = cc * kChunk + 2 * jp;
-          const bool v0 = S.rowid[tile * kKT + k0] >= 0, v1 = S.rowid[tile * kKT + k0 + 1] >= 0;
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            const uint32_t lo8 = v0 ? src[(2 * jp) * SML_LATENT_ROW_BYTES + 128 * b + d] : 0u;
-            const uint32_t hi8 = v1 ? src[(2 * jp + 1) * SML_LATENT_ROW_BYTES + 128 * b + d] : 0u;
-            vb[b][jp] = e4m3x2_to_h2(lo8 | (hi8 << 8));
-          }
-        }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&S.raw_empty[slot]);
-#pragma unroll
-        for (int b = 0; b < 4; ++b) ptx::tmem_st8(T0 + kColVT + 64 * b + 8 * cc + lane_off, vb[b]);
-      }
-      if (!ok) { *abort = 1; break; }
-      ptx::tmem_wait_st();
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&S.vt_full);
-    }
-  } else if (warp == 11) {
-    // ================= gather: one bulk copy per selected row =================
-    if (lane == 0) {
-      bool ok = ptx::mbar_wait(&S.rows_ready, 0, abort);
-      const int nchunks = ntiles * kRing;
-      int chunk = 0;
-      for (; ok && chunk < nchunks; ++chunk) {
-        const int slot = chunk % kRing;
-        if (!ptx::mbar_wait(&S.raw_empty[slot], ((chunk / kRing) & 1) ^ 1, abort)) { ok = false; break; }
-        uint32_t bytes = 0;
-        for (int j = 0; j < kChunk; ++j) bytes += S.rowid[chunk * kChunk + j] >= 0 ? SML_LATENT_ROW_BYTES : 0;
-        ptx::mbar_arrive_expect_tx(&S.raw_full[slot], bytes);
-        for (int j = 0; j < kChunk; ++j) {
-          const int32_t id = S.rowid[chunk * kChunk + j];
-          if (id >= 0)
-            ptx::bulk_load(S.raw[slot] + j * SML_LATENT_ROW_BYTES, P.latent + (size_t)id * SML_LATENT_ROW_BYTES,
-                           SML_LATENT_ROW_BYTES, &S.raw_full[slot]);
-        }
-      }
-      if (!ok) {
-        *abort = 1;
-        // Let copies already issued land before shared memory goes away.
-        for (int c = max(0, chunk - kRing); c < chunk; ++c)
-          ptx::mbar_wait(&S.raw_full[c % kRing], (c / kRing) & 1, nullptr, 1u << 16);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 10) {
+    ptx::cp_async_wait_all();   // no copy may still be landing when the CTA ends
+    if (!ok) *abort = 1;
+  } else if (warp == kWarpMma) {
     // ================= MMA issuer =================
     if (lane == 0) {
-      bool ok = ptx::mbar_wait(&S.q_ready, 0, abort);
-      const uint32_t id_qk = ptx::idesc_m128(kHC, 0);         // E4M3 x E4M3, K-major
-      const uint32_t id_pe = ptx::idesc_f16(kHC, 1, 0, 0);    // bf16
-      const uint32_t id_pv = ptx::idesc_f16(kHC, 0, 0, 1);    // f16; A (TMEM) K-major, B MN-major
-      for (int tile = 0; ok && tile < ntiles; ++tile) {
-        if (!ptx::mbar_wait(&S.e_full, tile & 1, abort)) { ok = false; break; }
-        ptx::tc_fence_after();
-        // S_b^T = C_b . (Qhi_b + Qlo_b)^T: four accumulators, 32 dims per step, interleaved
+      const uint32_t id_qk = ptx::idesc_f16(2 * kHC, 0, 0, 0);   // E4M3 x E4M3, both K-major, N = 32
+      const uint32_t id_pe = ptx::idesc_f16(kHC, 1, 0, 0);       // bf16, N = 16
+      const uint32_t id_pv = ptx::idesc_f16(3 * kHC, 0, 1, 1);   // E4M3 x E4M3, both MN-major, N = 48
+      auto issue_qk = [&](int buf) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < 4; ++k) {   // 32 latent dims per step
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            const uint64_t a = ptx::sdesc_sw128(ptx::smem_u32(S.lat[b]) + 32 * k);
-            ptx::mma_f8f6f4_ss(T0 + kColS + 16 * b, a, ptx::sdesc_sw128(ptx::smem_u32(S.qhi[b]) + 32 * k), id_qk, k > 0);
-            ptx::mma_f8f6f4_ss(T0 + kColS + 16 * b, a, ptx::sdesc_sw128(ptx::smem_u32(S.qlo[b]) + 32 * k), id_qk, 1);
-          }
+          for (int b = 0; b < 4; ++b)
+            ptx::mma_f8f6f4_ss(T0 + kColS + 32 * b, ptx::sdesc_sw128(ptx::smem_u32(S.lat[buf][b]) + 32 * k),
+                               ptx::sdesc_sw128(ptx::smem_u32(S.q8[b]) + 32 * k), id_qk, k > 0);
           if (P.rope_dim)
-            ptx::mma_f16_ss(T0 + kColSpe, ptx::sdesc_sw128(ptx::smem_u32(S.pe) + 32 * k),
+            ptx::mma_f16_ss(T0 + kColSpe, ptx::sdesc_sw128(ptx::smem_u32(S.pe[buf]) + 32 * k),
                             ptx::sdesc_sw128(ptx::smem_u32(S.qpe) + 32 * k), id_pe, k > 0);
         }
         ptx::mma_commit(&S.s_full);
-        ptx::mma_commit(&S.e_free);
-        if (!ptx::mbar_wait(&S.p_full, tile & 1, abort) || !ptx::mbar_wait(&S.vt_full, tile & 1, abort)) {
+      };
+      bool ok = ptx::mbar_wait(&S.q_ready, 0, abort) && ptx::mbar_wait(&S.e_full[0], 0, abort);
+      if (ok) {
+        ptx::tc_fence_after();
+        issue_qk(0);
+      }
+      for (int tile = 0; ok && tile < ntiles; ++tile) {
+        const int buf = tile & 1;
+        if (!ptx::mbar_wait(&S.p_full, tile & 1, abort)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        // O_b^T += V_b^T . P'_b^T: A = V_b^T in TMEM (16 keys = 8 columns per step);
-        // B = P'_b^T, MN-major core matrices (8-head blocks 128 B apart, 8-key groups 256 B apart).
+        // O_b^T += C_b^T . B_b^T, 32 keys per step.  A: the latent tile read
+        // MN-major (dims contiguous; 8-key swizzle atoms 1,024 B apart).  B:
+        // 8-key x 16-B core matrices, the three terms 128 B apart, 8-key
+        // groups 384 B apart.
 #pragma unroll
-        for (int k = 0; k < kKT / 16; ++k) {
+        for (int k = 0; k < kKT / 32; ++k) {
 #pragma unroll
           for (int b = 0; b < 4; ++b)
-            ptx::mma_f16_ts(T0 + kColO + 16 * b, T0 + kColVT + 64 * b + 8 * k,
-                            ptx::sdesc(ptx::smem_u32(S.p[b]) + 512 * k, 256, 128, 0), id_pv, (tile | k) != 0);
+            ptx::mma_f8f6f4_ss(T0 + kColO + kOStride * b, ptx::sdesc(ptx::smem_u32(S.lat[buf][b]) + 4096 * k, 16384, 1024, 2),
+                               ptx::sdesc(ptx::smem_u32(S.pb[b]) + 1536 * k, 384, 128, 0), id_pv, (tile | k) != 0);
         }
         ptx::mma_commit(&S.pv_done);
+        ptx::mma_commit(&S.e_free[buf]);
+        // next tile's QK^T, once its rows have landed and the softmax has read S
+        if (tile + 1 < ntiles) {
+          if (!ptx::mbar_wait(&S.e_full[buf ^ 1], ((tile + 1) >> 1) & 1, abort) ||
+              !ptx::mbar_wait(&S.s_free, tile & 1, abort)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          issue_qk(buf ^ 1);
+        }
       }
       if (!ok) *abort = 1;
       ptx::mma_commit(&S.drain);
@@ -432,17 +439,15 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
           // elements 16 c + 4 k .. + 3 of this thread's 64
           const uint4 vv = v[2 * c + (k >> 1)];
           const uint32_t wa = (k & 1) ? vv.z : vv.x, wb = (k & 1) ? vv.w : vv.y;
-          const float x0 = __uint_as_float(wa << 16) * inv, x1 = __uint_as_float(wa & 0xffff0000u) * inv;
-          const float x2 = __uint_as_float(wb << 16) * inv, x3 = __uint_as_float(wb & 0xffff0000u) * inv;
-          const uint32_t h01 = f2_to_e4m3x2(x0, x1), h23 = f2_to_e4m3x2(x2, x3);
-          const float2 r01 = e4m3x2_to_f2(h01), r23 = e4m3x2_to_f2(h23);
-          const uint32_t l01 = f2_to_e4m3x2(x0 - r01.x, x1 - r01.y), l23 = f2_to_e4m3x2(x2 - r23.x, x3 - r23.y);
-          hw[k] = (h01 & 0xffffu) | (h23 << 16);
-          lw[k] = (l01 & 0xffffu) | (l23 << 16);
+          float x0 = __uint_as_float(wa << 16) * inv, x1 = __uint_as_float(wa & 0xffff0000u) * inv;
+          float x2 = __uint_as_float(wb << 16) * inv, x3 = __uint_as_float(wb & 0xffff0000u) * inv;
+          const uint32_t h01 = split_e4m3x2(x0, x1), h23 = split_e4m3x2(x2, x3);
+          hw[k] = h01 | (h23 << 16);
+          lw[k] = f2_to_e4m3x2(x0, x1) | (f2_to_e4m3x2(x2, x3) << 16);
         }
         const int chunk = 4 * (part & 1) + c;
-        st_shared_v4(sw128(ptx::smem_u32(S.qhi[b]), h, chunk), hw[0], hw[1], hw[2], hw[3]);
-        st_shared_v4(sw128(ptx::smem_u32(S.qlo[b]), h, chunk), lw[0], lw[1], lw[2], lw[3]);
+        st_shared_v4(sw128(ptx::smem_u32(S.q8[b]), h, chunk), hw[0], hw[1], hw[2], hw[3]);
+        st_shared_v4(sw128(ptx::smem_u32(S.q8[b]), h + kHC, chunk), lw[0], lw[1], lw[2], lw[3]);
       }
       st_shared_v4(sw128(ptx::smem_u32(S.qpe), h, part), pv.x, pv.y, pv.z, pv.w);
       ptx::fence_proxy_async();
@@ -450,15 +455,17 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
       if (lane == 0) ptx::mbar_arrive(&S.q_ready);
     }
     const float zscale = P.sm_scale * (P.ssmax ? P.ssmax_s * logf((float)max(n, 1)) : 1.f);
-    float m[kHC];
+    float lrow[kHC];   // this key row's share of the row sums
 #pragma unroll
-    for (int h = 0; h < kHC; ++h) m[h] = -INFINITY;
-    bool ok = warp_wait(&S.q_ready, 0, abort);   // S.qs
-    float qs[kHC];
-#pragma unroll
-    for (int h = 0; h < kHC; ++h) qs[h] = S.qs[h];
+    for (int h = 0; h < kHC; ++h) lrow[h] = 0.f;
+    if (row < kHC) {
+      S.hm[row] = -INFINITY;
+      S.hsig[row] = 0.f;
+    }
+    bool ok = softmax_all(warp_wait(&S.q_ready, 0, abort));   // S.qs; orders the init above
     for (int tile = 0; ok && tile < ntiles; ++tile) {
-      if (!warp_wait(&S.e_full, tile & 1, abort) || !warp_wait(&S.s_full, tile & 1, abort)) {
+      const int buf = tile & 1;
+      if (!softmax_all(warp_wait(&S.e_full[buf], (tile >> 1) & 1, abort) && warp_wait(&S.s_full, tile & 1, abort))) {
         ok = false;
         break;
       }
@@ -466,147 +473,135 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
       const bool valid = S.rowid[tile * kKT + row] >= 0;
       float sc[4];
 #pragma unroll
-      for (int b = 0; b < 4; ++b) sc[b] = S.sc[row][b];
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&S.e_free);   // scales read
-      // z = zscale * (sum_b scale_b * s_h * S_b + S_pe), fp32
+      for (int b = 0; b < 4; ++b) sc[b] = S.sc[buf][row][b];
+      // z = zscale * (s_h * sum_b scale_b (S_b,hi + S_b,lo) + S_pe), fp32
       float z[kHC];
       {
-        uint32_t v[16];
-        float acc[kHC];
 #pragma unroll
-        for (int h = 0; h < kHC; ++h) acc[h] = 0.f;
+        for (int h = 0; h < kHC; ++h) z[h] = 0.f;
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
-          ptx::tmem_ld16(T0 + kColS + 16 * b + lane_off, v);
-          ptx::tmem_wait_ld();
+          uint32_t v[32];
+          ptx::tmem_ld32(T0 + kColS + 32 * b + lane_off, v);
+          ptx::tmem_wait_ld(v);
 #pragma unroll
-          for (int h = 0; h < kHC; ++h) acc[h] = fmaf(sc[b], __uint_as_float(v[h]), acc[h]);
+          for (int h = 0; h < kHC; ++h) z[h] = fmaf(sc[b], __uint_as_float(v[h]) + __uint_as_float(v[kHC + h]), z[h]);
         }
+#pragma unroll
+        for (int h = 0; h < kHC; ++h) z[h] *= S.qs[h];
         if (P.rope_dim) {
+          uint32_t v[16];
           ptx::tmem_ld16(T0 + kColSpe + lane_off, v);
-          ptx::tmem_wait_ld();
+          ptx::tmem_wait_ld(v);
 #pragma unroll
-          for (int h = 0; h < kHC; ++h) z[h] = __uint_as_float(v[h]);
-        } else {
-#pragma unroll
-          for (int h = 0; h < kHC; ++h) z[h] = 0.f;
+          for (int h = 0; h < kHC; ++h) z[h] += __uint_as_float(v[h]);
         }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&S.s_free);   // S read: the next tile's QK^T may overwrite it
 #pragma unroll
-        for (int h = 0; h < kHC; ++h) z[h] = valid ? fmaf(acc[h], qs[h], z[h]) * zscale : -INFINITY;
+        for (int h = 0; h < kHC; ++h) z[h] = valid ? z[h] * zscale : -INFINITY;
       }
-      column_reduce<true>(S, row, z);
-      // lazily raised running max; rescale O and the row-sum partials when it moves
-      float alpha[kHC];
-      bool any = false;
+      // the tile's largest block scale (masked rows were zero-filled: scale 0)
+      float scm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) scm = fmaxf(scm, __shfl_xor_sync(0xffffffffu, scm, o));
+      if (lane == 0) S.scw[tile & 1][warp] = scm;
+      const bool any = tile_stats(S, row, z, tile);
+#pragma unroll
+      for (int h = 0; h < kHC; ++h) lrow[h] *= S.halpha[h];
+      // The previous tile's PV reads the weight tiles and accumulates into O:
+      // wait for it before rescaling O or overwriting the weights.
+      if (tile > 0) {
+        if (!softmax_all(warp_wait(&S.pv_done, (tile - 1) & 1, abort))) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        if (any) {
+#pragma unroll 1
+          for (int b = 0; b < 4; ++b) {   // this thread: latent dim 128 b + row
+            uint32_t ov[32], ow[16];
+            ptx::tmem_ld32(T0 + kColO + kOStride * b + lane_off, ov);
+            ptx::tmem_ld16(T0 + kColO + kOStride * b + 32 + lane_off, ow);
+            ptx::tmem_wait_ld(ov, ow);
+#pragma unroll
+            for (int h = 0; h < kHC; ++h) {
+              const float f = S.hf[h];
+              ov[h] = __float_as_uint(__uint_as_float(ov[h]) * f);
+              ov[kHC + h] = __float_as_uint(__uint_as_float(ov[kHC + h]) * f);
+              ow[h] = __float_as_uint(__uint_as_float(ow[h]) * f);
+            }
+            ptx::tmem_st32(T0 + kColO + kOStride * b + lane_off, ov);
+            ptx::tmem_st16(T0 + kColO + kOStride * b + 32 + lane_off, ow);
+          }
+          ptx::tmem_wait_st();
+        }
+      }
+      // p = exp(z - m); weights x = p * scale_b / sigma as hi + mid + lo (E4M3)
 #pragma unroll
       for (int h = 0; h < kHC; ++h) {
-        const float tm = S.hstat[h];
-        alpha[h] = 1.f;
-        if (tm > m[h] + kLazyRescale || (m[h] == -INFINITY && tm != -INFINITY)) {
-          alpha[h] = m[h] == -INFINITY ? 0.f : expf(m[h] - tm);
-          m[h] = tm;
-          any = true;
-        }
+        const float p = z[h] == -INFINITY ? 0.f : expf(z[h] - S.hm[h]);
+        lrow[h] += p;
+        z[h] = p * S.hinv[h];
       }
-      if (any && tile > 0) {
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          uint32_t ov[16];
-          ptx::tmem_ld16(T0 + kColO + 16 * b + lane_off, ov);    // this thread: latent dim 128 b + row
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < kHC; ++h) ov[h] = __float_as_uint(__uint_as_float(ov[h]) * alpha[h]);
-          ptx::tmem_st16(T0 + kColO + 16 * b + lane_off, ov);
-          ptx::tmem_ld16(T0 + kColL + 16 * b + lane_off, ov);    // this thread: key row's partials
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < kHC; ++h) ov[h] = __float_as_uint(__uint_as_float(ov[h]) * alpha[h]);
-          ptx::tmem_st16(T0 + kColL + 16 * b + lane_off, ov);
-        }
-        ptx::tmem_wait_st();
-      }
-      float p[kHC];
-#pragma unroll
-      for (int h = 0; h < kHC; ++h) p[h] = z[h] == -INFINITY ? 0.f : expf(z[h] - m[h]);
-      // P'_b = fp16(p * scale_b); row-sum partial of block b += P'_b / scale_b
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
-        uint32_t lv[16], pw[8];
-        const float inv_sc = sc[b] > 0.f ? 1.f / sc[b] : 0.f;   // an all-zero block has scale 0
-        if (tile > 0) {
-          ptx::tmem_ld16(T0 + kColL + 16 * b + lane_off, lv);
-          ptx::tmem_wait_ld();
-        } else {
+        uint32_t wh[4], wm[4], wl[4];
 #pragma unroll
-          for (int h = 0; h < kHC; ++h) lv[h] = 0u;
+        for (int q = 0; q < 4; ++q) {   // heads 4 q .. 4 q + 3
+          float x0 = z[4 * q] * sc[b], x1 = z[4 * q + 1] * sc[b];
+          float x2 = z[4 * q + 2] * sc[b], x3 = z[4 * q + 3] * sc[b];
+          const uint32_t h01 = split_e4m3x2(x0, x1), h23 = split_e4m3x2(x2, x3);
+          const uint32_t m01 = split_e4m3x2(x0, x1), m23 = split_e4m3x2(x2, x3);
+          wh[q] = h01 | (h23 << 16);
+          wm[q] = m01 | (m23 << 16);
+          wl[q] = f2_to_e4m3x2(x0, x1) | (f2_to_e4m3x2(x2, x3) << 16);
         }
-#pragma unroll
-        for (int h = 0; h < kHC; h += 2) {
-          const __half2 ph = __floats2half2_rn(p[h] * sc[b], p[h + 1] * sc[b]);
-          const float2 pr = __half22float2(ph);
-          const float w0 = inv_sc > 0.f ? pr.x * inv_sc : p[h];
-          const float w1 = inv_sc > 0.f ? pr.y * inv_sc : p[h + 1];
-          lv[h] = __float_as_uint(__uint_as_float(lv[h]) + w0);
-          lv[h + 1] = __float_as_uint(__uint_as_float(lv[h + 1]) + w1);
-          pw[h >> 1] = *reinterpret_cast<const uint32_t*>(&ph);
-        }
-        ptx::tmem_st16(T0 + kColL + 16 * b + lane_off, lv);
-        const uint32_t pb = ptx::smem_u32(S.p[b]) + (row >> 3) * 256 + (row & 7) * 16;
-        st_shared_v4(pb, pw[0], pw[1], pw[2], pw[3]);          // heads 0-7
-        st_shared_v4(pb + 128, pw[4], pw[5], pw[6], pw[7]);    // heads 8-15
+        const uint32_t pb = ptx::smem_u32(S.pb[b]) + (row >> 3) * 384 + (row & 7) * 16;
+        st_shared_v4(pb, wh[0], wh[1], wh[2], wh[3]);
+        st_shared_v4(pb + 128, wm[0], wm[1], wm[2], wm[3]);
+        st_shared_v4(pb + 256, wl[0], wl[1], wl[2], wl[3]);
       }
-      ptx::tmem_wait_st();
       ptx::fence_proxy_async();
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&S.p_full);
     }
-    if (ok && !warp_wait(&S.pv_done, (ntiles - 1) & 1, abort)) ok = false;
+    ok = softmax_all(ok && warp_wait(&S.pv_done, (ntiles - 1) & 1, abort));
     if (!ok) *abort = 1;
     ptx::tc_fence_after();
-    // Per block: row sums over the 128 key lanes, then the normalised output.
-    float lsum0[kHC];
+    // Row sums over the 128 key lanes, then the output: sigma_h (hi + mid + lo) / l_h.
+    column_reduce<false>(S, row, lrow);
+    float osc[kHC];
 #pragma unroll
+    for (int h = 0; h < kHC; ++h) {
+      const float ls = S.hstat[h];
+      osc[h] = ls > 0.f ? S.hsig[h] / ls : 0.f;
+    }
+#pragma unroll 1
     for (int b = 0; b < 4; ++b) {
-      uint32_t lv[16];
-      ptx::tmem_ld16(T0 + kColL + 16 * b + lane_off, lv);
-      ptx::tmem_wait_ld();
-      float lf[kHC];
-#pragma unroll
-      for (int h = 0; h < kHC; ++h) lf[h] = __uint_as_float(lv[h]);
-      column_reduce<false>(S, row, lf);
-      float inv[kHC];
-#pragma unroll
-      for (int h = 0; h < kHC; ++h) {
-        const float ls = S.hstat[h];
-        inv[h] = ls > 0.f ? 1.f / ls : 0.f;
-        if (b == 0) lsum0[h] = ls;
-      }
-      uint32_t ov[16];
-      ptx::tmem_ld16(T0 + kColO + 16 * b + lane_off, ov);
-      ptx::tmem_wait_ld();
+      uint32_t ov[32], ow[16];
+      ptx::tmem_ld32(T0 + kColO + kOStride * b + lane_off, ov);
+      ptx::tmem_ld16(T0 + kColO + kOStride * b + 32 + lane_off, ow);
+      ptx::tmem_wait_ld(ov, ow);
       const int dim = 128 * b + row;
 #pragma unroll
-      for (int h = 0; h < kHC; ++h)
-        P.ws.part_out[(slot0 + (size_t)h * P.ws.splits) * SML_LATENT_DIM + dim] = __uint_as_float(ov[h]) * inv[h];
-    }
-    // lse from block 0's row sums: sum_i fp16(p_i * scale_i0) / scale_i0 ~ sum_i p_i.
-    if (row < kHC) {
-      float mrow = 0.f, lrow = 0.f;   // m[row], lsum0[row] without dynamic register indexing
-#pragma unroll
       for (int h = 0; h < kHC; ++h) {
-        mrow = (h == row) ? m[h] : mrow;
-        lrow = (h == row) ? lsum0[h] : lrow;
+        const float o = __uint_as_float(ov[h]) + __uint_as_float(ov[kHC + h]) + __uint_as_float(ow[h]);
+        P.ws.part_out[(slot0 + (size_t)h * P.ws.splits) * SML_LATENT_DIM + dim] = o * osc[h];
       }
-      P.ws.part_lse[slot0 + (size_t)row * P.ws.splits] = lrow > 0.f ? mrow + logf(lrow) : -INFINITY;
+    }
+    if (row < kHC) {
+      const float lsum = S.hstat[row];
+      P.ws.part_lse[slot0 + (size_t)row * P.ws.splits] = lsum > 0.f ? S.hm[row] + logf(lsum) : -INFINITY;
     }
   }
 
   ptx::tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && S.abort) raise_fault(P.status, SML_FAULT_TIMEOUT);
-  if (warp == 10) {
+  if (warp == kWarpMma) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(S.tmem_base, 512);
   }
