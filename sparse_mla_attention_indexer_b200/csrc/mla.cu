@@ -25,7 +25,8 @@
 //       S_pe^T = K_pe . Q_pe^T          (kind::f16, bf16),
 //       O_b^T += C_b^T . [Bhi_b; Bmid_b; Blo_b]^T  (C_b^T read MN-major from
 //       the same tile; N = 48: the three weight terms);
-//     the next tile's QK^T follows this tile's PV;
+//     the next tile's QK^T goes in ahead of this tile's PV, as soon as its
+//     rows have landed and the softmax has read S;
 //   * warps 0-3 (one thread per key) run the softmax on S^T and build the
 //     weights B_b[i, h] = p_ih scale_ib / sigma_h as three E4M3 terms whose
 //     sum carries 12 significant bits (finer than fp16); sigma_h is a per-head
@@ -363,6 +364,16 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
       }
       for (int tile = 0; ok && tile < ntiles; ++tile) {
         const int buf = tile & 1;
+        if (tile + 1 < ntiles) {
+          // next tile's QK^T once its rows have landed and the softmax has read S
+          if (!ptx::mbar_wait(&S.e_full[buf ^ 1], ((tile + 1) >> 1) & 1, abort) ||
+              !ptx::mbar_wait(&S.s_free, tile & 1, abort)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          issue_qk(buf ^ 1);
+        }
         if (!ptx::mbar_wait(&S.p_full, tile & 1, abort)) {
           ok = false;
           break;
@@ -381,16 +392,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
         }
         ptx::mma_commit(&S.pv_done);
         ptx::mma_commit(&S.e_free[buf]);
-        // next tile's QK^T, once its rows have landed and the softmax has read S
-        if (tile + 1 < ntiles) {
-          if (!ptx::mbar_wait(&S.e_full[buf ^ 1], ((tile + 1) >> 1) & 1, abort) ||
-              !ptx::mbar_wait(&S.s_free, tile & 1, abort)) {
-            ok = false;
-            break;
-          }
-          ptx::tc_fence_after();
-          issue_qk(buf ^ 1);
-        }
       }
       if (!ok) *abort = 1;
       ptx::mma_commit(&S.drain);
