@@ -84,7 +84,8 @@ __device__ __forceinline__ int block_scan_incl(int v, int* warp_tot, int* total)
 
 // Over the histogram sh.hist[0, nb): the bin holding the `need`-th largest
 // element, and how many elements lie in the bins above it.
-__device__ __forceinline__ void find_bin(int nb, int need, SelectShared& sh, int* bin, int* above_out) {
+template <typename Sh>
+__device__ __forceinline__ void find_bin(int nb, int need, Sh& sh, int* bin, int* above_out) {
   const int tid = threadIdx.x, nt = blockDim.x;
   const int bpt = nb / nt;   // nb is a multiple of nt
   int local = 0;
@@ -109,8 +110,8 @@ __device__ __forceinline__ void find_bin(int nb, int need, SelectShared& sh, int
 
 // Radix select over n keys: the k-th largest key tau (1 <= k <= n) and how
 // many keys equal to tau belong to the top k (*take).
-template <typename KeyAt>
-__device__ void radix_threshold(int n, int k, KeyAt key_at, SelectShared& sh, uint32_t* tau, int* take) {
+template <typename KeyAt, typename Sh>
+__device__ void radix_threshold(int n, int k, KeyAt key_at, Sh& sh, uint32_t* tau, int* take) {
   const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
   uint32_t prefix = 0, pmask = 0;
   int remaining = k;
@@ -460,10 +461,439 @@ topk_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32_t* __re
   }
 }
 
+// ---- one cluster per row --------------------------------------------------------
+//
+// Rows of up to kClusterMax chunks: the chunks' CTAs form one thread-block
+// cluster and select together, in one level, exchanging histograms, the keys
+// of the threshold bucket and the selected counts through distributed shared
+// memory at hardware cluster barriers.  Each CTA makes one pass over its chunk
+// that histograms the values at or above a sampled floor and compacts them,
+// in position order, into per-warp candidate lists; every later step touches
+// only those candidates.
+
+constexpr int kClusterMax = 8;
+constexpr int kWarps = kTopkThreads / 32;
+constexpr int kSegMax = kTopkChunk / kWarps;   // positions per warp segment
+
+struct ClusterShared {
+  int hist[kBuckets];              // this CTA's histogram (read by the whole cluster)
+  int gh[kBuckets];                // the cluster's histogram
+  uint16_t cpos[kWarps][kSegMax];  // candidate positions (chunk-local) per warp, ascending
+  int wcnt[kWarps];                // candidates per warp
+  uint32_t bkeys[kCandCap];        // this CTA's keys in the threshold bucket (read by the cluster)
+  uint32_t gkeys[kCandCap];        // the cluster's keys in the threshold bucket
+  int nbk;                         // this CTA's count of them (read by the cluster)
+  int sel[2];                      // this CTA's keys > tau and == tau (read by the cluster)
+  int samp_hist[256];
+  int warp_a[32], warp_b[32];
+  float red_lo[32], red_hi[32];
+  int bcast[2];
+  uint32_t bcast_tau;
+  float bcast_f;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA of the cluster; shared-memory writes before it are
+// visible to the cluster's reads after it.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Load a 32-bit word at `p`'s offset in the shared memory of cluster CTA `rank`.
+__device__ __forceinline__ uint32_t ld_cluster(const void* p, uint32_t rank) {
+  uint32_t a, v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"((uint32_t)__cvta_generic_to_shared(p)), "r"(rank));
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+
+// S.gh = the sum over the cluster of every CTA's S.hist[0, nb).
+__device__ __forceinline__ void cluster_hist_sum(ClusterShared& S, int nb, int C) {
+  __syncthreads();
+  cluster_sync();
+  for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+    int s = 0;
+    for (int r = 0; r < C; ++r) s += (int)ld_cluster(&S.hist[b], r);
+    S.gh[b] = s;
+  }
+  __syncthreads();
+  cluster_sync();   // nobody rewrites its histogram before every CTA has read it
+}
+
+// Warp 0: over h[0, nb) the bin holding the `need`-th largest element and the
+// count above it, into S.bcast.
+__device__ __forceinline__ void find_bin_desc_warp(const int* h, int nb, int need, ClusterShared& S) {
+  const int lane = threadIdx.x & 31;
+  const int per = nb / 32;
+  const int top = nb - 1 - lane * per;
+  int local = 0;
+  for (int j = 0; j < per; ++j) local += h[top - j];
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int before = incl - local;
+  if (before < need && need <= incl) {
+    int above = before;
+    for (int j = 0; j < per; ++j) {
+      const int hh = h[top - j];
+      if (need <= above + hh) {
+        S.bcast[0] = top - j;
+        S.bcast[1] = above;
+        break;
+      }
+      above += hh;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kTopkThreads, 1)
+topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32_t* __restrict__ cu_q,
+                    const int32_t* __restrict__ ctx_len, const float* __restrict__ scores,
+                    int32_t* __restrict__ idx, int32_t* __restrict__ idx_len, int32_t* status) {
+  extern __shared__ __align__(16) uint8_t tk_smem[];
+  uint32_t* keys = reinterpret_cast<uint32_t*>(tk_smem);
+  ClusterShared& S = *reinterpret_cast<ClusterShared*>(tk_smem + kTopkChunk * sizeof(uint32_t));
+  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int C = (int)cluster_size(), c = (int)cluster_rank();
+  const int t = blockIdx.y;
+  // Everything up to the first cluster barrier depends only on the row, so an
+  // early return is taken by the whole cluster or by none of it.
+  const int r = request_of_warp(cu_q, B, t);
+  const Req rq = load_request(cu_q, ctx_len, r, T, max_ctx, max_pages);
+  int32_t* out = idx + (size_t)t * K;
+  if (!rq.ok || t < rq.q0 || t - rq.q0 >= rq.Q) {
+    if (c == 0) {
+      for (int i = tid; i < K; i += nt) out[i] = -1;
+      if (tid == 0) {
+        idx_len[t] = 0;
+        raise_fault(status, SML_FAULT_LENGTHS);
+      }
+    }
+    return;
+  }
+  const int n = rq.L - rq.Q + (t - rq.q0) + 1;
+  if (n <= K) {
+    if (c == 0) {
+      for (int i = tid; i < K; i += nt) out[i] = i < n ? i : -1;
+      if (tid == 0) idx_len[t] = n;
+    }
+    return;
+  }
+  // Balanced chunks, multiples of 32 positions (n <= C * kTopkChunk).
+  const int per = ((n + C - 1) / C + 31) & ~31;
+  const int c0 = min(n, c * per), cn = min(n, c0 + per) - c0;
+  const float* row = scores + (size_t)t * max_ctx;
+
+  // 1. this chunk's keys into shared memory; the row's sample straight from
+  //    global memory (every CTA takes the same sample, so all agree on it).
+#pragma unroll 8
+  for (int i = tid; i < cn; i += nt) keys[i] = order_key(__ldcg(row + c0 + i));
+  const int ns = min(kSample, n);
+  float sv[kSample / kTopkThreads];
+  float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < kSample / kTopkThreads; ++u) {
+    const int j = tid + u * nt;
+    sv[u] = NAN;
+    if (j < ns) {
+      sv[u] = key_value(order_key(__ldcg(row + (int)((long long)j * n / ns))));
+      if (isfinite(sv[u])) {
+        lo = fminf(lo, sv[u]);
+        hi = fmaxf(hi, sv[u]);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    S.red_lo[warp] = lo;
+    S.red_hi[warp] = hi;
+  }
+  for (int b = tid; b < 256; b += nt) S.samp_hist[b] = 0;
+  if (tid == 0) S.bcast_f = -INFINITY;
+  __syncthreads();
+  lo = INFINITY;
+  hi = -INFINITY;
+  for (int w = 0; w < kWarps; ++w) {
+    lo = fminf(lo, S.red_lo[w]);
+    hi = fmaxf(hi, S.red_hi[w]);
+  }
+  // 2. floor: the sample's ceil(mu + 4 sqrt(mu) + 4)-th largest value's coarse
+  //    bin (mu = k ns / n), so that about k (1 + a margin) values lie above it.
+  const float width = hi - lo;
+  const bool finite_range = hi > lo && width < INFINITY;
+  float floor_v = -INFINITY;
+  if (finite_range && n > 2 * K) {
+    const float cscale = 254.f / width;
+#pragma unroll
+    for (int u = 0; u < kSample / kTopkThreads; ++u) {
+      const float v = sv[u];
+      if (tid + u * nt < ns) {
+        const int cb = !(v > -INFINITY) ? 0 : (v == INFINITY ? 255 : 1 + (int)fminf(fmaxf((v - lo) * cscale, 0.f), 253.f));
+        atomicAdd(&S.samp_hist[cb], 1);
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const float mu = (float)K * ns / (float)n;
+      const int need_s = min(ns, (int)ceilf(mu + 4.f * sqrtf(mu) + 4.f));
+      const int top = 255 - 8 * lane;
+      int local = 0;
+      for (int j = 0; j < 8; ++j) local += S.samp_hist[top - j];
+      int incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int above = incl - local;
+      if (above < need_s && need_s <= incl) {
+        for (int j = 0; j < 8; ++j) {
+          above += S.samp_hist[top - j];
+          if (need_s <= above) {
+            const int cb = top - j;
+            S.bcast_f = cb <= 1 ? -INFINITY : lo + (float)(cb - 1) / cscale;
+            break;
+          }
+        }
+      }
+    }
+    __syncthreads();
+    floor_v = S.bcast_f;
+  }
+  // Fine buckets: 0 = NaN / -inf, 1 .. kBuckets-2 linear in value from the
+  // floor (or the sample's minimum) to the sample's maximum, clamped at both
+  // ends, kBuckets-1 = +inf: monotone in the key.
+  bool full = !(floor_v > -INFINITY);
+  float base_v = full ? lo : floor_v;
+  float scale = finite_range && hi > base_v ? (float)(kBuckets - 3) / (hi - base_v) : 0.f;
+  auto bucket = [&](uint32_t key) -> int {
+    const float v = key_value(key);
+    if (v == INFINITY) return kBuckets - 1;
+    if (!(v > -INFINITY)) return 0;
+    return 1 + (int)fminf(fmaxf((v - base_v) * scale, 0.f), (float)(kBuckets - 3));
+  };
+  // 3. one pass over the chunk: candidates (key >= the floor's key; every key
+  //    when there is no floor) into per-warp lists in position order, and the
+  //    histogram of their buckets.
+  const int seg = ((cn + kWarps - 1) / kWarps + 31) & ~31;
+  const int wb = min(cn, warp * seg), we = min(cn, wb + seg);
+  const unsigned below = (1u << lane) - 1u;
+  int total = 0;
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    const uint32_t fkey = full ? 0u : order_key(base_v);
+    for (int b = tid; b < kBuckets; b += nt) S.hist[b] = 0;
+    __syncthreads();
+    int cnt = 0;
+    for (int i0 = wb; i0 < we; i0 += 32) {
+      const int i = i0 + lane;
+      const uint32_t key = i < we ? keys[i] : 0u;
+      const bool cand = i < we && key >= fkey;
+      const unsigned m = __ballot_sync(0xffffffffu, cand);
+      if (cand) {
+        S.cpos[warp][cnt + __popc(m & below)] = (uint16_t)i;
+        atomicAdd(&S.hist[bucket(key)], 1);
+      }
+      cnt += __popc(m);
+    }
+    if (lane == 0) S.wcnt[warp] = cnt;
+    cluster_hist_sum(S, kBuckets, C);
+    int part = 0;
+    for (int b = tid; b < kBuckets; b += nt) part += S.gh[b];
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) S.warp_a[warp] = part;
+    __syncthreads();
+    total = 0;
+    for (int w = 0; w < kWarps; ++w) total += S.warp_a[w];
+    if (full || total >= K) break;   // the same in every CTA of the cluster
+    full = true;                     // the sample misjudged: every key is a candidate
+    base_v = lo;
+    scale = finite_range ? (float)(kBuckets - 3) / width : 0.f;
+    __syncthreads();
+  }
+  // 4. the threshold bucket (the same in every CTA)
+  if (warp == 0) find_bin_desc_warp(S.gh, kBuckets, K, S);
+  if (tid == 0) S.nbk = 0;
+  __syncthreads();
+  const int bk = S.bcast[0], need = K - S.bcast[1];
+  const int wn = S.wcnt[warp];
+  // 5. this CTA's keys in the threshold bucket; tau = the need-th largest over
+  //    the cluster, take = how many keys equal to tau are selected.
+  for (int j = lane; j < wn; j += 32) {
+    const uint32_t key = keys[S.cpos[warp][j]];
+    if (bucket(key) == bk) {
+      const int slot = atomicAdd(&S.nbk, 1);
+      if (slot < kCandCap) S.bkeys[slot] = key;
+    }
+  }
+  __syncthreads();
+  cluster_sync();
+  int nbt = 0, offs = 0;
+  bool fits = true;
+  for (int q = 0; q < C; ++q) {
+    const int m = (int)ld_cluster(&S.nbk, q);
+    if (q < c) offs += m;
+    nbt += m;
+    fits = fits && m <= kCandCap;
+  }
+  fits = fits && nbt <= kCandCap;
+  uint32_t tau;
+  int take;
+  if (fits) {
+    for (int q = 0, o = 0; q < C; ++q) {
+      const int m = (int)ld_cluster(&S.nbk, q);
+      for (int j = tid; j < m; j += nt) S.gkeys[o + j] = ld_cluster(&S.bkeys[j], q);
+      o += m;
+    }
+    __syncthreads();
+    if (nbt <= kSmallCand) {
+      if (tid < nbt) {
+        const uint32_t key = S.gkeys[tid];
+        int gt = 0, ge = 0;
+        for (int j = 0; j < nbt; ++j) {
+          const uint32_t x = S.gkeys[j];
+          gt += x > key;
+          ge += x >= key;
+        }
+        if (gt < need && need <= ge) {
+          S.bcast_tau = key;
+          S.bcast[1] = need - gt;
+        }
+      }
+      __syncthreads();
+      tau = S.bcast_tau;
+      take = S.bcast[1];
+    } else {
+      radix_threshold(nbt, need, [&](int i) { return S.gkeys[i]; }, S, &tau, &take);
+    }
+    __syncthreads();
+  } else {
+    // Heavy ties: a radix select (11 / 11 / 10 key bits) over the threshold
+    // bucket's keys where they lie, the histograms summed over the cluster.
+    uint32_t prefix = 0, pmask = 0;
+    int remaining = need;
+    for (int pass = 0; pass < 3; ++pass) {
+      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+      const int nb = pass == 2 ? 1024 : 2048;
+      for (int b = tid; b < nb; b += nt) S.hist[b] = 0;
+      __syncthreads();
+      for (int j = lane; j < wn; j += 32) {
+        const uint32_t key = keys[S.cpos[warp][j]];
+        if (bucket(key) == bk && (key & pmask) == prefix) atomicAdd(&S.hist[(key >> shift) & (uint32_t)(nb - 1)], 1);
+      }
+      cluster_hist_sum(S, nb, C);
+      if (warp == 0) find_bin_desc_warp(S.gh, nb, remaining, S);
+      __syncthreads();
+      remaining -= S.bcast[1];
+      prefix |= (uint32_t)S.bcast[0] << shift;
+      pmask |= (uint32_t)(nb - 1) << shift;
+      __syncthreads();
+    }
+    tau = prefix;
+    take = remaining;
+  }
+  // 6. counts of keys > tau and == tau: per warp, per CTA, then over the cluster
+  int cgt = 0, ceq = 0;
+  for (int j0 = 0; j0 < wn; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t key = j < wn ? keys[S.cpos[warp][j]] : 0u;
+    cgt += __popc(__ballot_sync(0xffffffffu, j < wn && key > tau));
+    ceq += __popc(__ballot_sync(0xffffffffu, j < wn && key == tau));
+  }
+  if (lane == 0) {
+    S.warp_a[warp] = cgt;
+    S.warp_b[warp] = ceq;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int a = lane < kWarps ? S.warp_a[lane] : 0, b = lane < kWarps ? S.warp_b[lane] : 0;
+    const int a0 = a, b0 = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, a, o), y = __shfl_up_sync(0xffffffffu, b, o);
+      if (lane >= o) {
+        a += x;
+        b += y;
+      }
+    }
+    if (lane < kWarps) {
+      S.warp_a[lane] = a - a0;   // exclusive prefixes over the warps
+      S.warp_b[lane] = b - b0;
+    }
+    if (lane == kWarps - 1) {
+      S.sel[0] = a;
+      S.sel[1] = b;
+    }
+  }
+  __syncthreads();
+  cluster_sync();
+  // ties go to the lowest positions: the CTAs before this one take theirs first
+  int out0 = 0, eq_before = 0;
+  for (int q = 0; q < c; ++q) {
+    const int g = (int)ld_cluster(&S.sel[0], q), e = (int)ld_cluster(&S.sel[1], q);
+    out0 += g + max(0, min(e, take - eq_before));
+    eq_before += e;
+  }
+  const int my_take = max(0, take - eq_before);   // ties this CTA may still take
+  // 7. emission in position order
+  int g = S.warp_a[warp], e = S.warp_b[warp];
+  for (int j0 = 0; j0 < wn; j0 += 32) {
+    const int j = j0 + lane;
+    const int pos = j < wn ? S.cpos[warp][j] : 0;
+    const uint32_t key = j < wn ? keys[pos] : 0u;
+    const bool gt = j < wn && key > tau, eq = j < wn && key == tau;
+    const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+    const int gb = g + __popc(bg & below), eb = e + __popc(be & below);
+    if (gt || (eq && eb < my_take)) out[out0 + gb + min(eb, my_take)] = c0 + pos;
+    g += __popc(bg);
+    e += __popc(be);
+  }
+  if (c == 0 && tid == 0) idx_len[t] = K;
+  __syncthreads();
+  cluster_sync();   // shared memory stays until every CTA of the cluster is done reading it
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const sml_problem& p, const float* scores, int32_t* idx, int32_t* idx_len,
                         const TopkWs& ws, int32_t* status, cudaStream_t stream) {
+  if (ws.chunks <= kClusterMax) {
+    // one cluster of ws.chunks CTAs per row
+    const size_t smem = (size_t)kTopkChunk * sizeof(uint32_t) + sizeof(ClusterShared);
+    cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ws.chunks, p.num_tokens);
+    cfg.blockDim = dim3(kTopkThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = ws.chunks;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, p.num_requests, p.num_tokens, p.topk, p.max_ctx,
+                           p.max_pages, p.cu_q, p.ctx_len, scores, idx, idx_len, status);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   const size_t smem = (size_t)kTopkChunk * sizeof(uint32_t);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
