@@ -243,12 +243,18 @@ def barrier():
         torch.distributed.barrier()
 
 
-def max_over_ranks(x: float) -> float:
+def max_over_ranks(x: float, device: str = "cuda") -> float:
+    """The largest x over the ranks (every rank gets it); x itself on one process."""
     if torch.distributed.is_available() and torch.distributed.is_initialized():
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        t = torch.tensor([x], dtype=torch.float64, device=device)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         return float(t.item())
     return x
+
+
+def whole_job_rate(world: int, units_per_rank: float, ms_max: float) -> float:
+    """Units all ranks processed per second, timed by the slowest rank."""
+    return world * units_per_rank / (ms_max / 1e3)
 
 
 def cpu_baseline(wl, budget_s: float = 15.0):
@@ -326,14 +332,14 @@ def main():
         torch.distributed.destroy_process_group()
     if rank != 0:
         return
-    qps = world * wl.T / (ms_step / 1e3)
+    qps = whole_job_rate(world, wl.T, ms_step)
     idx_gbs = units["indexer_bytes"] / (ms_idx / 1e3) / 1e9
     line = {
         "metric": metric, "value": qps, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e4m3/f16 products, f32 accumulate", "data": "synthetic",
         "config": config_of(wl, args, world),
-        "gathered_tokens_per_s": world * units["gathered"] / (ms_step / 1e3),
+        "gathered_tokens_per_s": whole_job_rate(world, units["gathered"], ms_step),
         "stage_ms": {"indexer": ms_idx, "topk": ms_topk, "sparse_mla_and_merge": ms_mla},
         "indexer_hbm_gbs": idx_gbs, "indexer_frac_of_8000_gbs": idx_gbs / 8000.0,
         "mla_hbm_gbs": units["mla_bytes"] / (ms_mla / 1e3) / 1e9,
@@ -343,7 +349,7 @@ def main():
                      "algorithmic_bytes_per_launch": units["indexer_bytes"],
                      "traffic": INDEXER_NCU_TRAFFIC_BYTES},
         "clocks": clocks,
-        "e2e": {"value": world * wl.T / (e2e_ms / 1e3), "unit": "queries/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": whole_job_rate(world, wl.T, e2e_ms), "unit": "queries/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "entry_point": "sml_run_layer"},
         "gpu_launches": args.steps * 4,
         "cpu_baseline": cb,
