@@ -8,12 +8,12 @@ One step = one layer's sparse attention over one batch: the default workload is
 64 indexer heads of dim 128, top-2048, 64-token pages over a permuted shared
 pool (one TP8 rank of batched decode).  Inputs are seeded synthetic data.
 
-Timing: the step (the three stage calls, with a CUDA event before, between and
-after them) is captured once into a CUDA graph.  W untimed warm-up replays;
-then K replays, each preceded by a 256 MiB write that flushes L2, each timed on
-the device by its events (the events between stages give per-kernel times); a
+Timing: the step (the three stage calls) is captured once into a CUDA graph.
+W untimed warm-up replays; then K replays, each preceded by a 256 MiB write
+that flushes L2, each timed on the device by events around the replay; a
 barrier and a device synchronize bracket the timed region; the max over ranks
-is taken.  Under
+is taken.  Per-stage times (and the indexer's roofline) come from K more
+replays of a second graph with an event between the stages.  Under
 torchrun each rank runs its own batch on its own GPU (independent requests:
 weak scaling, no data-path collective).
 
@@ -155,15 +155,19 @@ def time_ours(args, wl, rank):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
-    # One step = the three stage calls, captured once into a CUDA graph with an
-    # event between stages, so the device timeline has no host gaps in it.
-    # Events recorded during capture become timing event nodes only with the
-    # runtime's "external" record flag.
+    # One step = the three stage calls, captured once into a CUDA graph.  The
+    # kernels are launched with programmatic stream serialization, so in the
+    # graph each may start while the one before it drains; events between the
+    # stages would cut those edges, so the step is timed from events around
+    # the replay, and a second graph with an event between stages gives the
+    # per-stage times (its own loop after the timed one).
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     cudart = ctypes.CDLL("libcudart.so.12")
     cudart.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
 
     def record(e, st, capturing):
+        # events recorded during capture become timing nodes only with the
+        # runtime's "external" record flag
         if capturing:
             rc = cudart.cudaEventRecordWithFlags(ctypes.c_void_p(e.cuda_event), ctypes.c_void_p(st.cuda_stream), 1)
             if rc != 0:
@@ -171,41 +175,62 @@ def time_ours(args, wl, rank):
         else:
             e.record(st)
 
-    def step(st, capturing=False):
-        record(ev[0], st, capturing)
+    def step(st, capturing=False, events=False):
+        if events:
+            record(ev[0], st, capturing)
         sml.sml_indexer_scores(p, lay.iq8, lay.iq_scale, lay.iw, dw.index_cache, scores, ws, st)
-        record(ev[1], st, capturing)
+        if events:
+            record(ev[1], st, capturing)
         sml.sml_topk(p, scores, idx, ln, ws, st)
-        record(ev[2], st, capturing)
+        if events:
+            record(ev[2], st, capturing)
         sml.sml_sparse_mla_decode(p, lay.q, dw.latent, idx, ln, out, lse, ws, st)
-        record(ev[3], st, capturing)
+        if events:
+            record(ev[3], st, capturing)
 
-    step(stream)                       # first calls outside capture (per-device set-up, events created)
+    step(stream, events=True)          # first calls outside capture (per-device set-up, events created)
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         step(torch.cuda.current_stream(), capturing=True)
+    graph_ev = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_ev):
+        step(torch.cuda.current_stream(), capturing=True, events=True)
     for _ in range(args.warmup):
         flush.fill_(1)
         graph.replay()
+        flush.fill_(1)
+        graph_ev.replay()
     torch.cuda.synchronize()
     code, bits = sml.sml_read_device_status(ws)
     if code != sml.SML_OK:
         raise RuntimeError(f"device status {code} bits {bits:#x}")
 
-    rows = []
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step_ms = []
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clocks:
         for _ in range(args.steps):
             flush.fill_(1)
+            t0.record(stream)
             graph.replay()
+            t1.record(stream)
             torch.cuda.synchronize()
-            rows.append([ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]), ev[2].elapsed_time(ev[3]),
-                         ev[0].elapsed_time(ev[3])])
+            step_ms.append(t0.elapsed_time(t1))
         barrier()
+        torch.cuda.synchronize()
+    # per-stage breakdown (the same steps with events between the stages)
+    rows = []
+    for _ in range(args.steps):
+        flush.fill_(1)
+        graph_ev.replay()
+        torch.cuda.synchronize()
+        rows.append([ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]), ev[2].elapsed_time(ev[3]),
+                     ev[0].elapsed_time(ev[3])])
     per = np.array(rows)
-    del graph
+    per = np.concatenate([per, np.array(step_ms)[:, None]], axis=1)
+    del graph, graph_ev
     code, bits = sml.sml_read_device_status(ws)
     if code != sml.SML_OK:
         raise RuntimeError(f"device status {code} bits {bits:#x}")
@@ -321,7 +346,8 @@ def main():
     wl = synth.SUITE[args.workload](seed=0)
     units = workload_units(wl)
     per, clocks, e2e_ms, h2d, d2h = time_ours(args, wl, rank)
-    ms_step = max_over_ranks(float(per[:, 3].mean()))
+    ms_step = max_over_ranks(float(per[:, 4].mean()))
+    ms_staged = max_over_ranks(float(per[:, 3].mean()))
     ms_idx = max_over_ranks(float(per[:, 0].mean()))
     ms_topk = max_over_ranks(float(per[:, 1].mean()))
     ms_mla = max_over_ranks(float(per[:, 2].mean()))
@@ -337,10 +363,11 @@ def main():
     line = {
         "metric": metric, "value": qps, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "e4m3/f16 products, f32 accumulate", "data": "synthetic",
+        "vs_baseline": None, "dtype": "e4m3 products (bf16 for the RoPE part), f32 accumulate", "data": "synthetic",
         "config": config_of(wl, args, world),
         "gathered_tokens_per_s": whole_job_rate(world, units["gathered"], ms_step),
-        "stage_ms": {"indexer": ms_idx, "topk": ms_topk, "sparse_mla_and_merge": ms_mla},
+        "stage_ms": {"indexer": ms_idx, "topk": ms_topk, "sparse_mla_and_merge": ms_mla,
+                     "step_with_stage_events": ms_staged},
         "indexer_hbm_gbs": idx_gbs, "indexer_frac_of_8000_gbs": idx_gbs / 8000.0,
         "mla_hbm_gbs": units["mla_bytes"] / (ms_mla / 1e3) / 1e9,
         "mla_tflops": units["mla_flops"] / (ms_mla / 1e3) / 1e12,

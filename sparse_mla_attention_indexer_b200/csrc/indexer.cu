@@ -264,10 +264,14 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     ptx::tmem_alloc(&S.tmem_base, kTmemCols);
     ptx::tmem_relinquish();
   }
+  ptx::griddep_wait();   // inputs may come from the previous kernel of the stream
   schedule<kThreads, kGroup>(P, S.red, S.sched);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
+  // This CTA holds its tensor memory now, so a dependent grid scheduled on the
+  // same SM cannot starve it of columns.
+  if (threadIdx.x == 0) ptx::griddep_launch_dependents();
   const int beg = S.sched[0], end = S.sched[1];
   volatile int* abort = &S.abort;
 
@@ -473,8 +477,8 @@ cudaError_t launch_cfg(const CUtensorMap& kmap, const CUtensorMap& qmap, const P
   const size_t smem = sizeof(Smem<C>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  indexer_tc_kernel<C><<<num_sms() * C::kCtasPerSm, C::kThreads, smem, stream>>>(kmap, qmap, P);
-  return cudaGetLastError();
+  return launch_pdl(indexer_tc_kernel<C>, dim3(num_sms() * C::kCtasPerSm), dim3(C::kThreads), smem, stream, 0,
+                    kmap, qmap, P);
 }
 
 }  // namespace

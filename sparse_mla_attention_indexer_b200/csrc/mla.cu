@@ -237,6 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, hg = blockIdx.y, t = blockIdx.z;
+  ptx::griddep_wait();   // the selection comes from the previous kernel
 
   // ---- this split's key range (uniform across the CTA) ----
   const int r = request_of_warp(P.cu_q, P.B, t);
@@ -284,6 +285,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
+  // This CTA holds its tensor memory now, so a dependent grid scheduled on the
+  // same SM cannot starve it of columns.
+  if (threadIdx.x == 0) ptx::griddep_launch_dependents();
   volatile int* abort = &S.abort;
   const uint32_t T0 = S.tmem_base;
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -612,6 +616,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
 __global__ void __launch_bounds__(128)
 lse_merge_kernel(int H, MlaWs ws, float* __restrict__ out, float* __restrict__ lse) {
   const int h = blockIdx.x, t = blockIdx.y, S = ws.splits;
+  if (threadIdx.x == 0) ptx::griddep_launch_dependents();
+  ptx::griddep_wait();   // the partials come from the previous kernel
   const size_t base = ((size_t)t * H + h) * S;
   float mx = -INFINITY;
   for (int s = 0; s < S; ++s) mx = fmaxf(mx, ws.part_lse[base + s]);
@@ -684,12 +690,11 @@ cudaError_t launch_sparse_mla(const sml_problem& p, const uint16_t* q, const uin
   const size_t smem = sizeof(Smem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(sparse_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(ws.splits, p.num_heads / kHC, p.num_tokens);
-  sparse_mla_tc_kernel<<<grid, kThreads, smem, stream>>>(P);
-  e = cudaGetLastError();
+  e = launch_pdl(sparse_mla_tc_kernel, dim3(ws.splits, p.num_heads / kHC, p.num_tokens), dim3(kThreads), smem,
+                 stream, 0, P);
   if (e != cudaSuccess) return e;
-  lse_merge_kernel<<<dim3(p.num_heads, p.num_tokens), 128, 0, stream>>>(p.num_heads, ws, out, lse);
-  return cudaGetLastError();
+  return launch_pdl(lse_merge_kernel, dim3(p.num_heads, p.num_tokens), dim3(128), 0, stream, 0, p.num_heads, ws, out,
+                    lse);
 }
 
 }  // namespace sml

@@ -1,5 +1,6 @@
 // Internal declarations shared by the libsml.so translation units.
 #pragma once
+#include <utility>
 
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -102,6 +103,36 @@ __device__ __forceinline__ Req load_request(const int32_t* __restrict__ cu_q,
   q.ok = q.q0 >= 0 && q.Q >= 1 && q.q0 <= T - q.Q && q.L >= q.Q && q.L <= max_ctx &&
          (q.L + SML_PAGE_TOKENS - 1) / SML_PAGE_TOKENS <= max_pages;
   return q;
+}
+
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel of the stream finishes, and reads nothing that
+// kernel may write before griddep_wait().  cluster_x > 0 also sets a cluster
+// of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[2];
+  int na = 0;
+  at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (cluster_x > 0) {
+    at[na].id = cudaLaunchAttributeClusterDimension;
+    at[na].val.clusterDim.x = (unsigned)cluster_x;
+    at[na].val.clusterDim.y = 1;
+    at[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = na;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // ---- launchers (one per kernel family; all enqueue on `stream`) --------------------

@@ -23,6 +23,7 @@
 //    finish (an arrival counter, no waiting) selects again over the
 //    concatenated candidates.  The global top-k is a subset of the union of
 //    the chunk top-ks, so the result is exact.
+#include "ptx.cuh"
 #include "sml_internal.cuh"
 
 namespace sml {
@@ -85,17 +86,17 @@ __device__ __forceinline__ int block_scan_incl(int v, int* warp_tot, int* total)
 // Over the histogram sh.hist[0, nb): the bin holding the `need`-th largest
 // element, and how many elements lie in the bins above it.
 template <typename Sh>
-__device__ __forceinline__ void find_bin(int nb, int need, Sh& sh, int* bin, int* above_out) {
+__device__ __forceinline__ void find_bin(int nb, int need, const int* hist, Sh& sh, int* bin, int* above_out) {
   const int tid = threadIdx.x, nt = blockDim.x;
   const int bpt = nb / nt;   // nb is a multiple of nt
   int local = 0;
-  for (int j = 0; j < bpt; ++j) local += sh.hist[nb - 1 - (tid * bpt + j)];
+  for (int j = 0; j < bpt; ++j) local += hist[nb - 1 - (tid * bpt + j)];
   int total;
   const int incl = block_scan_incl(local, sh.warp_a, &total);
   int above = incl - local;
   for (int j = 0; j < bpt; ++j) {
     const int b = nb - 1 - (tid * bpt + j);
-    const int h = sh.hist[b];
+    const int h = hist[b];
     if (above < need && need <= above + h) {
       sh.bcast[0] = b;
       sh.bcast[1] = above;
@@ -133,7 +134,7 @@ __device__ void radix_threshold(int n, int k, KeyAt key_at, Sh& sh, uint32_t* ta
     }
     __syncthreads();
     int b, above;
-    find_bin(nb, remaining, sh, &b, &above);
+    find_bin(nb, remaining, sh.hist, sh, &b, &above);
     remaining -= above;
     prefix |= (uint32_t)b << shift;
     pmask |= (uint32_t)(nb - 1) << shift;
@@ -392,6 +393,8 @@ topk_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32_t* __re
   __shared__ int is_last;
   const int tid = threadIdx.x, nt = blockDim.x;
   const int t = blockIdx.y, c = blockIdx.x;
+  if (tid == 0) ptx::griddep_launch_dependents();
+  ptx::griddep_wait();   // the scores come from the previous kernel
   const int r = request_of_warp(cu_q, B, t);
   const Req rq = load_request(cu_q, ctx_len, r, T, max_ctx, max_pages);
   const int q0 = rq.q0, Q = rq.Q, L = rq.L;
@@ -483,6 +486,8 @@ struct ClusterShared {
   uint32_t bkeys[kCandCap];        // this CTA's keys in the threshold bucket (read by the cluster)
   uint32_t gkeys[kCandCap];        // the cluster's keys in the threshold bucket
   int nbk;                         // this CTA's count of them (read by the cluster)
+  int above;                       // this CTA's keys in buckets above it (read by the cluster)
+  int nbq[kClusterMax], abq[kClusterMax];   // every CTA's nbk and above, copied here
   int sel[2];                      // this CTA's keys > tau and == tau (read by the cluster)
   int samp_hist[256];
   int warp_a[32], warp_b[32];
@@ -507,6 +512,11 @@ __device__ __forceinline__ uint32_t cluster_size() {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// Split form of cluster_sync: arrive once this CTA is done reading the others'
+// shared memory, wait before leaving (so no CTA's shared memory goes away
+// while another may still read it).
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 // Load a 32-bit word at `p`'s offset in the shared memory of cluster CTA `rank`.
 __device__ __forceinline__ uint32_t ld_cluster(const void* p, uint32_t rank) {
   uint32_t a, v;
@@ -515,46 +525,29 @@ __device__ __forceinline__ uint32_t ld_cluster(const void* p, uint32_t rank) {
   return v;
 }
 
-// S.gh = the sum over the cluster of every CTA's S.hist[0, nb).
+// S.gh = the sum over the cluster of every CTA's S.hist[0, nb).  The caller
+// passes a cluster barrier before any CTA rebuilds S.hist.
 __device__ __forceinline__ void cluster_hist_sum(ClusterShared& S, int nb, int C) {
   __syncthreads();
   cluster_sync();
-  for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+  // nb / blockDim.x bins per thread (2 or 4), every remote load in flight at once
+  constexpr int kPer = kBuckets / kTopkThreads;
+  uint32_t v[kPer][kClusterMax];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int b = threadIdx.x + u * kTopkThreads;
+#pragma unroll
+    for (int r = 0; r < kClusterMax; ++r) v[u][r] = (b < nb && r < C) ? ld_cluster(&S.hist[b], r) : 0u;
+  }
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int b = threadIdx.x + u * kTopkThreads;
     int s = 0;
-    for (int r = 0; r < C; ++r) s += (int)ld_cluster(&S.hist[b], r);
-    S.gh[b] = s;
+#pragma unroll
+    for (int r = 0; r < kClusterMax; ++r) s += (int)v[u][r];
+    if (b < nb) S.gh[b] = s;
   }
   __syncthreads();
-  cluster_sync();   // nobody rewrites its histogram before every CTA has read it
-}
-
-// Warp 0: over h[0, nb) the bin holding the `need`-th largest element and the
-// count above it, into S.bcast.
-__device__ __forceinline__ void find_bin_desc_warp(const int* h, int nb, int need, ClusterShared& S) {
-  const int lane = threadIdx.x & 31;
-  const int per = nb / 32;
-  const int top = nb - 1 - lane * per;
-  int local = 0;
-  for (int j = 0; j < per; ++j) local += h[top - j];
-  int incl = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  const int before = incl - local;
-  if (before < need && need <= incl) {
-    int above = before;
-    for (int j = 0; j < per; ++j) {
-      const int hh = h[top - j];
-      if (need <= above + hh) {
-        S.bcast[0] = top - j;
-        S.bcast[1] = above;
-        break;
-      }
-      above += hh;
-    }
-  }
 }
 
 __global__ void __launch_bounds__(kTopkThreads, 1)
@@ -567,6 +560,8 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
   const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
   const int C = (int)cluster_size(), c = (int)cluster_rank();
   const int t = blockIdx.y;
+  if (tid == 0) ptx::griddep_launch_dependents();
+  ptx::griddep_wait();   // the scores come from the previous kernel
   // Everything up to the first cluster barrier depends only on the row, so an
   // early return is taken by the whole cluster or by none of it.
   const int r = request_of_warp(cu_q, B, t);
@@ -597,8 +592,28 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
 
   // 1. this chunk's keys into shared memory; the row's sample straight from
   //    global memory (every CTA takes the same sample, so all agree on it).
+  if ((reinterpret_cast<uintptr_t>(row + c0) & 15) == 0) {
+    // 16-B loads, all of a thread's issued before any is used
+    const float4* src = reinterpret_cast<const float4*>(row + c0);
+    const int n4 = cn >> 2;
+    constexpr int kV = kTopkChunk / 4 / kTopkThreads;   // float4s per thread
+    float4 v[kV];
+#pragma unroll
+    for (int u = 0; u < kV; ++u) {
+      const int i = tid + u * nt;
+      v[u] = i < n4 ? __ldcg(src + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kV; ++u) {
+      const int i = tid + u * nt;
+      if (i < n4)
+        reinterpret_cast<uint4*>(keys)[i] = make_uint4(order_key(v[u].x), order_key(v[u].y), order_key(v[u].z), order_key(v[u].w));
+    }
+    for (int i = 4 * n4 + tid; i < cn; i += nt) keys[i] = order_key(__ldcg(row + c0 + i));
+  } else {
 #pragma unroll 8
-  for (int i = tid; i < cn; i += nt) keys[i] = order_key(__ldcg(row + c0 + i));
+    for (int i = tid; i < cn; i += nt) keys[i] = order_key(__ldcg(row + c0 + i));
+  }
   const int ns = min(kSample, n);
   float sv[kSample / kTopkThreads];
   float lo = INFINITY, hi = -INFINITY;
@@ -725,15 +740,27 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
     base_v = lo;
     scale = finite_range ? (float)(kBuckets - 3) / width : 0.f;
     __syncthreads();
+    cluster_sync();                  // every CTA has read this histogram before it is rebuilt
   }
-  // 4. the threshold bucket (the same in every CTA)
-  if (warp == 0) find_bin_desc_warp(S.gh, kBuckets, K, S);
+  // 4. the threshold bucket (the same in every CTA), and this CTA's count of
+  //    keys above it
   if (tid == 0) S.nbk = 0;
-  __syncthreads();
-  const int bk = S.bcast[0], need = K - S.bcast[1];
+  int bk, need;
+  {
+    int bin, above;
+    find_bin(kBuckets, K, S.gh, S, &bin, &above);
+    bk = bin;
+    need = K - above;
+  }
   const int wn = S.wcnt[warp];
-  // 5. this CTA's keys in the threshold bucket; tau = the need-th largest over
-  //    the cluster, take = how many keys equal to tau are selected.
+  {
+    int part = 0;
+    for (int b = bk + 1 + tid; b < kBuckets; b += nt) part += S.hist[b];
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) S.warp_b[warp] = part;
+  }
+  // 5. this CTA's keys in the threshold bucket, published with that count
   for (int j = lane; j < wn; j += 32) {
     const uint32_t key = keys[S.cpos[warp][j]];
     if (bucket(key) == bk) {
@@ -742,25 +769,42 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
     }
   }
   __syncthreads();
-  cluster_sync();
-  int nbt = 0, offs = 0;
+  if (tid == 0) {
+    int a = 0;
+    for (int w = 0; w < kWarps; ++w) a += S.warp_b[w];
+    S.above = a;
+  }
+  __syncthreads();
+  cluster_sync();   // also: every CTA is done reading the others' histograms
+  // every CTA's bucket-key count and count above, one round of remote loads
+  if (warp == 0 && lane < C) {
+    S.nbq[lane] = (int)ld_cluster(&S.nbk, lane);
+    S.abq[lane] = (int)ld_cluster(&S.above, lane);
+  }
+  __syncthreads();
+  int nbt = 0;
   bool fits = true;
   for (int q = 0; q < C; ++q) {
-    const int m = (int)ld_cluster(&S.nbk, q);
-    if (q < c) offs += m;
-    nbt += m;
-    fits = fits && m <= kCandCap;
+    nbt += S.nbq[q];
+    fits = fits && S.nbq[q] <= kCandCap;
   }
   fits = fits && nbt <= kCandCap;
+  // tau = the need-th largest key of the bucket over the cluster, take = how
+  // many keys equal to tau are selected; out0 = where this CTA's selection
+  // starts in the row's output, my_take = the ties this CTA may take (ties go
+  // to the lowest positions, so to the CTAs before this one first).
   uint32_t tau;
-  int take;
+  int take, out0 = 0, my_take = 0;
   if (fits) {
-    for (int q = 0, o = 0; q < C; ++q) {
-      const int m = (int)ld_cluster(&S.nbk, q);
-      for (int j = tid; j < m; j += nt) S.gkeys[o + j] = ld_cluster(&S.bkeys[j], q);
-      o += m;
+    // all the cluster's bucket keys, CTA by CTA: element i of the
+    // concatenation is key i - o_q of CTA q (o_q = the counts before q)
+    for (int i = tid; i < nbt; i += nt) {
+      int q = 0, o = 0;
+      while (i >= o + S.nbq[q]) o += S.nbq[q++];
+      S.gkeys[i] = ld_cluster(&S.bkeys[i - o], q);
     }
     __syncthreads();
+    cluster_arrive();   // done reading the other CTAs' shared memory: no remote access after this
     if (nbt <= kSmallCand) {
       if (tid < nbt) {
         const uint32_t key = S.gkeys[tid];
@@ -782,6 +826,31 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
       radix_threshold(nbt, need, [&](int i) { return S.gkeys[i]; }, S, &tau, &take);
     }
     __syncthreads();
+    if (warp == 0) {
+      // CTA q selects above_q + (its bucket keys > tau) + its share of the ties
+      int o = 0, eq_before = 0, off = 0;
+      for (int q = 0; q < c; ++q) {
+        const int m = S.nbq[q];
+        int gt = 0, eq = 0;
+        for (int j = lane; j < m; j += 32) {
+          const uint32_t x = S.gkeys[o + j];
+          gt += x > tau;
+          eq += x == tau;
+        }
+#pragma unroll
+        for (int w = 16; w >= 1; w >>= 1) {
+          gt += __shfl_xor_sync(0xffffffffu, gt, w);
+          eq += __shfl_xor_sync(0xffffffffu, eq, w);
+        }
+        off += S.abq[q] + gt + max(0, min(eq, take - eq_before));
+        eq_before += eq;
+        o += m;
+      }
+      if (lane == 0) {
+        S.bcast[0] = off;
+        S.bcast[1] = max(0, take - eq_before);
+      }
+    }
   } else {
     // Heavy ties: a radix select (11 / 11 / 10 key bits) over the threshold
     // bucket's keys where they lie, the histograms summed over the cluster.
@@ -797,17 +866,56 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
         if (bucket(key) == bk && (key & pmask) == prefix) atomicAdd(&S.hist[(key >> shift) & (uint32_t)(nb - 1)], 1);
       }
       cluster_hist_sum(S, nb, C);
-      if (warp == 0) find_bin_desc_warp(S.gh, nb, remaining, S);
-      __syncthreads();
-      remaining -= S.bcast[1];
-      prefix |= (uint32_t)S.bcast[0] << shift;
+      int b, above;
+      find_bin(nb, remaining, S.gh, S, &b, &above);
+      remaining -= above;
+      prefix |= (uint32_t)b << shift;
       pmask |= (uint32_t)(nb - 1) << shift;
-      __syncthreads();
+      cluster_sync();   // every CTA has read this histogram before it is rebuilt
     }
     tau = prefix;
     take = remaining;
+    // this CTA's counts of keys > tau and == tau, exchanged over the cluster
+    int cg = 0, ce = 0;
+    for (int j0 = 0; j0 < wn; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t key = j < wn ? keys[S.cpos[warp][j]] : 0u;
+      cg += __popc(__ballot_sync(0xffffffffu, j < wn && key > tau));
+      ce += __popc(__ballot_sync(0xffffffffu, j < wn && key == tau));
+    }
+    if (lane == 0) {
+      S.warp_a[warp] = cg;
+      S.warp_b[warp] = ce;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int a = 0, b = 0;
+      for (int w = 0; w < kWarps; ++w) {
+        a += S.warp_a[w];
+        b += S.warp_b[w];
+      }
+      S.sel[0] = a;
+      S.sel[1] = b;
+    }
+    __syncthreads();
+    cluster_sync();
+    if (tid == 0) {
+      int off = 0, eq_before = 0;
+      for (int q = 0; q < c; ++q) {
+        const int g = (int)ld_cluster(&S.sel[0], q), e = (int)ld_cluster(&S.sel[1], q);
+        off += g + max(0, min(e, take - eq_before));
+        eq_before += e;
+      }
+      S.bcast[0] = off;
+      S.bcast[1] = max(0, take - eq_before);
+    }
+    __syncthreads();
+    cluster_arrive();
   }
-  // 6. counts of keys > tau and == tau: per warp, per CTA, then over the cluster
+  __syncthreads();
+  out0 = S.bcast[0];
+  my_take = S.bcast[1];
+  // 6. this CTA's counts per warp (exclusive prefixes over the warps)
   int cgt = 0, ceq = 0;
   for (int j0 = 0; j0 < wn; j0 += 32) {
     const int j = j0 + lane;
@@ -815,6 +923,7 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
     cgt += __popc(__ballot_sync(0xffffffffu, j < wn && key > tau));
     ceq += __popc(__ballot_sync(0xffffffffu, j < wn && key == tau));
   }
+  __syncthreads();
   if (lane == 0) {
     S.warp_a[warp] = cgt;
     S.warp_b[warp] = ceq;
@@ -832,24 +941,11 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
       }
     }
     if (lane < kWarps) {
-      S.warp_a[lane] = a - a0;   // exclusive prefixes over the warps
+      S.warp_a[lane] = a - a0;
       S.warp_b[lane] = b - b0;
-    }
-    if (lane == kWarps - 1) {
-      S.sel[0] = a;
-      S.sel[1] = b;
     }
   }
   __syncthreads();
-  cluster_sync();
-  // ties go to the lowest positions: the CTAs before this one take theirs first
-  int out0 = 0, eq_before = 0;
-  for (int q = 0; q < c; ++q) {
-    const int g = (int)ld_cluster(&S.sel[0], q), e = (int)ld_cluster(&S.sel[1], q);
-    out0 += g + max(0, min(e, take - eq_before));
-    eq_before += e;
-  }
-  const int my_take = max(0, take - eq_before);   // ties this CTA may still take
   // 7. emission in position order
   int g = S.warp_a[warp], e = S.warp_b[warp];
   for (int j0 = 0; j0 < wn; j0 += 32) {
@@ -864,8 +960,7 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
     e += __popc(be);
   }
   if (c == 0 && tid == 0) idx_len[t] = K;
-  __syncthreads();
-  cluster_sync();   // shared memory stays until every CTA of the cluster is done reading it
+  cluster_wait();   // shared memory stays until every CTA of the cluster is done reading it
 }
 
 }  // namespace
@@ -877,32 +972,17 @@ cudaError_t launch_topk(const sml_problem& p, const float* scores, int32_t* idx,
     const size_t smem = (size_t)kTopkChunk * sizeof(uint32_t) + sizeof(ClusterShared);
     cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(ws.chunks, p.num_tokens);
-    cfg.blockDim = dim3(kTopkThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = ws.chunks;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, p.num_requests, p.num_tokens, p.topk, p.max_ctx,
-                           p.max_pages, p.cu_q, p.ctx_len, scores, idx, idx_len, status);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    return launch_pdl(topk_cluster_kernel, dim3(ws.chunks, p.num_tokens), dim3(kTopkThreads), smem, stream, ws.chunks,
+                      p.num_requests, p.num_tokens, p.topk, p.max_ctx, p.max_pages, p.cu_q, p.ctx_len, scores, idx,
+                      idx_len, status);
   }
   const size_t smem = (size_t)kTopkChunk * sizeof(uint32_t);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(ws.chunks, p.num_tokens);
-  topk_kernel<<<grid, kTopkThreads, smem, stream>>>(p.num_requests, p.num_tokens, p.topk,
-                                                    p.max_ctx, p.max_pages, p.cu_q, p.ctx_len,
-                                                    scores, idx, idx_len, ws, status);
-  return cudaGetLastError();
+  return launch_pdl(topk_kernel, dim3(ws.chunks, p.num_tokens), dim3(kTopkThreads), smem, stream, 0, p.num_requests,
+                    p.num_tokens, p.topk, p.max_ctx, p.max_pages, p.cu_q, p.ctx_len, scores, idx, idx_len, ws,
+                    status);
 }
 
 }  // namespace sml
