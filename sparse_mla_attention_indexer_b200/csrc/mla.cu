@@ -16,10 +16,11 @@
 // its N, and 16 heads as M would waste 3/4 of the smallest M).  Both products
 // run on kind::f8f6f4 straight from the gathered E4M3 latent tile: nothing of
 // the latent is ever converted.
-//   * warps 4-14 gather the selected 656-B rows with 16-B asynchronous copies
-//     (one row per warp instruction) into 128-B-swizzled tiles: E4M3 latent,
-//     bf16 RoPE key, block scales aside; two tile buffers.  Random rows need
-//     many requests in flight per SM, hence many gather warps;
+//   * warps 4-14 gather the selected 656-B rows, eight rows per warp batch
+//     (16-B register loads, one row per warp instruction), into
+//     128-B-swizzled tiles: E4M3 latent, bf16 RoPE key, block scales aside;
+//     two tile buffers.  Random rows need many loads in flight per SM, hence
+//     many gather warps and deep batches;
 //   * warp 15 issues the MMAs:
 //       S_b^T = C_b . [Qhi_b; Qlo_b]^T  (K-major; N = 32: both query terms),
 //       S_pe^T = K_pe . Q_pe^T          (kind::f16, bf16),
@@ -51,6 +52,9 @@ constexpr int kKT = 128;         // keys per tile
 constexpr int kMaxSplit = 512;   // keys per split (4 tiles)
 constexpr int kThreads = 512;    // warps 0-3 softmax, 4-14 gather, 15 MMA
 constexpr int kGatherWarps = 11;
+constexpr int kBatchRows = 8;                     // rows per gather batch (16 loads in flight per thread)
+constexpr int kBatchesPerTile = 128 / kBatchRows;  // >= kGatherWarps: every gather warp has a batch in every tile
+static_assert(kBatchesPerTile >= kGatherWarps, "a gather warp without a batch in a tile would never signal it");
 constexpr int kWarpMma = 15;
 constexpr float kLazyRescale = 8.f;   // nats
 
@@ -102,6 +106,15 @@ struct Params {
 // Byte address of (row, 16-B chunk) in a 128-B-swizzled tile of 128-B rows.
 __device__ __forceinline__ uint32_t sw128(uint32_t base, int row, int chunk) {
   return base + (row >> 3) * 1024 + (row & 7) * 128 + ((chunk ^ (row & 7)) << 4);
+}
+
+// 16-B global load that does not allocate in L1 (each row is read once).
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -266,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(&S.e_full[i], 32 * kGatherWarps);   // one arrival per gather thread, on completion of its copies
+      ptx::mbar_init(&S.e_full[i], kGatherWarps);   // one arrival per gather warp
       ptx::mbar_init(&S.e_free[i], 1);   // PV of the tile done (it is the tile's last reader)
     }
     ptx::mbar_init(&S.q_ready, 4);
@@ -314,33 +327,55 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
       S.rowid[k] = id;
     }
     asm volatile("bar.sync 2, %0;" ::"n"(kGT) : "memory");
-    // Rows -> tiles, one row per warp instruction: lane l copies latent chunk l
-    // (block l / 8, chunk l % 8), then lane 0 the four scales and lanes 1-8
-    // the RoPE key.  A masked row is zero-filled (nothing is read).  The
-    // tile's barrier completes when every gather thread's copies have landed,
-    // so the warps go straight on to the next tile: two tiles in flight.
+    // Rows -> tiles in batches of kBatchRows rows per warp (a tile is
+    // kKT / kBatchRows batches; batch i goes to warp i % kGatherWarps): the
+    // batch's loads go into registers first (lane l: 16-B latent chunk l, then
+    // lane 0 the four scales and lanes 1-8 the RoPE key), then the warp waits
+    // for the tile's buffer to be free and stores them 128-B-swizzled, so the
+    // loads are in flight while the buffer drains.  A masked row is zeros.  A
+    // warp signals a tile after storing its last batch of it.
     const int gw = warp - 4;
+    const int nb_total = ntiles * kBatchesPerTile;
     bool ok = true;
-    for (int tile = 0; tile < ntiles; ++tile) {
-      const int buf = tile & 1;
-      if (tile >= 2 && !warp_wait(&S.e_free[buf], ((tile >> 1) - 1) & 1, abort)) { ok = false; break; }
+    for (int bi = gw; bi < nb_total; bi += kGatherWarps) {
+      const int tile = bi / kBatchesPerTile, buf = tile & 1;
+      const int row0 = (bi % kBatchesPerTile) * kBatchRows;
+      uint4 va[kBatchRows], vb[kBatchRows];
+#pragma unroll
+      for (int u = 0; u < kBatchRows; ++u) {
+        const int32_t id = S.rowid[tile * kKT + row0 + u];
+        const uint8_t* src = P.latent + (size_t)(id >= 0 ? id : 0) * SML_LATENT_ROW_BYTES;
+        va[u] = make_uint4(0u, 0u, 0u, 0u);
+        vb[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (id >= 0) {
+          va[u] = ldg_stream(src + 16 * lane);
+          if (lane == 0 || (lane <= 8 && P.rope_dim)) vb[u] = ldg_stream(src + SML_LATENT_DIM + 16 * lane);
+        }
+      }
+      // first batch of this tile for this warp: the buffer must be free (PV of tile - 2 done)
+      if (tile >= 2 && bi - kGatherWarps < tile * kBatchesPerTile &&
+          !warp_wait(&S.e_free[buf], ((tile >> 1) - 1) & 1, abort)) {
+        ok = false;
+        break;
+      }
       const uint32_t lat_l = ptx::smem_u32(S.lat[buf][lane >> 3]);
       const uint32_t pe_b = ptx::smem_u32(S.pe[buf]);
       const uint32_t sc_b = ptx::smem_u32(&S.sc[buf][0][0]);
-      for (int row = gw; row < kKT; row += kGatherWarps) {
-        const int32_t id = S.rowid[tile * kKT + row];
-        const uint8_t* src = id >= 0 ? P.latent + (size_t)id * SML_LATENT_ROW_BYTES : P.latent;
-        const uint32_t nb = id >= 0 ? 16u : 0u;
-        ptx::cp_async16(sw128(lat_l, row, lane & 7), src + 16 * lane, nb);
+#pragma unroll
+      for (int u = 0; u < kBatchRows; ++u) {
+        const int row = row0 + u;
+        st_shared_v4(sw128(lat_l, row, lane & 7), va[u].x, va[u].y, va[u].z, va[u].w);
         if (lane == 0)
-          ptx::cp_async16(sc_b + row * 16, src + SML_LATENT_DIM, nb);
+          st_shared_v4(sc_b + row * 16, vb[u].x, vb[u].y, vb[u].z, vb[u].w);
         else if (lane <= 8 && P.rope_dim)
-          ptx::cp_async16(sw128(pe_b, row, lane - 1), src + SML_LATENT_DIM + 16 * lane, nb);
+          st_shared_v4(sw128(pe_b, row, lane - 1), vb[u].x, vb[u].y, vb[u].z, vb[u].w);
       }
-      // every gather thread arrives once its own copies of this tile have landed
-      ptx::cp_async_arrive_noinc(&S.e_full[buf]);
+      if (bi + kGatherWarps >= (tile + 1) * kBatchesPerTile) {   // this warp's last batch of the tile
+        ptx::fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&S.e_full[buf]);
+      }
     }
-    ptx::cp_async_wait_all();   // no copy may still be landing when the CTA ends
     if (!ok) *abort = 1;
   } else if (warp == kWarpMma) {
     // ================= MMA issuer =================
