@@ -280,7 +280,7 @@ class L2Flush:
 
     def __call__(self):
         self.wbuf.fill_(1)
-        torch.sum(self.rbuf, dtype=torch.int64, out=self.sink)
+        torch.sum(self.rbuf, dim=0, dtype=torch.int64, out=self.sink)
 
 
 def barrier():

@@ -16,11 +16,11 @@
 // its N, and 16 heads as M would waste 3/4 of the smallest M).  Both products
 // run on kind::f8f6f4 straight from the gathered E4M3 latent tile: nothing of
 // the latent is ever converted.
-//   * warps 4-14 gather the selected 656-B rows, 12 rows of each tile per
-//     warp (16 register loads of 16 B per lane, all in flight before any is
-//     stored), into 128-B-swizzled tiles: E4M3 latent, bf16 RoPE key, block
-//     scales aside; two tile buffers.  Random rows need many loads in flight
-//     per SM, hence many gather warps;
+//   * warps 4-14 gather the selected 656-B rows, eight rows per warp batch
+//     (16-B register loads, one row per warp instruction), into
+//     128-B-swizzled tiles: E4M3 latent, bf16 RoPE key, block scales aside;
+//     two tile buffers.  Random rows need many loads in flight per SM, hence
+//     many gather warps and deep batches;
 //   * warp 15 issues the MMAs:
 //       S_b^T = C_b . [Qhi_b; Qlo_b]^T  (K-major; N = 32: both query terms),
 //       S_pe^T = K_pe . Q_pe^T          (kind::f16, bf16),
@@ -52,11 +52,9 @@ constexpr int kKT = 128;         // keys per tile
 constexpr int kMaxSplit = 512;   // keys per split (4 tiles)
 constexpr int kThreads = 512;    // warps 0-3 softmax, 4-14 gather, 15 MMA
 constexpr int kGatherWarps = 11;
-constexpr int kBatchRows = 12;                   // rows of a tile per gather warp
-constexpr int kRowChunks = SML_LATENT_ROW_BYTES / 16;   // 41 16-B chunks per 656-B row
-constexpr int kLoadsPerLane = (kBatchRows * kRowChunks + 31) / 32;   // 16
-static_assert(kBatchRows * kGatherWarps >= 128 && kBatchRows * (kGatherWarps - 1) < 128,
-              "every gather warp owns rows of every tile");
+constexpr int kBatchRows = 8;                     // rows per gather batch (16 loads in flight per thread)
+constexpr int kBatchesPerTile = 128 / kBatchRows;  // >= kGatherWarps: every gather warp has a batch in every tile
+static_assert(kBatchesPerTile >= kGatherWarps, "a gather warp without a batch in a tile would never signal it");
 constexpr int kWarpMma = 15;
 constexpr float kLazyRescale = 8.f;   // nats
 
@@ -329,51 +327,54 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
       S.rowid[k] = id;
     }
     asm volatile("bar.sync 2, %0;" ::"n"(kGT) : "memory");
-    // Rows -> tiles: gather warp w owns rows [12 w, 12 w + 12) of every tile
-    // (the last warp the 8 left), 41 16-B chunks per row (32 latent chunks,
-    // the four scales, 8 RoPE chunks) laid end to end, so every lane's 16
-    // loads carry data.  The loads of a tile go into registers first; the
-    // warp then waits for the tile's buffer to be free (PV of tile - 2 done),
-    // stores them 128-B-swizzled and signals the tile.  A masked row is zeros.
+    // Rows -> tiles in batches of kBatchRows rows per warp (a tile is
+    // kKT / kBatchRows batches; batch i goes to warp i % kGatherWarps): the
+    // batch's loads go into registers first (lane l: 16-B latent chunk l, then
+    // lane 0 the four scales and lanes 1-8 the RoPE key), then the warp waits
+    // for the tile's buffer to be free and stores them 128-B-swizzled, so the
+    // loads are in flight while the buffer drains.  A masked row is zeros.  A
+    // warp signals a tile after storing its last batch of it.
     const int gw = warp - 4;
-    const int row0 = gw * kBatchRows;
-    const int nrows = min(kBatchRows, kKT - row0);
-    const int nchunks = nrows * kRowChunks;
+    const int nb_total = ntiles * kBatchesPerTile;
     bool ok = true;
-    for (int tile = 0; tile < ntiles; ++tile) {
-      const int buf = tile & 1;
-      uint4 v[kLoadsPerLane];
+    for (int bi = gw; bi < nb_total; bi += kGatherWarps) {
+      const int tile = bi / kBatchesPerTile, buf = tile & 1;
+      const int row0 = (bi % kBatchesPerTile) * kBatchRows;
+      uint4 va[kBatchRows], vb[kBatchRows];
 #pragma unroll
-      for (int j = 0; j < kLoadsPerLane; ++j) {
-        const int c = lane + 32 * j;
-        const int rr = c / kRowChunks, cc = c - rr * kRowChunks;
-        v[j] = make_uint4(0u, 0u, 0u, 0u);
-        if (c < nchunks && (cc <= 32 || P.rope_dim)) {
-          const int32_t id = S.rowid[tile * kKT + row0 + rr];
-          if (id >= 0) v[j] = ldg_stream(P.latent + (size_t)id * SML_LATENT_ROW_BYTES + 16 * cc);
+      for (int u = 0; u < kBatchRows; ++u) {
+        const int32_t id = S.rowid[tile * kKT + row0 + u];
+        const uint8_t* src = P.latent + (size_t)(id >= 0 ? id : 0) * SML_LATENT_ROW_BYTES;
+        va[u] = make_uint4(0u, 0u, 0u, 0u);
+        vb[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (id >= 0) {
+          va[u] = ldg_stream(src + 16 * lane);
+          if (lane == 0 || (lane <= 8 && P.rope_dim)) vb[u] = ldg_stream(src + SML_LATENT_DIM + 16 * lane);
         }
       }
-      if (tile >= 2 && !warp_wait(&S.e_free[buf], ((tile >> 1) - 1) & 1, abort)) {
+      // first batch of this tile for this warp: the buffer must be free (PV of tile - 2 done)
+      if (tile >= 2 && bi - kGatherWarps < tile * kBatchesPerTile &&
+          !warp_wait(&S.e_free[buf], ((tile >> 1) - 1) & 1, abort)) {
         ok = false;
         break;
       }
+      const uint32_t lat_l = ptx::smem_u32(S.lat[buf][lane >> 3]);
+      const uint32_t pe_b = ptx::smem_u32(S.pe[buf]);
+      const uint32_t sc_b = ptx::smem_u32(&S.sc[buf][0][0]);
 #pragma unroll
-      for (int j = 0; j < kLoadsPerLane; ++j) {
-        const int c = lane + 32 * j;
-        const int rr = c / kRowChunks, cc = c - rr * kRowChunks;
-        if (c < nchunks) {
-          const int row = row0 + rr;
-          if (cc < 32)
-            st_shared_v4(sw128(ptx::smem_u32(S.lat[buf][cc >> 3]), row, cc & 7), v[j].x, v[j].y, v[j].z, v[j].w);
-          else if (cc == 32)
-            st_shared_v4(ptx::smem_u32(&S.sc[buf][row][0]), v[j].x, v[j].y, v[j].z, v[j].w);
-          else if (P.rope_dim)
-            st_shared_v4(sw128(ptx::smem_u32(S.pe[buf]), row, cc - 33), v[j].x, v[j].y, v[j].z, v[j].w);
-        }
+      for (int u = 0; u < kBatchRows; ++u) {
+        const int row = row0 + u;
+        st_shared_v4(sw128(lat_l, row, lane & 7), va[u].x, va[u].y, va[u].z, va[u].w);
+        if (lane == 0)
+          st_shared_v4(sc_b + row * 16, vb[u].x, vb[u].y, vb[u].z, vb[u].w);
+        else if (lane <= 8 && P.rope_dim)
+          st_shared_v4(sw128(pe_b, row, lane - 1), vb[u].x, vb[u].y, vb[u].z, vb[u].w);
       }
-      ptx::fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&S.e_full[buf]);
+      if (bi + kGatherWarps >= (tile + 1) * kBatchesPerTile) {   // this warp's last batch of the tile
+        ptx::fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&S.e_full[buf]);
+      }
     }
     if (!ok) *abort = 1;
   } else if (warp == kWarpMma) {
