@@ -184,6 +184,35 @@ __device__ __forceinline__ int block_scan(int v, int* red, int* sum) {
 // per kThreads requests instead of one dependent load chain per request.
 template <int kThreads, int kGroup>
 __device__ void schedule(const Params& P, int* red, int* out /* beg, end, r0, off0 */) {
+  if (P.B <= kThreads) {
+    // One request per thread: one round of loads and one scan give both the
+    // total and where this CTA's share starts.
+    Walker<kGroup> w{&P};
+    w.r = threadIdx.x;
+    int cnt = 0;
+    if (w.r < P.B) {
+      w.load_req();
+      if (!w.rq.ok && blockIdx.x == 0) raise_fault(P.status, SML_FAULT_LENGTHS);
+      cnt = w.request_items();
+    }
+    int total;
+    const int incl = block_scan<kThreads>(cnt, red, &total);
+    const long long G = gridDim.x;
+    const int beg = (int)((long long)total * blockIdx.x / G);
+    const int end = (int)((long long)total * (blockIdx.x + 1) / G);
+    if (threadIdx.x == 0) {
+      out[0] = beg;
+      out[1] = end;
+      out[2] = P.B;
+      out[3] = 0;
+    }
+    __syncthreads();
+    if (beg < end && cnt > 0 && beg >= incl - cnt && beg < incl) {
+      out[2] = w.r;
+      out[3] = beg - (incl - cnt);
+    }
+    return;
+  }
   int total = 0;
   for (int base = 0; base < P.B; base += kThreads) {
     Walker<kGroup> w{&P};
