@@ -8,6 +8,8 @@
 #include <math.h>
 #include <stdio.h>
 
+#include <map>
+#include <mutex>
 #include <string>
 
 #include "sml_internal.cuh"
@@ -167,6 +169,34 @@ int cuda_fail(cudaError_t e, const char* fn) {
 }
 
 }  // namespace
+
+int device_sm_count() {
+  static std::mutex mu;
+  static int count[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> g(mu);
+  if (count[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    count[dev] = n > 0 ? n : 148;
+  }
+  return count[dev];
+}
+
+cudaError_t set_max_smem(const void* func, size_t bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, size_t> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> g(mu);
+  size_t& have = done[{func, dev}];
+  if (have >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) have = bytes;
+  return e;
+}
 
 size_t topk_region_bytes(const sml_problem& p) { return layout(p, SML_STAGE_TOPK).total; }
 size_t mla_region_bytes(const sml_problem& p) { return layout(p, SML_STAGE_MLA).total; }

@@ -26,6 +26,8 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 
+#include <mutex>
+
 #include "ptx.cuh"
 #include "sml_internal.cuh"
 
@@ -494,19 +496,42 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-int num_sms() {
-  int dev = 0, n = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
-}
+// Encoded tensor maps depend only on the address, the shape and the device:
+// the last few are kept so that a call with the same caches and batch shape
+// (every decode step) does not re-encode them.
+struct MapCache {
+  struct Entry {
+    const void* base;
+    int64_t n;
+    int dev;
+    CUtensorMap map;
+  };
+  std::mutex mu;
+  Entry e[8] = {};
+  int next = 0;
+  template <typename Encode>
+  bool get(const void* base, int64_t n, CUtensorMap* out, Encode&& encode) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> g(mu);
+    for (const Entry& x : e)
+      if (x.base == base && x.n == n && x.dev == dev && base != nullptr) {
+        *out = x.map;
+        return true;
+      }
+    if (!encode(out)) return false;
+    e[next] = Entry{base, n, dev, *out};
+    next = (next + 1) % 8;
+    return true;
+  }
+};
 
 template <class C>
 cudaError_t launch_cfg(const CUtensorMap& kmap, const CUtensorMap& qmap, const Params& P, cudaStream_t stream) {
   const size_t smem = sizeof(Smem<C>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(indexer_tc_kernel<C>), smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(indexer_tc_kernel<C>, dim3(num_sms() * C::kCtasPerSm), dim3(C::kThreads), smem, stream, 0,
+  return launch_pdl(indexer_tc_kernel<C>, dim3(device_sm_count() * C::kCtasPerSm), dim3(C::kThreads), smem, stream, 0,
                     kmap, qmap, P);
 }
 
@@ -518,28 +543,29 @@ cudaError_t launch_indexer(const sml_problem& p, const uint8_t* iq8, const float
   auto enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap kmap, qmap;
-  {
+  static MapCache kcache, qcache;
+  const bool kok = kcache.get(index_base, index_pages, &kmap, [&](CUtensorMap* m) {
     // The pool as [pages][64 rows][128 B]: one box = the 64 keys of one page.
     cuuint64_t dims[3] = {SML_INDEX_DIM, SML_PAGE_TOKENS, (cuuint64_t)index_pages};
     cuuint64_t strides[2] = {SML_INDEX_DIM, SML_INDEX_PAGE_BYTES};
     cuuint32_t box[3] = {SML_INDEX_DIM, SML_PAGE_TOKENS, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    if (enc(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(index_base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
-  {
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(index_base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  });
+  if (!kok) return cudaErrorInvalidValue;
+  const bool qok = qcache.get(iq8, p.num_tokens, &qmap, [&](CUtensorMap* m) {
     // Indexer queries as [T * 64 rows][128 B]: one box = the 64 heads of a token.
     cuuint64_t dims[2] = {SML_INDEX_DIM, (cuuint64_t)p.num_tokens * SML_INDEX_HEADS};
     cuuint64_t strides[1] = {SML_INDEX_DIM};
     cuuint32_t box[2] = {SML_INDEX_DIM, SML_INDEX_HEADS};
     cuuint32_t estr[2] = {1, 1};
-    if (enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(iq8), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(iq8), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  });
+  if (!qok) return cudaErrorInvalidValue;
   Params P;
   P.B = p.num_requests;
   P.T = p.num_tokens;

@@ -723,7 +723,7 @@ cudaError_t launch_sparse_mla(const sml_problem& p, const uint16_t* q, const uin
   P.ws = ws;
   P.status = status;
   const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(sparse_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(sparse_mla_tc_kernel), smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(sparse_mla_tc_kernel, dim3(ws.splits, p.num_heads / kHC, p.num_tokens), dim3(kThreads), smem,
                  stream, 0, P);

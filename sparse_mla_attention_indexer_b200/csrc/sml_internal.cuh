@@ -105,6 +105,11 @@ __device__ __forceinline__ Req load_request(const int32_t* __restrict__ cu_q,
   return q;
 }
 
+// Host-side per-device caches for the launchers (thread-safe): the SM count,
+// and the dynamic shared-memory attribute, set once per kernel and device.
+int device_sm_count();
+cudaError_t set_max_smem(const void* func, size_t bytes);
+
 // Launch with programmatic stream serialization: the kernel may be scheduled
 // while the previous kernel of the stream finishes, and reads nothing that
 // kernel may write before griddep_wait().  cluster_x > 0 also sets a cluster

@@ -970,15 +970,14 @@ cudaError_t launch_topk(const sml_problem& p, const float* scores, int32_t* idx,
   if (ws.chunks <= kClusterMax) {
     // one cluster of ws.chunks CTAs per row
     const size_t smem = (size_t)kTopkChunk * sizeof(uint32_t) + sizeof(ClusterShared);
-    cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_max_smem(reinterpret_cast<const void*>(topk_cluster_kernel), smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(topk_cluster_kernel, dim3(ws.chunks, p.num_tokens), dim3(kTopkThreads), smem, stream, ws.chunks,
                       p.num_requests, p.num_tokens, p.topk, p.max_ctx, p.max_pages, p.cu_q, p.ctx_len, scores, idx,
                       idx_len, status);
   }
   const size_t smem = (size_t)kTopkChunk * sizeof(uint32_t);
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(topk_kernel), smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(topk_kernel, dim3(ws.chunks, p.num_tokens), dim3(kTopkThreads), smem, stream, 0, p.num_requests,
                     p.num_tokens, p.topk, p.max_ctx, p.max_pages, p.cu_q, p.ctx_len, scores, idx, idx_len, ws,
