@@ -12,9 +12,10 @@ Modules:
   formats -- E4M3 / bf16 decoding and the paged cache byte layouts
   dsa     -- indexer scores, visible lengths, exact top-k
   mla     -- absorbed-query attention, sparse and dense MLA, LSE merge, one layer
+  producers -- FP8 quantisation and the cache writes just before the step
 
 Every function is pinned by tests under ``tests/`` (``-m "not gpu"``) to
 values the pages print, closed forms, invariants, library routines and brute
 force on tiny inputs; none is "parity unpinned".
 """
-from . import dsa, formats, mla  # noqa: F401
+from . import dsa, formats, mla, producers  # noqa: F401

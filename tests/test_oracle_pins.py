@@ -380,3 +380,129 @@ def test_ssmax_factor_one_is_ssmax_off(small):
     a = mla.run_layer(v_on, small.latent, small.index_cache, tokens=[0])
     b = mla.run_layer(v_off, small.latent, small.index_cache, tokens=[0])
     assert np.array_equal(a[0][0], b[0][0]) and np.allclose(a[1], b[1], rtol=1e-12)
+
+
+# --- producers: FP8 quantisation and cache writes ---------------------------------
+
+from oracle import producers as PR  # noqa: E402
+
+
+def _torch_e4m3(x: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_e4m3_encode_round_trips_every_finite_code():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    vals = F.decode_e4m3(codes).astype(np.float32)
+    assert np.array_equal(PR.e4m3_encode(vals), codes)
+
+
+def test_e4m3_encode_ties_go_to_the_even_code():
+    # midpoint between every pair of neighbouring finite magnitudes
+    mags = F.decode_e4m3(np.arange(0x7F, dtype=np.uint8))
+    mids = ((mags[:-1] + mags[1:]) / 2).astype(np.float32)
+    assert np.array_equal(mids.astype(np.float64), (mags[:-1] + mags[1:]) / 2)   # exact in fp32
+    got = PR.e4m3_encode(mids).astype(int)
+    lo = np.arange(0x7E)
+    want = np.where(lo % 2 == 0, lo, lo + 1)
+    assert np.array_equal(got, want)
+    assert np.array_equal(PR.e4m3_encode(-mids).astype(int), want | 0x80)
+
+
+def test_e4m3_encode_matches_torch_cast_and_brute_force_nearest():
+    rng = synth.stream(5, "e4m3_encode")
+    x = (rng.standard_normal(20000) * np.exp2(rng.uniform(-14, 9, 20000))).astype(np.float32)
+    x = x[np.abs(x) < 464]                        # torch's cast has no saturation past 464
+    got = PR.e4m3_encode(x)
+    assert np.array_equal(got, _torch_e4m3(x))
+    # brute force over every finite code: the chosen value is a nearest one
+    finite = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    vals = F.decode_e4m3(finite)
+    sub = x[:2000].astype(np.float64)
+    best = np.abs(vals[None, :] - sub[:, None]).min(axis=1)
+    assert np.array_equal(np.abs(F.decode_e4m3(got[:2000]) - sub), best)
+
+
+def test_e4m3_encode_saturates_and_keeps_signed_zero():
+    x = np.array([448.0, 463.9, 464.0, 1e4, 3e38, -500.0, 0.0, -0.0], dtype=np.float32)
+    assert PR.e4m3_encode(x).tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0x00, 0x80]
+
+
+def test_quantise_block_invariants():
+    rng = synth.stream(6, "quant_block")
+    for scale_exp in (-30, -3, 0, 5, 30):
+        x = (rng.standard_normal(128) * 2.0 ** scale_exp).astype(np.float32)
+        codes, s = PR.quantise_block(x)
+        assert s.dtype == np.float32 and s > 0
+        # the block's largest magnitude lands on the largest finite code
+        assert codes[np.argmax(np.abs(x))] & 0x7F == 0x7E
+        back = F.decode_e4m3(codes) * float(s)
+        bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * float(s)) * (1 + 1e-6)
+        assert np.all(np.abs(back - x) <= bound)
+    codes, s = PR.quantise_block(np.zeros(128, dtype=np.float32))
+    assert s == 1.0 and not codes.any()
+    codes, s = PR.quantise_block(np.array([-0.0, 0.0], dtype=np.float32))
+    assert s == 1.0 and codes.tolist() == [0x80, 0x00]
+
+
+def test_quantiser_agrees_with_the_torch_based_generator():
+    # synth.quantise_rows quantises with PyTorch's cast: an independent implementation
+    x = synth.stream(7, "gen_vs_oracle").standard_normal((32, 512), dtype=np.float32)
+    gcodes, gscale = synth.quantise_rows(x, 128)
+    for i in range(32):
+        for b in range(4):
+            codes, s = PR.quantise_block(x[i, b * 128:(b + 1) * 128])
+            assert s == gscale[i, b]
+            assert np.array_equal(codes, gcodes[i, b * 128:(b + 1) * 128])
+
+
+def test_cache_writes_read_back_through_the_layout_readers():
+    rng = synth.stream(8, "writes")
+    n, pages = 40, 3
+    slot = rng.permutation(pages * 64)[:n].astype(np.int32)
+    slot[5] = -1
+    c = synth.to_bf16_bits(rng.standard_normal((n, 512)).astype(np.float32))
+    kpe = synth.to_bf16_bits(rng.standard_normal((n, 64)).astype(np.float32))
+    k = synth.to_bf16_bits(rng.standard_normal((n, 128)).astype(np.float32))
+    lat0 = rng.integers(0, 256, pages * F.LATENT_PAGE_BYTES, dtype=np.uint8)
+    idx0 = rng.integers(0, 256, pages * F.INDEXER_PAGE_BYTES, dtype=np.uint8)
+    lat, bad1 = PR.write_latent(lat0, c, kpe, slot)
+    idx, bad2 = PR.write_indexer_k(idx0, k, slot)
+    assert not bad1 and not bad2
+    w = slot >= 0
+    c_hat, pe = F.latent_rows(lat, slot[w] // 64, slot[w] % 64)
+    cx = F.decode_bf16(c[w])
+    assert np.array_equal(pe, F.decode_bf16(kpe[w]))
+    bound = np.maximum(np.abs(cx) * 2.0 ** -4, 2.0 ** -10 * np.abs(cx).reshape(-1, 4, 128).max(2).repeat(128, 1) / 448)
+    assert np.all(np.abs(c_hat - cx) <= bound * (1 + 1e-6))
+    kh = F.indexer_keys(idx, slot[w] // 64, slot[w] % 64)
+    kx = F.decode_bf16(k[w])
+    kb = np.maximum(np.abs(kx) * 2.0 ** -4, 2.0 ** -10 * np.abs(kx).max(1, keepdims=True) / 448)
+    assert np.all(np.abs(kh - kx) <= kb * (1 + 1e-6))
+    # rows of other slots are untouched; the skipped token wrote nothing
+    lat_rows = np.zeros(pages * 64, bool)
+    lat_rows[slot[w]] = True
+    lr = lat.reshape(pages * 64, F.LATENT_ROW_BYTES)
+    assert np.array_equal(lr[~lat_rows], lat0.reshape(pages * 64, -1)[~lat_rows])
+    keys = idx.reshape(pages, -1)[:, :F.INDEXER_KEYS_BYTES].reshape(pages * 64, 128)
+    keys0 = idx0.reshape(pages, -1)[:, :F.INDEXER_KEYS_BYTES].reshape(pages * 64, 128)
+    assert np.array_equal(keys[~lat_rows], keys0[~lat_rows])
+    # a NoPE row stores a zero RoPE key; an out-of-range slot is reported, not written
+    lat2, bad = PR.write_latent(lat0, c[:2], None, np.array([7, pages * 64], dtype=np.int32))
+    assert bad
+    _, pe2 = F.latent_rows(lat2, [0], [7])
+    assert not pe2.any()
+    assert np.array_equal(lat2[F.LATENT_ROW_BYTES * 8:], lat0[F.LATENT_ROW_BYTES * 8:])
+
+
+def test_indexer_q_quantisation_is_one_block_per_token():
+    rng = synth.stream(9, "iq")
+    iq = synth.to_bf16_bits((rng.standard_normal((3, 64, 128)) * np.array([1e-3, 1.0, 50.0])[:, None, None])
+                            .astype(np.float32))
+    codes, scales = PR.quantise_indexer_q(iq)
+    x = F.decode_bf16(iq)
+    for t in range(3):
+        assert scales[t] == np.float32(np.float32(np.abs(x[t]).max()) / np.float32(448))
+        assert (codes[t] & 0x7F).max() == 0x7E
+        back = F.decode_e4m3(codes[t]) * float(scales[t])
+        assert np.all(np.abs(back - x[t]) <= np.maximum(np.abs(x[t]) * 2.0 ** -4, 2.0 ** -10 * float(scales[t])) * (1 + 1e-6))
