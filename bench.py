@@ -285,6 +285,64 @@ def time_ours(args, wl, rank):
     return per, clocks.summary(), float(np.mean(e2e_ms)), h2d, d2h
 
 
+# Algorithmic bytes per new token of the producers: bf16 inputs and the int32
+# slot read, codes, scales and the copied RoPE key written.
+PRODUCER_BYTES = {
+    "indexer_k_cache_write": 128 * 2 + 4 + 128 + 4,
+    "latent_cache_write": 512 * 2 + 64 * 2 + 4 + 656,
+    "indexer_q_quant": 64 * 128 * 2 + 64 * 128 + 4,
+}
+
+
+def time_producers(decode_tokens: int, iters: int, peak: float):
+    """The producers that fill the caches before a step, each timed alone with
+    events on its stream after an L2 flush: at the decode batch (one new token
+    per query token of the workload) and at a bulk batch (16,384 new tokens, a
+    prefill chunk's 2,048 indexer queries), into separate pools of 1,024 pages
+    at random distinct slots."""
+    flush = L2Flush()
+    st = torch.cuda.current_stream()
+    pages = 1024
+    lat = torch.zeros(pages * synth.LATENT_PAGE, dtype=torch.uint8, device="cuda")
+    idx = torch.zeros(pages * synth.INDEX_PAGE, dtype=torch.uint8, device="cuda")
+
+    def bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+
+    def run(n_cache, n_q):
+        slot = torch.from_numpy(synth.producer_slots(11, f"bench/slot/{n_cache}", n_cache, pages)).cuda()
+        k = bf16(synth.producer_rows(11, "bench/k", n_cache, 128, spread=False))
+        c = bf16(synth.producer_rows(11, "bench/c", n_cache, 512, spread=False))
+        kpe = bf16(synth.producer_rows(11, "bench/kpe", n_cache, 64, spread=False))
+        iq = bf16(synth.producer_rows(11, "bench/iq", n_q, 64 * 128, spread=False))
+        iq8 = torch.empty(n_q * 64 * 128, dtype=torch.uint8, device="cuda")
+        iqs = torch.empty(n_q, dtype=torch.float32, device="cuda")
+        calls = {
+            "indexer_k_cache_write": (n_cache, lambda: sml.sml_indexer_k_cache_write(k, slot, idx, None, st)),
+            "latent_cache_write": (n_cache, lambda: sml.sml_latent_cache_write(c, kpe, slot, lat, None, st)),
+            "indexer_q_quant": (n_q, lambda: sml.sml_indexer_q_quant(iq, iq8, iqs, st)),
+        }
+        res = {}
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for name, (n, call) in calls.items():
+            ms = []
+            for i in range(iters + 3):
+                flush()
+                e0.record(st)
+                call()
+                e1.record(st)
+                st.synchronize()
+                if i >= 3:
+                    ms.append(e0.elapsed_time(e1))
+            t = float(np.mean(ms))
+            gbs = n * PRODUCER_BYTES[name] / (t / 1e3) / 1e9
+            res[name] = {"tokens": n, "us": t * 1e3, "gbs": gbs, "frac": gbs / peak}
+        return res
+
+    return {"decode_batch": run(decode_tokens, decode_tokens), "bulk": run(16384, 2048),
+            "bytes_per_token": PRODUCER_BYTES}
+
+
 class L2Flush:
     """Before every step: write a 256 MiB buffer (evicts everything the last
     step left in the 126 MB L2), then read another 256 MiB buffer, so the dirty
@@ -394,6 +452,7 @@ def main():
     ms_mla = max_over_ranks(float(per[:, 2].mean()))
     e2e_ms = max_over_ranks(e2e_ms)
     peak, peak_kind = peaks()
+    producers = time_producers(wl.T, args.steps, peak) if rank == 0 else None
     cb = cpu_baseline(wl) if rank == 0 and world == 1 else None
     if world > 1:
         torch.distributed.destroy_process_group()
@@ -421,6 +480,7 @@ def main():
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "entry_point": "sml_run_layer"},
         "gpu_launches": args.steps * 4,
         "cpu_baseline": cb,
+        "producers": producers,
     }
     print(json.dumps(line))
 

@@ -11,6 +11,10 @@
  *                          selected keys, then a log-sum-exp merge)
  *   sml_run_layer          the three in a row, or only the attention for a
  *                          shared-indexer layer that reuses a prior top-k
+ *   sml_indexer_k_cache_write, sml_latent_cache_write, sml_indexer_q_quant
+ *                          the producers just before the step: FP8
+ *                          quantisation of new tokens into the two caches,
+ *                          and of the indexer queries
  *
  * Sources: vLLM blog "vLLM 首日支持 Mistral Large 4：1T 参数 MoE 多模态模型",
  * highlights list (MLA with KV LoRA rank 512 and RoPE dim 64; a DSA indexer
@@ -207,6 +211,43 @@ int sml_run_layer(const sml_problem* p, const void* q, const void* iq8, const fl
 int sml_sparse_mla_decode_noalloc(const sml_problem* p, const void* q, sml_cache latent,
                                   const int32_t* idx, const int32_t* idx_len, float* out, float* lse,
                                   void* stream);
+
+/* ---- producers: quantise new tokens and write the caches the step reads ----
+ *
+ * vLLM blog "vLLM 首日支持 Mistral Large 4", paragraph "可断开的 CUDA 图和融合":
+ * the first round of hand-written fusions covers the indexer Q path and the
+ * indexer K path, and the decode round writes the indexer K straight into the
+ * FP8 cache; section "实现细节 / 模型架构": the step reads an fp8_ds_mla latent
+ * cache and an FP8 indexer cache.  Reading (the pages print no quantiser):
+ * a block x is stored as E4M3 codes of q = x / s, s = amax|x| / 448 (s = 1
+ * when amax = 0), s and q in fp32 (IEEE division), each code the nearest E4M3
+ * value to q with ties to the even code and magnitudes past 448 clamped to
+ * 448.  Blocks: 128 latent values (four per row), one 128-value indexer key,
+ * one query token's 64 x 128 indexer values.  Inputs must be finite.
+ *
+ * slot[i] = physical page * 64 + row of new token i (int32, device); -1 skips
+ * the token.  A slot outside [-1, num_pages * 64) is skipped and, when
+ * `workspace` is not NULL (any initialised workspace, >= 256 B), sets
+ * SML_FAULT_PAGE in its status word.  Two tokens with the same slot race.
+ * n = 0 is a no-op.  Rows that no slot names are left untouched. */
+
+/* Indexer K path: k [n, 128] bf16 (16-B aligned) -> 128 e4m3 codes at
+ * page*8448 + row*128 and the fp32 scale at page*8448 + 8192 + row*4. */
+int sml_indexer_k_cache_write(const void* k, const int32_t* slot, int32_t n, sml_cache index_cache,
+                              void* workspace, void* stream);
+
+/* fp8_ds_mla latent write: c [n, 512] bf16 and k_pe [n, 64] bf16 (both 16-B
+ * aligned; k_pe NULL for a NoPE layer, whose rows get a zero RoPE key) ->
+ * the 656-B row at page*41984 + row*656: [512 e4m3][4 fp32 block scales]
+ * [64 bf16 k_pe]. */
+int sml_latent_cache_write(const void* c, const void* k_pe, const int32_t* slot, int32_t n,
+                           sml_cache latent, void* workspace, void* stream);
+
+/* Indexer Q path: iq [T, 64, 128] bf16 (16-B aligned) -> iq8 [T, 64, 128]
+ * e4m3 codes (16-B aligned) and iq_scale [T] fp32, one block per token: the
+ * inputs of sml_indexer_scores.  The indexer's SSMax factor is not folded in
+ * here; sml_indexer_scores applies it. */
+int sml_indexer_q_quant(const void* iq, int32_t num_tokens, void* iq8, float* iq_scale, void* stream);
 
 /* Synchronise `stream`, then return SML_OK, SML_ERR_DEVICE_FAULT or
  * SML_ERR_TIMEOUT from the workspace's sticky status word (its SML_FAULT_*

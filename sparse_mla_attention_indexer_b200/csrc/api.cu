@@ -330,6 +330,61 @@ int sml_run_layer(const sml_problem* p, const void* q, const void* iq8, const fl
   return e == cudaSuccess ? SML_OK : cuda_fail(e, "sml_run_layer");
 }
 
+// ---- producers ------------------------------------------------------------------
+
+namespace {
+
+void check_producer(Checker& c, int32_t n, const int32_t* slot, sml_cache cache, const char* what,
+                    int64_t max_pages, void* workspace) {
+  c.check(n >= 0, SML_ERR_INVALID_ARG, "n < 0");
+  c.check(n == 0 || (slot != nullptr && aligned(slot, 4)), SML_ERR_INVALID_ARG, "slot NULL or not 4-B aligned");
+  check_cache(c, cache, what);
+  c.check(cache.num_pages <= max_pages, SML_ERR_UNSUPPORTED, "num_pages * 64 slots exceed int32");
+  c.check(workspace == nullptr || aligned(workspace, 256), SML_ERR_WORKSPACE, "workspace not 256-B aligned");
+}
+
+constexpr int64_t kMaxSlotPages = ((int64_t)1 << 31) / SML_PAGE_TOKENS;
+
+}  // namespace
+
+int sml_indexer_k_cache_write(const void* k, const int32_t* slot, int32_t n, sml_cache index_cache,
+                              void* workspace, void* stream) {
+  Checker c;
+  check_producer(c, n, slot, index_cache, "index_cache", kMaxSlotPages, workspace);
+  c.check(n == 0 || (k != nullptr && aligned(k, 16)), SML_ERR_INVALID_ARG, "k NULL or not 16-B aligned");
+  if (c.done("sml_indexer_k_cache_write") != SML_OK) return c.code;
+  cudaError_t e = launch_indexer_k_write(k, slot, n, const_cast<void*>(index_cache.base), index_cache.num_pages,
+                                         workspace ? status_of(workspace) : nullptr,
+                                         static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SML_OK : cuda_fail(e, "sml_indexer_k_cache_write");
+}
+
+int sml_latent_cache_write(const void* cl, const void* k_pe, const int32_t* slot, int32_t n, sml_cache latent,
+                           void* workspace, void* stream) {
+  Checker c;
+  check_producer(c, n, slot, latent, "latent", kMaxSlotPages, workspace);
+  c.check(n == 0 || (cl != nullptr && aligned(cl, 16)), SML_ERR_INVALID_ARG, "c NULL or not 16-B aligned");
+  c.check(aligned(k_pe, 16), SML_ERR_INVALID_ARG, "k_pe not 16-B aligned");
+  if (c.done("sml_latent_cache_write") != SML_OK) return c.code;
+  cudaError_t e = launch_latent_write(cl, k_pe, slot, n, const_cast<void*>(latent.base), latent.num_pages,
+                                      workspace ? status_of(workspace) : nullptr,
+                                      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SML_OK : cuda_fail(e, "sml_latent_cache_write");
+}
+
+int sml_indexer_q_quant(const void* iq, int32_t num_tokens, void* iq8, float* iq_scale, void* stream) {
+  Checker c;
+  c.check(num_tokens >= 0, SML_ERR_INVALID_ARG, "num_tokens < 0");
+  const bool any = num_tokens > 0;
+  c.check(!any || (iq != nullptr && aligned(iq, 16)), SML_ERR_INVALID_ARG, "iq NULL or not 16-B aligned");
+  c.check(!any || (iq8 != nullptr && aligned(iq8, 16)), SML_ERR_INVALID_ARG, "iq8 NULL or not 16-B aligned");
+  c.check(!any || (iq_scale != nullptr && aligned(iq_scale, 4)), SML_ERR_INVALID_ARG,
+          "iq_scale NULL or not 4-B aligned");
+  if (c.done("sml_indexer_q_quant") != SML_OK) return c.code;
+  cudaError_t e = launch_indexer_q_quant(iq, num_tokens, iq8, iq_scale, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SML_OK : cuda_fail(e, "sml_indexer_q_quant");
+}
+
 int sml_read_device_status(void* workspace, int clear, int32_t* bits, void* stream) {
   Checker c;
   c.check(workspace != nullptr, SML_ERR_WORKSPACE, "workspace is NULL");

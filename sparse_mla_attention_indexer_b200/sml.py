@@ -92,11 +92,15 @@ def lib() -> ctypes.CDLL:
         L.sml_sparse_mla_decode_noalloc.argtypes = [pp, vp, Cache, vp, vp, vp, vp, vp]
         L.sml_run_layer.argtypes = [pp, vp, vp, vp, vp, Cache, Cache, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sml_read_device_status.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_int32), vp]
+        L.sml_indexer_k_cache_write.argtypes = [vp, vp, ctypes.c_int32, Cache, vp, vp]
+        L.sml_latent_cache_write.argtypes = [vp, vp, vp, ctypes.c_int32, Cache, vp, vp]
+        L.sml_indexer_q_quant.argtypes = [vp, ctypes.c_int32, vp, vp, vp]
         L.sml_status_string.argtypes = [i32]
         for name in ("sml_status_string", "sml_last_error", "sml_version"):
             getattr(L, name).restype = ctypes.c_char_p
         for name in ("sml_workspace_init", "sml_indexer_scores", "sml_topk", "sml_sparse_mla_decode",
-                     "sml_sparse_mla_decode_noalloc", "sml_run_layer", "sml_read_device_status"):
+                     "sml_sparse_mla_decode_noalloc", "sml_run_layer", "sml_read_device_status",
+                     "sml_indexer_k_cache_write", "sml_latent_cache_write", "sml_indexer_q_quant"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -122,6 +126,10 @@ def _s(stream) -> int | None:
     if isinstance(stream, int):
         return stream
     return stream.cuda_stream
+
+
+def _numel(x) -> int:
+    return 0 if x is None else int(x.numel())
 
 
 def _check(code: int):
@@ -195,6 +203,24 @@ def sml_run_layer(problem, q, iq8, iq_scale, iw, latent, index_cache, reuse_idx,
                                cache(latent, LATENT_PAGE_BYTES), cache(index_cache, INDEX_PAGE_BYTES),
                                _p(reuse_idx), _p(reuse_len), _p(idx_out), _p(len_out), _p(out),
                                _p(lse), _p(workspace), _nbytes(workspace), _s(stream)))
+
+
+def sml_indexer_k_cache_write(k, slot, index_cache, workspace=None, stream=None):
+    """Quantise new indexer keys k [n, 128] bf16 into the indexer cache at slot [n] int32."""
+    _check(lib().sml_indexer_k_cache_write(_p(k), _p(slot), _numel(slot), cache(index_cache, INDEX_PAGE_BYTES),
+                                           _p(workspace), _s(stream)))
+
+
+def sml_latent_cache_write(c, k_pe, slot, latent, workspace=None, stream=None):
+    """Quantise new latent rows c [n, 512] bf16 (+ k_pe [n, 64] bf16, or None) into the
+    fp8_ds_mla cache at slot [n] int32."""
+    _check(lib().sml_latent_cache_write(_p(c), _p(k_pe), _p(slot), _numel(slot), cache(latent, LATENT_PAGE_BYTES),
+                                        _p(workspace), _s(stream)))
+
+
+def sml_indexer_q_quant(iq, iq8, iq_scale, stream=None):
+    """Indexer queries iq [T, 64, 128] bf16 -> iq8 (e4m3 codes, uint8) and iq_scale [T] fp32."""
+    _check(lib().sml_indexer_q_quant(_p(iq), _numel(iq_scale), _p(iq8), _p(iq_scale), _s(stream)))
 
 
 def sml_read_device_status(workspace, clear: bool = True, stream=None):

@@ -273,3 +273,35 @@ SUITE = {
     "long_context": long_context,
     "prefill_chunk": prefill_chunk,
 }
+
+
+# --- inputs of the producers (new tokens before they enter the caches) ---------
+
+def producer_rows(seed: int, name: str, n: int, dim: int, spread: bool = True) -> np.ndarray:
+    """bf16 bits [n, dim] of new tokens' values, N(0, 1) per element.
+
+    ``spread``: each row is also multiplied by 2^U(-24, 24), and the first rows
+    are the special cases a quantiser meets: all zeros, all negative zeros, one
+    non-zero element, values near bf16's largest and smallest normal magnitudes,
+    and a row with a single element far above the rest."""
+    rng = stream(seed, name)
+    x = rng.standard_normal((n, dim), dtype=np.float32)
+    if spread:
+        x *= np.exp2(rng.uniform(-24, 24, size=(n, 1))).astype(np.float32)
+        special = [np.zeros(dim, np.float32), -np.zeros(dim, np.float32),
+                   np.eye(1, dim, dim // 3, dtype=np.float32)[0] * -3.0,
+                   x[0] / np.abs(x[0]).max() * np.float32(3.0e38),
+                   x[0] / np.abs(x[0]).max() * np.float32(2.0e-38),
+                   np.where(np.arange(dim) == 7, np.float32(1e4), x[0] / np.abs(x[0]).max())]
+        for i, row in enumerate(special[:n]):
+            x[i] = row
+    return to_bf16_bits(x)
+
+
+def producer_slots(seed: int, name: str, n: int, num_pages: int, skip_every: int = 0) -> np.ndarray:
+    """n distinct slots (page * 64 + row) of a num_pages pool, in random order;
+    every skip_every-th one is -1 (a padding token)."""
+    slot = stream(seed, name).permutation(num_pages * PAGE)[:n].astype(np.int32)
+    if skip_every:
+        slot[::skip_every] = -1
+    return slot

@@ -73,3 +73,21 @@ def test_unsupported_only_when_nothing_is_invalid(L):
     code = L.sml_topk(ctypes.byref(p), 0x1000, 0x2000, 0x3000, 0x100, 1 << 30, None)
     assert code == sml.SML_ERR_UNSUPPORTED
     assert sml.sml_status_string(code) == "unsupported shape or option"
+
+
+def test_producers_reject_bad_arguments_without_cuda(L):
+    code = L.sml_indexer_k_cache_write(0x1008, None, 4, sml.Cache(0x1001, 0), 0x80, None)
+    assert code == sml.SML_ERR_INVALID_ARG
+    msg = sml.sml_last_error()
+    for part in ("k NULL or not 16-B aligned", "slot", "index_cache.base", "num_pages"):
+        assert part in msg, msg
+    code = L.sml_latent_cache_write(None, 0x1004, 0x2000, -1, sml.Cache(0x10000, 1 << 40), None, None)
+    assert code == sml.SML_ERR_INVALID_ARG
+    msg = sml.sml_last_error()
+    for part in ("n < 0", "k_pe not 16-B aligned", "exceed int32"):
+        assert part in msg, msg
+    code = L.sml_indexer_q_quant(0x1000, 5, None, 0x2002, None)
+    assert code == sml.SML_ERR_INVALID_ARG
+    assert "iq8" in sml.sml_last_error() and "iq_scale" in sml.sml_last_error()
+    # empty batches need no buffers
+    assert L.sml_indexer_q_quant(None, 0, None, None, None) == sml.SML_OK
