@@ -10,11 +10,14 @@
 // saturation (the hardware conversion), so a code is a pure function of the
 // block's bf16 bits.
 //
-// All three are streaming copies with a little arithmetic: one warp per new
-// token for the two cache writes (the key's or the row's 128-B / 512-B
-// stores are one coalesced transaction per warp, at a slot the block table
-// scatters anywhere in the pool), one CTA per query token for the 16-KB
-// indexer query; grids are a few CTAs per SM with grid-stride loops.
+// All three are streaming copies with a little arithmetic, bound by how many
+// bytes are in flight: every thread issues all of its loads before it uses
+// any of them (the slot check does not hold back the data load).  The cache writes take two new
+// tokens per warp (a token's 128-B key or 512-B codes are one coalesced store
+// per warp, at a slot the block table scatters anywhere in the pool); the
+// query quantiser takes one 16-KB token per 256-thread CTA (its loads are all
+// in flight at once; staging them through shared memory with bulk copies
+// measured slower).
 #include <cuda_fp8.h>
 
 #include "ptx.cuh"
@@ -24,6 +27,7 @@ namespace sml {
 namespace {
 
 constexpr int kWarpsPerCta = 8;
+constexpr int kTokPerWarp = 2;
 constexpr float kE4m3Max = 448.f;
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -55,54 +59,78 @@ __device__ __forceinline__ bool slot_ok(int s, long long slots, int lane, int32_
   return false;
 }
 
-// One warp per new token: 128 bf16 in (256 B), 128 codes + one scale out.
+// Two new tokens per warp: 128 bf16 in (256 B) and 128 codes + one scale out each.
 __global__ void __launch_bounds__(32 * kWarpsPerCta)
 indexer_k_write_kernel(const uint2* __restrict__ k, const int32_t* __restrict__ slot, int n,
                        uint8_t* __restrict__ cache, long long slots, int32_t* status) {
   ptx::griddep_wait();
   if (threadIdx.x == 0) ptx::griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
-  for (int i = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); i < n; i += gridDim.x * kWarpsPerCta) {
-    const int s = __ldg(slot + i);
-    if (!slot_ok(s, slots, lane, status)) continue;
-    const uint2 v = __ldg(k + (size_t)i * (SML_INDEX_DIM / 4) + lane);
-    float a = fmaxf(absmax2(v.x), absmax2(v.y));
+  const int step = gridDim.x * kWarpsPerCta * kTokPerWarp;
+  for (int i0 = (blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5)) * kTokPerWarp; i0 < n; i0 += step) {
+    int s[kTokPerWarp];
+    uint2 v[kTokPerWarp];
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    const float sc = block_scale(a);
-    uint8_t* page = cache + (size_t)(s / SML_PAGE_TOKENS) * SML_INDEX_PAGE_BYTES;
-    const int row = s % SML_PAGE_TOKENS;
-    reinterpret_cast<uint32_t*>(page + row * SML_INDEX_DIM)[lane] = quant2(v.x, sc) | (quant2(v.y, sc) << 16);
-    if (lane == 0) reinterpret_cast<float*>(page + SML_PAGE_TOKENS * SML_INDEX_DIM)[row] = sc;
+    for (int u = 0; u < kTokPerWarp; ++u) {
+      const int i = i0 + u;
+      s[u] = i < n ? __ldg(slot + i) : -1;
+      if (i < n) v[u] = __ldg(k + (size_t)i * (SML_INDEX_DIM / 4) + lane);
+    }
+#pragma unroll
+    for (int u = 0; u < kTokPerWarp; ++u) {
+      if (!slot_ok(s[u], slots, lane, status)) continue;
+      float a = fmaxf(absmax2(v[u].x), absmax2(v[u].y));
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      const float sc = block_scale(a);
+      uint8_t* page = cache + (size_t)(s[u] / SML_PAGE_TOKENS) * SML_INDEX_PAGE_BYTES;
+      const int row = s[u] % SML_PAGE_TOKENS;
+      reinterpret_cast<uint32_t*>(page + row * SML_INDEX_DIM)[lane] =
+          quant2(v[u].x, sc) | (quant2(v[u].y, sc) << 16);
+      if (lane == 0) reinterpret_cast<float*>(page + SML_PAGE_TOKENS * SML_INDEX_DIM)[row] = sc;
+    }
   }
 }
 
-// One warp per new token: lane l quantises latent values [16 l, 16 l + 16),
-// eight lanes per 128-value block; lanes 0..7 copy the 128-B RoPE key.
+// Two new tokens per warp: lane l quantises latent values [16 l, 16 l + 16)
+// of each, eight lanes per 128-value block; lanes 0..7 copy the 128-B RoPE key.
 __global__ void __launch_bounds__(32 * kWarpsPerCta)
 latent_write_kernel(const uint4* __restrict__ c, const uint4* __restrict__ kpe, const int32_t* __restrict__ slot,
                     int n, uint8_t* __restrict__ cache, long long slots, int32_t* status) {
   ptx::griddep_wait();
   if (threadIdx.x == 0) ptx::griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
-  for (int i = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); i < n; i += gridDim.x * kWarpsPerCta) {
-    const int s = __ldg(slot + i);
-    if (!slot_ok(s, slots, lane, status)) continue;
-    const uint4* src = c + (size_t)i * (SML_LATENT_DIM / 8) + 2 * lane;
-    const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-    float a = fmaxf(fmaxf(fmaxf(absmax2(v0.x), absmax2(v0.y)), fmaxf(absmax2(v0.z), absmax2(v0.w))),
-                    fmaxf(fmaxf(absmax2(v1.x), absmax2(v1.y)), fmaxf(absmax2(v1.z), absmax2(v1.w))));
+  const int step = gridDim.x * kWarpsPerCta * kTokPerWarp;
+  for (int i0 = (blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5)) * kTokPerWarp; i0 < n; i0 += step) {
+    int s[kTokPerWarp];
+    uint4 v0[kTokPerWarp], v1[kTokPerWarp], pe[kTokPerWarp];
 #pragma unroll
-    for (int o = 4; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    const float sc = block_scale(a);
-    uint8_t* row = cache + (size_t)(s / SML_PAGE_TOKENS) * SML_LATENT_PAGE_BYTES +
-                   (size_t)(s % SML_PAGE_TOKENS) * SML_LATENT_ROW_BYTES;
-    const uint2 q0 = quant8(v0, sc), q1 = quant8(v1, sc);
-    reinterpret_cast<uint4*>(row)[lane] = make_uint4(q0.x, q0.y, q1.x, q1.y);
-    if ((lane & 7) == 0) reinterpret_cast<float*>(row + SML_LATENT_DIM)[lane >> 3] = sc;
-    if (lane < 8) {
-      const uint4 pe = kpe ? __ldg(kpe + (size_t)i * (SML_ROPE_DIM / 8) + lane) : make_uint4(0, 0, 0, 0);
-      reinterpret_cast<uint4*>(row + SML_LATENT_DIM + 16)[lane] = pe;
+    for (int u = 0; u < kTokPerWarp; ++u) {
+      const int i = i0 + u;
+      s[u] = i < n ? __ldg(slot + i) : -1;
+      pe[u] = make_uint4(0, 0, 0, 0);
+      if (i < n) {
+        const uint4* src = c + (size_t)i * (SML_LATENT_DIM / 8) + 2 * lane;
+        v0[u] = __ldg(src);
+        v1[u] = __ldg(src + 1);
+        if (kpe && lane < 8) pe[u] = __ldg(kpe + (size_t)i * (SML_ROPE_DIM / 8) + lane);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kTokPerWarp; ++u) {
+      if (!slot_ok(s[u], slots, lane, status)) continue;
+      const uint4 a0 = v0[u], a1 = v1[u];
+      float a = fmaxf(fmaxf(fmaxf(absmax2(a0.x), absmax2(a0.y)), fmaxf(absmax2(a0.z), absmax2(a0.w))),
+                      fmaxf(fmaxf(absmax2(a1.x), absmax2(a1.y)), fmaxf(absmax2(a1.z), absmax2(a1.w))));
+#pragma unroll
+      for (int o = 4; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      const float sc = block_scale(a);
+      uint8_t* row = cache + (size_t)(s[u] / SML_PAGE_TOKENS) * SML_LATENT_PAGE_BYTES +
+                     (size_t)(s[u] % SML_PAGE_TOKENS) * SML_LATENT_ROW_BYTES;
+      const uint2 q0 = quant8(a0, sc), q1 = quant8(a1, sc);
+      reinterpret_cast<uint4*>(row)[lane] = make_uint4(q0.x, q0.y, q1.x, q1.y);
+      if ((lane & 7) == 0) reinterpret_cast<float*>(row + SML_LATENT_DIM)[lane >> 3] = sc;
+      if (lane < 8) reinterpret_cast<uint4*>(row + SML_LATENT_DIM + 16)[lane] = pe[u];
     }
   }
 }
@@ -151,7 +179,7 @@ int token_grid(int n, int per_cta, int ctas_per_sm) {
 cudaError_t launch_indexer_k_write(const void* k, const int32_t* slot, int n, void* cache, int64_t num_pages,
                                    int32_t* status, cudaStream_t stream) {
   if (n == 0) return cudaSuccess;
-  return launch_pdl(indexer_k_write_kernel, dim3(token_grid(n, kWarpsPerCta, 8)), dim3(32 * kWarpsPerCta), 0,
+  return launch_pdl(indexer_k_write_kernel, dim3(token_grid(n, kWarpsPerCta * kTokPerWarp, 8)), dim3(32 * kWarpsPerCta), 0,
                     stream, 0, static_cast<const uint2*>(k), slot, n, static_cast<uint8_t*>(cache),
                     (long long)num_pages * SML_PAGE_TOKENS, status);
 }
@@ -159,7 +187,7 @@ cudaError_t launch_indexer_k_write(const void* k, const int32_t* slot, int n, vo
 cudaError_t launch_latent_write(const void* c, const void* kpe, const int32_t* slot, int n, void* cache,
                                 int64_t num_pages, int32_t* status, cudaStream_t stream) {
   if (n == 0) return cudaSuccess;
-  return launch_pdl(latent_write_kernel, dim3(token_grid(n, kWarpsPerCta, 8)), dim3(32 * kWarpsPerCta), 0,
+  return launch_pdl(latent_write_kernel, dim3(token_grid(n, kWarpsPerCta * kTokPerWarp, 8)), dim3(32 * kWarpsPerCta), 0,
                     stream, 0, static_cast<const uint4*>(c), static_cast<const uint4*>(kpe), slot, n,
                     static_cast<uint8_t*>(cache), (long long)num_pages * SML_PAGE_TOKENS, status);
 }
