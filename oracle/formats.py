@@ -35,6 +35,8 @@ NaN only for exponent and mantissa fields all ones.
 """
 from __future__ import annotations
 
+from typing import NamedTuple
+
 import numpy as np
 
 # --- sizes fixed by the pages -------------------------------------------------
@@ -89,11 +91,14 @@ def _le_f32(raw: np.ndarray) -> np.ndarray:
     return raw.view("<f4").astype(np.float64)
 
 
-def latent_rows(cache: np.ndarray, pages: np.ndarray, rows: np.ndarray):
-    """Read latent rows (physical page, row in page) from an fp8_ds_mla pool.
+def latent_rows(cache, pages: np.ndarray, rows: np.ndarray):
+    """Read latent rows (physical page, row in page) from an fp8_ds_mla pool
+    (uint8 bytes) or a ``PlainE4M3Pool``.
 
     Returns (c_hat [n, 512] = e4m3 * block scale, k_pe [n, 64]) in float64.
     """
+    if isinstance(cache, PlainE4M3Pool):
+        return plain_e4m3_rows(cache, pages, rows)
     pages = np.asarray(pages, dtype=np.int64)
     rows = np.asarray(rows, dtype=np.int64)
     start = pages * LATENT_PAGE_BYTES + rows * LATENT_ROW_BYTES
@@ -115,6 +120,30 @@ def indexer_keys(cache: np.ndarray, pages: np.ndarray, rows: np.ndarray) -> np.n
     sstart = pages * INDEXER_PAGE_BYTES + INDEXER_KEYS_BYTES + rows * 4
     scale = _le_f32(cache[sstart[:, None] + np.arange(4)[None, :]])[:, 0]
     return decode_e4m3(codes) * scale[:, None]
+
+
+PLAIN_E4M3_PAGE_BYTES = PAGE_TOKENS * PLAIN_E4M3_ROW_BYTES          # 36,864
+
+
+class PlainE4M3Pool(NamedTuple):
+    """A latent pool in the plain per-tensor E4M3 format (blog, section "ROCm
+    实现细节", paragraph "FP8 潜在缓存": all 576 latent dims stored as FP8 with
+    one per-tensor scale, 576 B per token).  Reading: a row is [512 x e4m3
+    latent][64 x e4m3 RoPE key], a page 64 rows back to back, and ``scale``
+    the pool's fp32 scale."""
+    data: np.ndarray
+    scale: float
+
+
+def plain_e4m3_rows(pool: PlainE4M3Pool, pages: np.ndarray, rows: np.ndarray):
+    """Read latent rows from a plain E4M3 pool: (c_hat [n, 512], k_pe [n, 64]),
+    every code times the pool scale, in float64."""
+    pages = np.asarray(pages, dtype=np.int64)
+    rows = np.asarray(rows, dtype=np.int64)
+    start = pages * PLAIN_E4M3_PAGE_BYTES + rows * PLAIN_E4M3_ROW_BYTES
+    raw = pool.data[start[:, None] + np.arange(PLAIN_E4M3_ROW_BYTES)[None, :]]
+    v = decode_e4m3(raw) * float(np.float32(pool.scale))
+    return v[:, :LATENT_DIM], v[:, LATENT_DIM:]
 
 
 def physical(block_table_row: np.ndarray, positions: np.ndarray):

@@ -37,7 +37,8 @@ Readings (the pages print no quantiser):
   passes none and its 128 B are zero.
 
 Byte layouts: those of ``formats`` (fp8_ds_mla row [512 x e4m3][4 x fp32]
-[64 x bf16]; indexer page [64 x 128 B keys][64 x fp32 scales]).
+[64 x bf16]; plain E4M3 row [576 x e4m3] under one pool scale that the caller
+gives; indexer page [64 x 128 B keys][64 x fp32 scales]).
 """
 from __future__ import annotations
 
@@ -135,3 +136,25 @@ def quantise_indexer_q(iq_bits: np.ndarray):
     for t in range(iq.shape[0]):
         codes[t], scales[t] = quantise_block(iq[t])
     return codes, scales
+
+
+def write_latent_plain_e4m3(pool: F.PlainE4M3Pool, c_bits: np.ndarray, kpe_bits, slot: np.ndarray):
+    """Latent rows (bf16 bits [n, 512]) and RoPE keys (bf16 bits [n, 64], or
+    None: zero codes) into a copy of a plain E4M3 pool: every value's code is
+    that of fp32(x) / scale, with the pool's given per-tensor scale (blog,
+    section "ROCm 实现细节", paragraph "FP8 潜在缓存").  Returns (new pool, any
+    slot out of range)."""
+    out = np.array(pool.data, dtype=np.uint8, copy=True)
+    num_pages = out.size // F.PLAIN_E4M3_PAGE_BYTES
+    ids, pages, rows, bad = _slots(slot, num_pages)
+    s = np.float32(pool.scale)
+    c = F.decode_bf16(c_bits).astype(np.float32)
+    pe = F.decode_bf16(kpe_bits).astype(np.float32) if kpe_bits is not None else None
+    for i, p, r in zip(ids, pages, rows):
+        row = np.zeros(F.PLAIN_E4M3_ROW_BYTES, dtype=np.uint8)
+        row[:F.LATENT_DIM] = e4m3_encode((c[i] / s).astype(np.float32))
+        if pe is not None:
+            row[F.LATENT_DIM:] = e4m3_encode((pe[i] / s).astype(np.float32))
+        start = p * F.PLAIN_E4M3_PAGE_BYTES + r * F.PLAIN_E4M3_ROW_BYTES
+        out[start: start + F.PLAIN_E4M3_ROW_BYTES] = row
+    return F.PlainE4M3Pool(out, float(s)), bad

@@ -35,6 +35,9 @@ import torch
 PAGE = 64
 LATENT_ROW = 656
 LATENT_PAGE = PAGE * LATENT_ROW
+PLAIN_ROW = 576                      # plain per-tensor E4M3 latent row
+PLAIN_PAGE = PAGE * PLAIN_ROW
+PLAIN_SCALE = 8.0 / 448.0            # pool scale of plain E4M3 latents: N(0, 1) values within +-8
 INDEX_PAGE = PAGE * 132
 E4M3_MAX = 448.0
 
@@ -93,6 +96,8 @@ class Workload:
     ssmax_s: float = 0.4
     ssmax_s_index: float = 0.4
     sm_scale: float = 1.0 / math.sqrt(576.0)
+    latent_format: str = "fp8_ds_mla"   # or "e4m3": 576-B rows under one pool scale
+    latent_scale: float = 0.0
 
     @property
     def B(self):
@@ -168,7 +173,7 @@ def _fill_index(seed: int, name: str, num_pages: int, chunk_pages: int = 2048) -
 
 def _scribble_tails(wl: Workload, rng: np.random.Generator):
     """Random bytes in the unused rows of each request's last page."""
-    lat = wl.latent.reshape(wl.num_pages, PAGE, LATENT_ROW)
+    lat = wl.latent.reshape(wl.num_pages, PAGE, PLAIN_ROW if wl.latent_format == "e4m3" else LATENT_ROW)
     idx = wl.index_cache.reshape(wl.num_pages, INDEX_PAGE)
     for r in range(wl.B):
         L = int(wl.ctx_len[r])
@@ -194,13 +199,28 @@ def make_layer(seed: int, tag: str, T: int, H: int, rope_dim: int, with_indexer:
     return lay
 
 
+def _fill_plain(seed: int, name: str, num_pages: int, chunk_pages: int = 512) -> np.ndarray:
+    """Plain E4M3 latent pool: 576 values N(0, 1) per row (512 latent, 64 RoPE),
+    codes of x / PLAIN_SCALE."""
+    out = np.empty((num_pages, PLAIN_PAGE), dtype=np.uint8)
+
+    def fill(i, p0, p1):
+        x = stream(seed, f"{name}/plain/{i}").standard_normal(((p1 - p0) * PAGE, PLAIN_ROW), dtype=np.float32)
+        out[p0:p1] = to_e4m3(x / np.float32(PLAIN_SCALE)).reshape(p1 - p0, PLAIN_PAGE)
+
+    _chunked(num_pages, chunk_pages, fill)
+    return out.reshape(-1)
+
+
 def make_workload(name: str, ctx_len, q_count, num_heads: int, topk: int = 2048,
                   layers=(("rope", 64, True, None),), permuted: bool = True, ssmax: bool = False,
-                  seed: int = 0, extra_pages: int = 0) -> Workload:
+                  seed: int = 0, extra_pages: int = 0, latent_format: str = "fp8_ds_mla") -> Workload:
     """Build a batch of requests with the given context lengths and query counts.
 
     ``layers``: tuples (tag, rope_dim, with_indexer, reuse_from).
     ``extra_pages``: unused pages appended to the pool (random bytes).
+    ``latent_format``: "fp8_ds_mla" (656-B rows) or "e4m3" (576-B rows, one
+    pool scale PLAIN_SCALE).
     """
     ctx_len = np.asarray(ctx_len, dtype=np.int32)
     q_count = np.asarray(q_count, dtype=np.int32)
@@ -219,11 +239,13 @@ def make_workload(name: str, ctx_len, q_count, num_heads: int, topk: int = 2048,
     for r in range(B):
         block_table[r, :pages_per[r]] = phys[off:off + pages_per[r]]
         off += pages_per[r]
+    plain = latent_format == "e4m3"
+    assert plain or latent_format == "fp8_ds_mla"
     wl = Workload(name=name, num_heads=num_heads, topk=topk, cu_q=cu_q, ctx_len=ctx_len,
                   block_table=block_table, num_pages=num_pages,
-                  latent=_fill_latent(seed, name, num_pages),
+                  latent=_fill_plain(seed, name, num_pages) if plain else _fill_latent(seed, name, num_pages),
                   index_cache=_fill_index(seed, name, num_pages),
-                  ssmax=ssmax)
+                  ssmax=ssmax, latent_format=latent_format, latent_scale=PLAIN_SCALE if plain else 0.0)
     _scribble_tails(wl, stream(seed, name + "/tails"))
     T = int(cu_q[-1])
     for tag, rope_dim, with_idx, reuse in layers:

@@ -14,11 +14,18 @@ from __future__ import annotations
 
 import numpy as np
 
-from oracle import dsa, mla
+from oracle import dsa, formats, mla
 
 SCORE_REL = 1e-4
 OUT_RMS_REL = 2e-3
 LSE_ABS = 2e-3
+
+
+def oracle_latent(wl):
+    """The workload's latent pool as the oracle reads it."""
+    if wl.latent_format == "e4m3":
+        return formats.PlainE4M3Pool(wl.latent, wl.latent_scale)
+    return wl.latent
 
 
 def check_scores(wl, layer_i, scores_gpu, tokens=None, sample=None, seed=0):
@@ -66,7 +73,7 @@ def check_topk(wl, scores_gpu, idx_gpu, len_gpu, tokens=None):
 def check_attention(wl, layer_i, idx_gpu, len_gpu, out_gpu, lse_gpu, tokens=None):
     v = wl.view(layer_i)
     tokens = list(range(wl.T)) if tokens is None else list(tokens)
-    ref_o, ref_l = mla.sparse_mla(v, wl.latent, idx_gpu, len_gpu, tokens=tokens)
+    ref_o, ref_l = mla.sparse_mla(v, oracle_latent(wl), idx_gpu, len_gpu, tokens=tokens)
     got_o = out_gpu[tokens].astype(np.float64)
     got_l = lse_gpu[tokens].astype(np.float64)
     rms = float(np.sqrt(np.mean(ref_o ** 2)))

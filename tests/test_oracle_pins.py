@@ -506,3 +506,77 @@ def test_indexer_q_quantisation_is_one_block_per_token():
         assert (codes[t] & 0x7F).max() == 0x7E
         back = F.decode_e4m3(codes[t]) * float(scales[t])
         assert np.all(np.abs(back - x[t]) <= np.maximum(np.abs(x[t]) * 2.0 ** -4, 2.0 ** -10 * float(scales[t])) * (1 + 1e-6))
+
+
+# --- the plain per-tensor E4M3 latent format (576 B per token) --------------------
+
+def test_plain_e4m3_row_layout_from_independent_packing():
+    g = golden()
+    assert F.PLAIN_E4M3_ROW_BYTES == g["latent_row_plain_e4m3"] == 576
+    pool = bytearray(2 * 64 * 576)
+    page, row = 1, 21
+    codes = bytes((0x08 + 3 * i) % 0x7E for i in range(576))
+    off = page * 64 * 576 + row * 576
+    pool[off: off + 576] = codes
+    c, pe = F.plain_e4m3_rows(F.PlainE4M3Pool(np.frombuffer(bytes(pool), dtype=np.uint8), 0.375), [page], [row])
+    assert c.shape == (1, 512) and pe.shape == (1, 64)
+    assert all(c[0, d] == F.e4m3_value(codes[d]) * 0.375 for d in range(512))
+    assert all(pe[0, d] == F.e4m3_value(codes[512 + d]) * 0.375 for d in range(64))
+
+
+def test_plain_pool_gives_the_attention_of_an_equal_fp8_ds_mla_pool(small):
+    """Values that both formats hold exactly (every block scale equal to the
+    power-of-two pool scale, RoPE keys that are E4M3 values times it) give
+    identical rows and identical attention through the two readers."""
+    wl = small
+    s = 2.0 ** -5
+    rng = synth.stream(10, "plain_vs_ds")
+    n_rows = wl.num_pages * 64
+    codes = rng.integers(0, 0x7F, size=(n_rows, 576), dtype=np.uint8) | (rng.integers(0, 2, (n_rows, 576)) << 7).astype(np.uint8)
+    plain = F.PlainE4M3Pool(codes.reshape(-1), s)
+    ds = np.zeros((n_rows, F.LATENT_ROW_BYTES), dtype=np.uint8)
+    ds[:, :512] = codes[:, :512]
+    ds[:, 512:528] = np.full((n_rows, 4), s, dtype="<f4").view(np.uint8)
+    pe = (F.decode_e4m3(codes[:, 512:]) * s).astype(np.float32)
+    ds[:, 528:] = synth.to_bf16_bits(pe).astype("<u2").view(np.uint8).reshape(n_rows, 128)
+    assert np.array_equal(F.decode_bf16(synth.to_bf16_bits(pe)), pe.astype(np.float64))   # exact in bf16
+    ds = ds.reshape(-1)
+    pages = np.arange(wl.num_pages).repeat(64)
+    rows = np.tile(np.arange(64), wl.num_pages)
+    c1, p1 = F.latent_rows(plain, pages, rows)
+    c2, p2 = F.latent_rows(ds, pages, rows)
+    assert np.array_equal(c1, c2) and np.array_equal(p1, p2)
+    v = wl.view(0)
+    T = wl.T
+    idx = np.tile(np.arange(64), (T, 1))
+    ln = np.minimum(64, dsa.visible_lengths(wl.cu_q, wl.ctx_len))
+    o1, l1 = mla.sparse_mla(v, plain, idx, ln)
+    o2, l2 = mla.sparse_mla(v, ds, idx, ln)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_plain_e4m3_writer_round_trip_and_untouched_rows():
+    rng = synth.stream(11, "plain_writer")
+    pages, n = 2, 30
+    slot = synth.producer_slots(11, "plain_writer/slot", n, pages, 7)
+    c = synth.to_bf16_bits(rng.standard_normal((n, 512)).astype(np.float32))
+    kpe = synth.to_bf16_bits(rng.standard_normal((n, 64)).astype(np.float32))
+    s = 6.0 / 448.0
+    pool0 = F.PlainE4M3Pool(rng.integers(0, 256, pages * F.PLAIN_E4M3_PAGE_BYTES, dtype=np.uint8), s)
+    pool, bad = PR.write_latent_plain_e4m3(pool0, c, kpe, slot)
+    assert not bad and pool.scale == np.float32(s)
+    w = slot >= 0
+    ch, ph = F.plain_e4m3_rows(pool, slot[w] // 64, slot[w] % 64)
+    for got, want in ((ch, F.decode_bf16(c[w])), (ph, F.decode_bf16(kpe[w]))):
+        inside = np.abs(want) <= 448 * np.float32(s)
+        bound = np.maximum(np.abs(want) * 2.0 ** -4, 2.0 ** -10 * float(np.float32(s))) * (1 + 1e-6)
+        assert np.all(np.abs(got - want)[inside] <= bound[inside])
+        # outside the range the code saturates at +-448 s
+        assert np.all(np.abs(got[~inside]) == 448 * float(np.float32(s)))
+    touched = np.zeros(pages * 64, bool)
+    touched[slot[w]] = True
+    a = pool.data.reshape(pages * 64, 576)
+    b = pool0.data.reshape(pages * 64, 576)
+    assert np.array_equal(a[~touched], b[~touched])
+    nope, _ = PR.write_latent_plain_e4m3(pool0, c[:1], None, np.array([3], dtype=np.int32))
+    assert not nope.data[3 * 576 + 512: 4 * 576].any()
