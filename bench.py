@@ -47,7 +47,7 @@ FLUSH_BYTES = 256 << 20
 # dram__bytes_read.sum + dram__bytes_write.sum of one indexer launch on this
 # workload, from the ncu capture summarised in profiles/ (None = not captured
 # for the current kernel).
-INDEXER_NCU_TRAFFIC_BYTES = 163_692_032
+INDEXER_NCU_TRAFFIC_BYTES = 163_259_136
 
 
 def dist_env():
@@ -282,7 +282,29 @@ def time_ours(args, wl, rank):
         stream.synchronize()
         if i >= args.warmup:
             e2e_ms.append(e0.elapsed_time(e1))
-    return per, clocks.summary(), float(np.mean(e2e_ms)), h2d, d2h
+    # The same attention over a plain per-tensor E4M3 latent pool (576-B rows)
+    # with the same block table and selection: one graph of the MLA call.
+    plain = torch.from_numpy(synth.plain_pool(0, wl.name + "/plain_pool", wl.num_pages)).cuda()
+    lat_plain = sml.E4M3Latent(plain, synth.PLAIN_SCALE)
+    g_plain = torch.cuda.CUDAGraph()
+    sml.sml_sparse_mla_decode(p, lay.q, lat_plain, idx, ln, out, lse, ws, stream)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g_plain):
+        sml.sml_sparse_mla_decode(p, lay.q, lat_plain, idx, ln, out, lse, ws, torch.cuda.current_stream())
+    plain_ms = []
+    for i in range(args.warmup + args.steps):
+        flush()
+        t0.record(stream)
+        g_plain.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            plain_ms.append(t0.elapsed_time(t1))
+    del g_plain
+    code, bits = sml.sml_read_device_status(ws)
+    if code != sml.SML_OK:
+        raise RuntimeError(f"device status {code} bits {bits:#x}")
+    return per, clocks.summary(), float(np.mean(e2e_ms)), h2d, d2h, float(np.mean(plain_ms))
 
 
 # Algorithmic bytes per new token of the producers: bf16 inputs and the int32
@@ -444,7 +466,7 @@ def main():
         torch.cuda.set_device(0)
     wl = synth.SUITE[args.workload](seed=0)
     units = workload_units(wl)
-    per, clocks, e2e_ms, h2d, d2h = time_ours(args, wl, rank)
+    per, clocks, e2e_ms, h2d, d2h, plain_ms = time_ours(args, wl, rank)
     ms_step = max_over_ranks(float(per[:, 4].mean()))
     ms_staged = max_over_ranks(float(per[:, 3].mean()))
     ms_idx = max_over_ranks(float(per[:, 0].mean()))
@@ -481,6 +503,9 @@ def main():
         "gpu_launches": args.steps * 4,
         "cpu_baseline": cb,
         "producers": producers,
+        "latent_e4m3_576": {"sparse_mla_and_merge_ms": plain_ms,
+                            "hbm_gbs": units["gathered"] * 576 / (plain_ms / 1e3) / 1e9,
+                            "note": "the same selection over a plain per-tensor E4M3 latent pool (576-B rows)"},
     }
     print(json.dumps(line))
 

@@ -116,10 +116,24 @@ typedef struct sml_problem {
   const int32_t* block_table;  /* [B * max_pages], physical page ids */
 } sml_problem;
 
-/* A paged cache pool: num_pages pages starting at base (256-B aligned). */
+/* Latent cache formats (sml_cache.format of a latent pool; an indexer pool
+ * takes 0).  SML_LATENT_E4M3 is the plain per-tensor E4M3 cache of the blog's
+ * section "ROCm 实现细节", paragraph "FP8 潜在缓存": all 576 latent dims in FP8
+ * under one per-tensor scale, 576 B per token.  Reading: a row is
+ * [512 x e4m3 latent][64 x e4m3 RoPE key], value = code * scale. */
+#define SML_LATENT_FP8_DS_MLA 0
+#define SML_LATENT_E4M3 1
+#define SML_LATENT_E4M3_ROW_BYTES 576
+#define SML_LATENT_E4M3_PAGE_BYTES (SML_PAGE_TOKENS * SML_LATENT_E4M3_ROW_BYTES)
+
+/* A paged cache pool: num_pages pages starting at base (256-B aligned).  A
+ * zero-initialised descriptor (format 0) is the fp8_ds_mla latent layout or
+ * the indexer layout. */
 typedef struct sml_cache {
   const void* base;
   int64_t num_pages;
+  int32_t format;   /* latent pools: SML_LATENT_*; indexer pools: 0 */
+  float scale;      /* SML_LATENT_E4M3: the pool's scale, finite and > 0; else ignored */
 } sml_cache;
 
 /* Bytes of workspace the given stage needs for this problem (0 on invalid
@@ -236,10 +250,11 @@ int sml_sparse_mla_decode_noalloc(const sml_problem* p, const void* q, sml_cache
 int sml_indexer_k_cache_write(const void* k, const int32_t* slot, int32_t n, sml_cache index_cache,
                               void* workspace, void* stream);
 
-/* fp8_ds_mla latent write: c [n, 512] bf16 and k_pe [n, 64] bf16 (both 16-B
- * aligned; k_pe NULL for a NoPE layer, whose rows get a zero RoPE key) ->
- * the 656-B row at page*41984 + row*656: [512 e4m3][4 fp32 block scales]
- * [64 bf16 k_pe]. */
+/* Latent write: c [n, 512] bf16 and k_pe [n, 64] bf16 (both 16-B aligned;
+ * k_pe NULL for a NoPE layer, whose rows get a zero RoPE key).  By the pool's
+ * format: SML_LATENT_FP8_DS_MLA -> the 656-B row at page*41984 + row*656:
+ * [512 e4m3][4 fp32 block scales][64 bf16 k_pe]; SML_LATENT_E4M3 -> the 576-B
+ * row at page*36864 + row*576: the codes of every value / latent.scale. */
 int sml_latent_cache_write(const void* c, const void* k_pe, const int32_t* slot, int32_t n,
                            sml_cache latent, void* workspace, void* stream);
 

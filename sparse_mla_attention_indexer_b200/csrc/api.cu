@@ -74,11 +74,19 @@ void check_problem(Checker& c, const sml_problem* p) {
   c.check(p->block_table != nullptr, SML_ERR_INVALID_ARG, "block_table is NULL");
 }
 
-void check_cache(Checker& c, sml_cache cache, const char* what) {
+void check_cache(Checker& c, sml_cache cache, const char* what, bool latent) {
   std::string w(what);
   if (!cache.base) c.fail(SML_ERR_INVALID_ARG, (w + ".base is NULL").c_str());
   else if (!aligned(cache.base, 256)) c.fail(SML_ERR_INVALID_ARG, (w + ".base not 256-B aligned").c_str());
   if (cache.num_pages < 1) c.fail(SML_ERR_INVALID_ARG, (w + ".num_pages < 1").c_str());
+  if (!latent) {
+    if (cache.format != 0) c.fail(SML_ERR_UNSUPPORTED, (w + ".format not 0").c_str());
+  } else if (cache.format == SML_LATENT_E4M3) {
+    if (!(isfinite(cache.scale) && cache.scale > 0.f))
+      c.fail(SML_ERR_INVALID_ARG, (w + ".scale not finite and positive").c_str());
+  } else if (cache.format != SML_LATENT_FP8_DS_MLA) {
+    c.fail(SML_ERR_UNSUPPORTED, (w + ".format not an SML_LATENT_* format").c_str());
+  }
 }
 
 struct Layout {
@@ -238,7 +246,7 @@ int sml_indexer_scores(const sml_problem* p, const void* iq8, const float* iq_sc
   c.check(iq_scale != nullptr, SML_ERR_INVALID_ARG, "iq_scale is NULL");
   c.check(iw != nullptr, SML_ERR_INVALID_ARG, "iw is NULL");
   c.check(scores != nullptr, SML_ERR_INVALID_ARG, "scores is NULL");
-  check_cache(c, index_cache, "index_cache");
+  check_cache(c, index_cache, "index_cache", false);
   check_workspace(c, p, SML_STAGE_INDEXER, workspace, ws_bytes);
   if (c.done("sml_indexer_scores") != SML_OK) return c.code;
   cudaError_t e = launch_indexer(*p, static_cast<const uint8_t*>(iq8), iq_scale, iw,
@@ -272,12 +280,11 @@ int sml_sparse_mla_decode(const sml_problem* p, const void* q, sml_cache latent,
   c.check(idx_len != nullptr, SML_ERR_INVALID_ARG, "idx_len is NULL");
   c.check(out != nullptr && aligned(out, 16), SML_ERR_INVALID_ARG, "out NULL or not 16-B aligned");
   c.check(lse != nullptr, SML_ERR_INVALID_ARG, "lse is NULL");
-  check_cache(c, latent, "latent");
+  check_cache(c, latent, "latent", true);
   check_workspace(c, p, SML_STAGE_MLA, workspace, ws_bytes);
   if (c.done("sml_sparse_mla_decode") != SML_OK) return c.code;
   const Layout L = layout(*p, SML_STAGE_MLA);
-  cudaError_t e = launch_sparse_mla(*p, static_cast<const uint16_t*>(q),
-                                    static_cast<const uint8_t*>(latent.base), latent.num_pages, idx,
+  cudaError_t e = launch_sparse_mla(*p, static_cast<const uint16_t*>(q), latent, idx,
                                     idx_len, out, lse, mla_ws(*p, L, workspace), status_of(workspace),
                                     static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SML_OK : cuda_fail(e, "sml_sparse_mla_decode");
@@ -294,7 +301,7 @@ int sml_run_layer(const sml_problem* p, const void* q, const void* iq8, const fl
   c.check(q != nullptr && aligned(q, 16), SML_ERR_INVALID_ARG, "q NULL or not 16-B aligned");
   c.check(out != nullptr && aligned(out, 16), SML_ERR_INVALID_ARG, "out NULL or not 16-B aligned");
   c.check(lse != nullptr, SML_ERR_INVALID_ARG, "lse is NULL");
-  check_cache(c, latent, "latent");
+  check_cache(c, latent, "latent", true);
   if (reuse) {
     c.check(reuse_len != nullptr, SML_ERR_INVALID_ARG, "reuse_idx given without reuse_len");
   } else {
@@ -304,7 +311,7 @@ int sml_run_layer(const sml_problem* p, const void* q, const void* iq8, const fl
     c.check(iw != nullptr, SML_ERR_INVALID_ARG, "iw is NULL");
     c.check(idx_out != nullptr, SML_ERR_INVALID_ARG, "idx_out is NULL");
     c.check(len_out != nullptr, SML_ERR_INVALID_ARG, "len_out is NULL");
-    check_cache(c, index_cache, "index_cache");
+    check_cache(c, index_cache, "index_cache", false);
   }
   check_workspace(c, p, SML_STAGE_LAYER, workspace, ws_bytes);
   if (c.done("sml_run_layer") != SML_OK) return c.code;
@@ -324,8 +331,8 @@ int sml_run_layer(const sml_problem* p, const void* q, const void* iq8, const fl
     use_len = len_out;
   }
   if (e == cudaSuccess)
-    e = launch_sparse_mla(*p, static_cast<const uint16_t*>(q), static_cast<const uint8_t*>(latent.base),
-                          latent.num_pages, use_idx, use_len, out, lse, mla_ws(*p, L, workspace), status,
+    e = launch_sparse_mla(*p, static_cast<const uint16_t*>(q), latent, use_idx, use_len, out, lse,
+                          mla_ws(*p, L, workspace), status,
                           st);
   return e == cudaSuccess ? SML_OK : cuda_fail(e, "sml_run_layer");
 }
@@ -335,10 +342,10 @@ int sml_run_layer(const sml_problem* p, const void* q, const void* iq8, const fl
 namespace {
 
 void check_producer(Checker& c, int32_t n, const int32_t* slot, sml_cache cache, const char* what,
-                    int64_t max_pages, void* workspace) {
+                    int64_t max_pages, void* workspace, bool latent) {
   c.check(n >= 0, SML_ERR_INVALID_ARG, "n < 0");
   c.check(n == 0 || (slot != nullptr && aligned(slot, 4)), SML_ERR_INVALID_ARG, "slot NULL or not 4-B aligned");
-  check_cache(c, cache, what);
+  check_cache(c, cache, what, latent);
   c.check(cache.num_pages <= max_pages, SML_ERR_UNSUPPORTED, "num_pages * 64 slots exceed int32");
   c.check(workspace == nullptr || aligned(workspace, 256), SML_ERR_WORKSPACE, "workspace not 256-B aligned");
 }
@@ -350,7 +357,7 @@ constexpr int64_t kMaxSlotPages = ((int64_t)1 << 31) / SML_PAGE_TOKENS;
 int sml_indexer_k_cache_write(const void* k, const int32_t* slot, int32_t n, sml_cache index_cache,
                               void* workspace, void* stream) {
   Checker c;
-  check_producer(c, n, slot, index_cache, "index_cache", kMaxSlotPages, workspace);
+  check_producer(c, n, slot, index_cache, "index_cache", kMaxSlotPages, workspace, false);
   c.check(n == 0 || (k != nullptr && aligned(k, 16)), SML_ERR_INVALID_ARG, "k NULL or not 16-B aligned");
   if (c.done("sml_indexer_k_cache_write") != SML_OK) return c.code;
   cudaError_t e = launch_indexer_k_write(k, slot, n, const_cast<void*>(index_cache.base), index_cache.num_pages,
@@ -362,12 +369,11 @@ int sml_indexer_k_cache_write(const void* k, const int32_t* slot, int32_t n, sml
 int sml_latent_cache_write(const void* cl, const void* k_pe, const int32_t* slot, int32_t n, sml_cache latent,
                            void* workspace, void* stream) {
   Checker c;
-  check_producer(c, n, slot, latent, "latent", kMaxSlotPages, workspace);
+  check_producer(c, n, slot, latent, "latent", kMaxSlotPages, workspace, true);
   c.check(n == 0 || (cl != nullptr && aligned(cl, 16)), SML_ERR_INVALID_ARG, "c NULL or not 16-B aligned");
   c.check(aligned(k_pe, 16), SML_ERR_INVALID_ARG, "k_pe not 16-B aligned");
   if (c.done("sml_latent_cache_write") != SML_OK) return c.code;
-  cudaError_t e = launch_latent_write(cl, k_pe, slot, n, const_cast<void*>(latent.base), latent.num_pages,
-                                      workspace ? status_of(workspace) : nullptr,
+  cudaError_t e = launch_latent_write(cl, k_pe, slot, n, latent, workspace ? status_of(workspace) : nullptr,
                                       static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SML_OK : cuda_fail(e, "sml_latent_cache_write");
 }

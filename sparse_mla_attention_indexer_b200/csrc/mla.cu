@@ -97,6 +97,7 @@ struct Params {
   const uint16_t* q;
   const uint8_t* latent;
   int64_t latent_pages;
+  float latent_scale;   // plain E4M3 pool: its scale
   const int32_t* idx;
   const int32_t* idx_len;
   MlaWs ws;
@@ -129,6 +130,11 @@ __device__ __forceinline__ uint32_t f2_to_e4m3x2(float a, float b) {
 __device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t two) {
   const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
   return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// Two floats that are bf16 values -> their bf16 bits, low half = a.
+__device__ __forceinline__ uint32_t bf16x2_bits(float a, float b) {
+  return (__float_as_uint(a) >> 16) | (__float_as_uint(b) & 0xffff0000u);
 }
 
 // x (two values) -> E4M3 codes of the nearest value and the exact residual.
@@ -245,6 +251,10 @@ __device__ __forceinline__ bool tile_stats(Smem& S, int row, const float (&z)[kH
   return any != 0;
 }
 
+// kPlain: the latent pool is plain E4M3 (576-B rows under one scale); else
+// fp8_ds_mla.  A template parameter, so that each gather loop is compiled for
+// its own row layout.
+template <bool kPlain>
 __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params P) {
   extern __shared__ uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -341,15 +351,21 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
       const int tile = bi / kBatchesPerTile, buf = tile & 1;
       const int row0 = (bi % kBatchesPerTile) * kBatchRows;
       uint4 va[kBatchRows], vb[kBatchRows];
+      uint32_t live = 0;   // bit u: row u of the batch is a selected row (plain E4M3 only)
 #pragma unroll
       for (int u = 0; u < kBatchRows; ++u) {
         const int32_t id = S.rowid[tile * kKT + row0 + u];
-        const uint8_t* src = P.latent + (size_t)(id >= 0 ? id : 0) * SML_LATENT_ROW_BYTES;
+        const uint8_t* src =
+            P.latent + (size_t)(id >= 0 ? id : 0) * (kPlain ? SML_LATENT_E4M3_ROW_BYTES : SML_LATENT_ROW_BYTES);
         va[u] = make_uint4(0u, 0u, 0u, 0u);
         vb[u] = make_uint4(0u, 0u, 0u, 0u);
         if (id >= 0) {
+          if (kPlain) live |= 1u << u;
           va[u] = ldg_stream(src + 16 * lane);
-          if (lane == 0 || (lane <= 8 && P.rope_dim)) vb[u] = ldg_stream(src + SML_LATENT_DIM + 16 * lane);
+          // fp8_ds_mla: lane 0 the four block scales, lanes 1-8 the bf16 RoPE
+          // key; plain E4M3: lanes 0-3 the 64 RoPE codes
+          if (kPlain ? (lane < 4 && P.rope_dim) : (lane == 0 || (lane <= 8 && P.rope_dim)))
+            vb[u] = ldg_stream(src + SML_LATENT_DIM + 16 * lane);
         }
       }
       // first batch of this tile for this warp: the buffer must be free (PV of tile - 2 done)
@@ -365,10 +381,30 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
       for (int u = 0; u < kBatchRows; ++u) {
         const int row = row0 + u;
         st_shared_v4(sw128(lat_l, row, lane & 7), va[u].x, va[u].y, va[u].z, va[u].w);
-        if (lane == 0)
+        if (kPlain) {
+          // one scale for every block (zero for a masked row); RoPE codes
+          // widened to bf16 (exact: E4M3 values are bf16 values)
+          if (lane == 0) {
+            const uint32_t sb = (live >> u) & 1 ? __float_as_uint(P.latent_scale) : 0u;
+            st_shared_v4(sc_b + row * 16, sb, sb, sb, sb);
+          }
+          if (lane < 4 && P.rope_dim) {
+            const uint32_t w[4] = {vb[u].x, vb[u].y, vb[u].z, vb[u].w};
+            uint32_t o[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float2 lo = e4m3x2_to_f2(w[k]), hi = e4m3x2_to_f2(w[k] >> 16);
+              o[2 * k] = bf16x2_bits(lo.x, lo.y);
+              o[2 * k + 1] = bf16x2_bits(hi.x, hi.y);
+            }
+            st_shared_v4(sw128(pe_b, row, 2 * lane), o[0], o[1], o[2], o[3]);
+            st_shared_v4(sw128(pe_b, row, 2 * lane + 1), o[4], o[5], o[6], o[7]);
+          }
+        } else if (lane == 0) {
           st_shared_v4(sc_b + row * 16, vb[u].x, vb[u].y, vb[u].z, vb[u].w);
-        else if (lane <= 8 && P.rope_dim)
+        } else if (lane <= 8 && P.rope_dim) {
           st_shared_v4(sw128(pe_b, row, lane - 1), vb[u].x, vb[u].y, vb[u].z, vb[u].w);
+        }
       }
       if (bi + kGatherWarps >= (tile + 1) * kBatchesPerTile) {   // this warp's last batch of the tile
         ptx::fence_proxy_async();
@@ -530,11 +566,13 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
 #pragma unroll
         for (int h = 0; h < kHC; ++h) z[h] *= S.qs[h];
         if (P.rope_dim) {
+          // plain E4M3 keys hold codes: their scale multiplies the RoPE term
+          const float pe_scale = kPlain ? P.latent_scale : 1.f;
           uint32_t v[16];
           ptx::tmem_ld16(T0 + kColSpe + lane_off, v);
           ptx::tmem_wait_ld(v);
 #pragma unroll
-          for (int h = 0; h < kHC; ++h) z[h] += __uint_as_float(v[h]);
+          for (int h = 0; h < kHC; ++h) z[h] = fmaf(pe_scale, __uint_as_float(v[h]), z[h]);
         }
         ptx::tc_fence_before();
         __syncwarp();
@@ -696,11 +734,11 @@ int mla_splits(const sml_problem& p, int* keys_per_split) {
   return (p.topk + kps - 1) / kps;
 }
 
-cudaError_t launch_sparse_mla(const sml_problem& p, const uint16_t* q, const uint8_t* latent_base,
-                              int64_t latent_pages, const int32_t* idx, const int32_t* idx_len,
+cudaError_t launch_sparse_mla(const sml_problem& p, const uint16_t* q, const sml_cache& latent,
+                              const int32_t* idx, const int32_t* idx_len,
                               float* out, float* lse, const MlaWs& ws, int32_t* status,
                               cudaStream_t stream) {
-  if (latent_pages > (int64_t)(INT32_MAX / SML_PAGE_TOKENS)) return cudaErrorInvalidValue;
+  if (latent.num_pages > (int64_t)(INT32_MAX / SML_PAGE_TOKENS)) return cudaErrorInvalidValue;
   Params P;
   P.B = p.num_requests;
   P.T = p.num_tokens;
@@ -716,17 +754,19 @@ cudaError_t launch_sparse_mla(const sml_problem& p, const uint16_t* q, const uin
   P.ctx_len = p.ctx_len;
   P.block_table = p.block_table;
   P.q = q;
-  P.latent = latent_base;
-  P.latent_pages = latent_pages;
+  P.latent = static_cast<const uint8_t*>(latent.base);
+  P.latent_pages = latent.num_pages;
+  const bool plain = latent.format == SML_LATENT_E4M3;
+  P.latent_scale = plain ? latent.scale : 1.f;
   P.idx = idx;
   P.idx_len = idx_len;
   P.ws = ws;
   P.status = status;
   const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(sparse_mla_tc_kernel), smem);
+  auto kernel = plain ? sparse_mla_tc_kernel<true> : sparse_mla_tc_kernel<false>;
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(kernel), smem);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(sparse_mla_tc_kernel, dim3(ws.splits, p.num_heads / kHC, p.num_tokens), dim3(kThreads), smem,
-                 stream, 0, P);
+  e = launch_pdl(kernel, dim3(ws.splits, p.num_heads / kHC, p.num_tokens), dim3(kThreads), smem, stream, 0, P);
   if (e != cudaSuccess) return e;
   return launch_pdl(lse_merge_kernel, dim3(p.num_heads, p.num_tokens), dim3(128), 0, stream, 0, p.num_heads, ws, out,
                     lse);

@@ -1,6 +1,7 @@
 // sml_sparse_mla_decode_noalloc: sparse MLA decode whose split partials live in
 // a fixed scratch array compiled into the library, for callers that cannot
 // hand the library a workspace (see include/sml.h).
+#include <math.h>
 #include <stdio.h>
 
 #include <mutex>
@@ -65,6 +66,11 @@ extern "C" int sml_sparse_mla_decode_noalloc(const sml_problem* p, const void* q
   if (!lse) fail(SML_ERR_INVALID_ARG, "lse is NULL");
   if (!latent.base || ((uintptr_t)latent.base % 256)) fail(SML_ERR_INVALID_ARG, "latent.base NULL or not 256-B aligned");
   if (latent.num_pages < 1) fail(SML_ERR_INVALID_ARG, "latent.num_pages < 1");
+  if (latent.format == SML_LATENT_E4M3) {
+    if (!(isfinite(latent.scale) && latent.scale > 0.f)) fail(SML_ERR_INVALID_ARG, "latent.scale not finite and positive");
+  } else if (latent.format != SML_LATENT_FP8_DS_MLA) {
+    fail(SML_ERR_UNSUPPORTED, "latent.format not an SML_LATENT_* format");
+  }
   MlaWs ws{};
   size_t need = 0;
   if (code == SML_OK) {
@@ -93,9 +99,8 @@ extern "C" int sml_sparse_mla_decode_noalloc(const sml_problem* p, const void* q
     ws.part_out = reinterpret_cast<float*>(b);
     ws.part_lse = reinterpret_cast<float*>(b + align_up(slots * SML_LATENT_DIM * sizeof(float)));
     // No status word: the device checks still mask bad positions and pages.
-    e = launch_sparse_mla(*p, static_cast<const uint16_t*>(q),
-                          static_cast<const uint8_t*>(latent.base), latent.num_pages, idx, idx_len,
-                          out, lse, ws, nullptr, static_cast<cudaStream_t>(stream));
+    e = launch_sparse_mla(*p, static_cast<const uint16_t*>(q), latent, idx, idx_len, out, lse, ws, nullptr,
+                          static_cast<cudaStream_t>(stream));
   }
   if (e != cudaSuccess) {
     set_last_error(std::string("sml_sparse_mla_decode_noalloc: ") + cudaGetErrorString(e));

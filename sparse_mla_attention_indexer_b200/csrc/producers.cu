@@ -135,6 +135,46 @@ latent_write_kernel(const uint4* __restrict__ c, const uint4* __restrict__ kpe, 
   }
 }
 
+// The plain E4M3 pool (blog, section "ROCm 实现细节", paragraph "FP8 潜在缓存"):
+// every one of a row's 576 values becomes the code of x / scale with the
+// pool's given scale.  Two new tokens per warp: lane l codes latent values
+// [16 l, 16 l + 16) into bytes [16 l, 16 l + 16) of the 576-B row; lanes 0..7
+// code RoPE values [8 l, 8 l + 8) into bytes 512 + 8 l.
+__global__ void __launch_bounds__(32 * kWarpsPerCta)
+latent_write_plain_kernel(const uint4* __restrict__ c, const uint4* __restrict__ kpe,
+                          const int32_t* __restrict__ slot, int n, float scale, uint8_t* __restrict__ cache,
+                          long long slots, int32_t* status) {
+  ptx::griddep_wait();
+  if (threadIdx.x == 0) ptx::griddep_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int step = gridDim.x * kWarpsPerCta * kTokPerWarp;
+  for (int i0 = (blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5)) * kTokPerWarp; i0 < n; i0 += step) {
+    int s[kTokPerWarp];
+    uint4 v0[kTokPerWarp], v1[kTokPerWarp], pe[kTokPerWarp];
+#pragma unroll
+    for (int u = 0; u < kTokPerWarp; ++u) {
+      const int i = i0 + u;
+      s[u] = i < n ? __ldg(slot + i) : -1;
+      pe[u] = make_uint4(0, 0, 0, 0);
+      if (i < n) {
+        const uint4* src = c + (size_t)i * (SML_LATENT_DIM / 8) + 2 * lane;
+        v0[u] = __ldg(src);
+        v1[u] = __ldg(src + 1);
+        if (kpe && lane < 8) pe[u] = __ldg(kpe + (size_t)i * (SML_ROPE_DIM / 8) + lane);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kTokPerWarp; ++u) {
+      if (!slot_ok(s[u], slots, lane, status)) continue;
+      uint8_t* row = cache + (size_t)(s[u] / SML_PAGE_TOKENS) * SML_LATENT_E4M3_PAGE_BYTES +
+                     (size_t)(s[u] % SML_PAGE_TOKENS) * SML_LATENT_E4M3_ROW_BYTES;
+      const uint2 q0 = quant8(v0[u], scale), q1 = quant8(v1[u], scale);
+      reinterpret_cast<uint4*>(row)[lane] = make_uint4(q0.x, q0.y, q1.x, q1.y);
+      if (lane < 8) reinterpret_cast<uint2*>(row + SML_LATENT_DIM)[lane] = kpe ? quant8(pe[u], scale) : make_uint2(0, 0);
+    }
+  }
+}
+
 // One CTA per query token: 64 x 128 bf16 in (16 KB), one block.
 constexpr int kQThreads = 256;
 constexpr int kQVec = SML_INDEX_HEADS * SML_INDEX_DIM / 8 / kQThreads;   // uint4 loads per thread: 4
@@ -184,12 +224,17 @@ cudaError_t launch_indexer_k_write(const void* k, const int32_t* slot, int n, vo
                     (long long)num_pages * SML_PAGE_TOKENS, status);
 }
 
-cudaError_t launch_latent_write(const void* c, const void* kpe, const int32_t* slot, int n, void* cache,
-                                int64_t num_pages, int32_t* status, cudaStream_t stream) {
+cudaError_t launch_latent_write(const void* c, const void* kpe, const int32_t* slot, int n, const sml_cache& cache,
+                                int32_t* status, cudaStream_t stream) {
   if (n == 0) return cudaSuccess;
-  return launch_pdl(latent_write_kernel, dim3(token_grid(n, kWarpsPerCta * kTokPerWarp, 8)), dim3(32 * kWarpsPerCta), 0,
-                    stream, 0, static_cast<const uint4*>(c), static_cast<const uint4*>(kpe), slot, n,
-                    static_cast<uint8_t*>(cache), (long long)num_pages * SML_PAGE_TOKENS, status);
+  const dim3 grid(token_grid(n, kWarpsPerCta * kTokPerWarp, 8)), block(32 * kWarpsPerCta);
+  uint8_t* base = static_cast<uint8_t*>(const_cast<void*>(cache.base));
+  const long long slots = (long long)cache.num_pages * SML_PAGE_TOKENS;
+  if (cache.format == SML_LATENT_E4M3)
+    return launch_pdl(latent_write_plain_kernel, grid, block, 0, stream, 0, static_cast<const uint4*>(c),
+                      static_cast<const uint4*>(kpe), slot, n, cache.scale, base, slots, status);
+  return launch_pdl(latent_write_kernel, grid, block, 0, stream, 0, static_cast<const uint4*>(c),
+                    static_cast<const uint4*>(kpe), slot, n, base, slots, status);
 }
 
 cudaError_t launch_indexer_q_quant(const void* iq, int T, void* iq8, float* iq_scale, cudaStream_t stream) {

@@ -146,14 +146,14 @@ cudaError_t launch_indexer(const sml_problem& p, const uint8_t* iq8, const float
                            float* scores, int32_t* status, cudaStream_t stream);
 cudaError_t launch_topk(const sml_problem& p, const float* scores, int32_t* idx, int32_t* idx_len,
                         const TopkWs& ws, int32_t* status, cudaStream_t stream);
-cudaError_t launch_sparse_mla(const sml_problem& p, const uint16_t* q, const uint8_t* latent_base,
-                              int64_t latent_pages, const int32_t* idx, const int32_t* idx_len,
+cudaError_t launch_sparse_mla(const sml_problem& p, const uint16_t* q, const sml_cache& latent,
+                              const int32_t* idx, const int32_t* idx_len,
                               float* out, float* lse, const MlaWs& ws, int32_t* status,
                               cudaStream_t stream);
 cudaError_t launch_indexer_k_write(const void* k, const int32_t* slot, int n, void* cache, int64_t num_pages,
                                    int32_t* status, cudaStream_t stream);
-cudaError_t launch_latent_write(const void* c, const void* kpe, const int32_t* slot, int n, void* cache,
-                                int64_t num_pages, int32_t* status, cudaStream_t stream);
+cudaError_t launch_latent_write(const void* c, const void* kpe, const int32_t* slot, int n, const sml_cache& cache,
+                                int32_t* status, cudaStream_t stream);
 cudaError_t launch_indexer_q_quant(const void* iq, int T, void* iq8, float* iq_scale, cudaStream_t stream);
 
 }  // namespace sml

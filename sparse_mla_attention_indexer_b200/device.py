@@ -34,6 +34,8 @@ class DeviceWorkload:
         self.ctx_len = torch.from_numpy(wl.ctx_len).to(device)
         self.block_table = torch.from_numpy(np.ascontiguousarray(wl.block_table)).to(device)
         self.latent = torch.from_numpy(wl.latent).to(device)
+        if wl.latent_format == "e4m3":
+            self.latent = sml.E4M3Latent(self.latent, wl.latent_scale)
         self.index_cache = torch.from_numpy(wl.index_cache).to(device)
         self.layers = [DeviceLayer(lay, device) for lay in wl.layers]
         self.T, self.H, self.K = wl.T, wl.num_heads, wl.topk

@@ -10,6 +10,7 @@ from __future__ import annotations
 import ctypes
 import os
 import re
+from typing import NamedTuple
 
 import torch
 
@@ -38,7 +39,10 @@ SML_STAGE_LAYER = 4
 
 PAGE_TOKENS = 64
 LATENT_PAGE_BYTES = 64 * 656
+LATENT_E4M3_PAGE_BYTES = 64 * 576
 INDEX_PAGE_BYTES = 64 * 132
+SML_LATENT_FP8_DS_MLA = 0
+SML_LATENT_E4M3 = 1
 
 
 class SmlError(RuntimeError):
@@ -67,7 +71,15 @@ class Problem(ctypes.Structure):
 
 
 class Cache(ctypes.Structure):
-    _fields_ = [("base", ctypes.c_void_p), ("num_pages", ctypes.c_int64)]
+    _fields_ = [("base", ctypes.c_void_p), ("num_pages", ctypes.c_int64), ("format", ctypes.c_int32),
+                ("scale", ctypes.c_float)]
+
+
+class E4M3Latent(NamedTuple):
+    """A latent pool in the plain per-tensor E4M3 format (576-B rows) and its scale;
+    a bare uint8 tensor is an fp8_ds_mla pool."""
+    pool: torch.Tensor
+    scale: float
 
 
 _lib = None
@@ -158,8 +170,16 @@ def make_problem(*, num_heads, topk, rope_dim, cu_q, ctx_len, block_table, max_c
 def cache(pool, page_bytes: int) -> Cache:
     """Cache descriptor of a uint8 pool tensor (or None for an absent cache)."""
     if pool is None:
-        return Cache(None, 0)
-    return Cache(_p(pool), _nbytes(pool) // page_bytes)
+        return Cache(None, 0, 0, 0.0)
+    return Cache(_p(pool), _nbytes(pool) // page_bytes, 0, 0.0)
+
+
+def latent_cache(latent) -> Cache:
+    """Descriptor of a latent pool: a uint8 tensor (fp8_ds_mla) or an E4M3Latent."""
+    if isinstance(latent, E4M3Latent):
+        return Cache(_p(latent.pool), _nbytes(latent.pool) // LATENT_E4M3_PAGE_BYTES, SML_LATENT_E4M3,
+                     float(latent.scale))
+    return cache(latent, LATENT_PAGE_BYTES)
 
 
 def sml_workspace_size(problem: Problem, stage: int) -> int:
@@ -185,7 +205,7 @@ def sml_topk(problem, scores, idx, idx_len, workspace, stream=None):
 
 
 def sml_sparse_mla_decode(problem, q, latent, idx, idx_len, out, lse, workspace, stream=None):
-    _check(lib().sml_sparse_mla_decode(ctypes.byref(problem), _p(q), cache(latent, LATENT_PAGE_BYTES),
+    _check(lib().sml_sparse_mla_decode(ctypes.byref(problem), _p(q), latent_cache(latent),
                                        _p(idx), _p(idx_len), _p(out), _p(lse), _p(workspace),
                                        _nbytes(workspace), _s(stream)))
 
@@ -193,14 +213,14 @@ def sml_sparse_mla_decode(problem, q, latent, idx, idx_len, out, lse, workspace,
 def sml_sparse_mla_decode_noalloc(problem, q, latent, idx, idx_len, out, lse, stream=None):
     """Sparse MLA decode without a workspace (scratch built into the library)."""
     _check(lib().sml_sparse_mla_decode_noalloc(ctypes.byref(problem), _p(q),
-                                               cache(latent, LATENT_PAGE_BYTES), _p(idx),
+                                               latent_cache(latent), _p(idx),
                                                _p(idx_len), _p(out), _p(lse), _s(stream)))
 
 
 def sml_run_layer(problem, q, iq8, iq_scale, iw, latent, index_cache, reuse_idx, reuse_len,
                   idx_out, len_out, out, lse, workspace, stream=None):
     _check(lib().sml_run_layer(ctypes.byref(problem), _p(q), _p(iq8), _p(iq_scale), _p(iw),
-                               cache(latent, LATENT_PAGE_BYTES), cache(index_cache, INDEX_PAGE_BYTES),
+                               latent_cache(latent), cache(index_cache, INDEX_PAGE_BYTES),
                                _p(reuse_idx), _p(reuse_len), _p(idx_out), _p(len_out), _p(out),
                                _p(lse), _p(workspace), _nbytes(workspace), _s(stream)))
 
@@ -214,7 +234,7 @@ def sml_indexer_k_cache_write(k, slot, index_cache, workspace=None, stream=None)
 def sml_latent_cache_write(c, k_pe, slot, latent, workspace=None, stream=None):
     """Quantise new latent rows c [n, 512] bf16 (+ k_pe [n, 64] bf16, or None) into the
     fp8_ds_mla cache at slot [n] int32."""
-    _check(lib().sml_latent_cache_write(_p(c), _p(k_pe), _p(slot), _numel(slot), cache(latent, LATENT_PAGE_BYTES),
+    _check(lib().sml_latent_cache_write(_p(c), _p(k_pe), _p(slot), _numel(slot), latent_cache(latent),
                                         _p(workspace), _s(stream)))
 
 

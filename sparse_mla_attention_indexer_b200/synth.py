@@ -199,7 +199,7 @@ def make_layer(seed: int, tag: str, T: int, H: int, rope_dim: int, with_indexer:
     return lay
 
 
-def _fill_plain(seed: int, name: str, num_pages: int, chunk_pages: int = 512) -> np.ndarray:
+def plain_pool(seed: int, name: str, num_pages: int, chunk_pages: int = 512) -> np.ndarray:
     """Plain E4M3 latent pool: 576 values N(0, 1) per row (512 latent, 64 RoPE),
     codes of x / PLAIN_SCALE."""
     out = np.empty((num_pages, PLAIN_PAGE), dtype=np.uint8)
@@ -243,7 +243,7 @@ def make_workload(name: str, ctx_len, q_count, num_heads: int, topk: int = 2048,
     assert plain or latent_format == "fp8_ds_mla"
     wl = Workload(name=name, num_heads=num_heads, topk=topk, cu_q=cu_q, ctx_len=ctx_len,
                   block_table=block_table, num_pages=num_pages,
-                  latent=_fill_plain(seed, name, num_pages) if plain else _fill_latent(seed, name, num_pages),
+                  latent=plain_pool(seed, name, num_pages) if plain else _fill_latent(seed, name, num_pages),
                   index_cache=_fill_index(seed, name, num_pages),
                   ssmax=ssmax, latent_format=latent_format, latent_scale=PLAIN_SCALE if plain else 0.0)
     _scribble_tails(wl, stream(seed, name + "/tails"))

@@ -4,6 +4,7 @@ CUDA call (so these run without a GPU)."""
 import ctypes
 
 import pytest
+import torch
 
 from sparse_mla_attention_indexer_b200 import build as sml_build
 from sparse_mla_attention_indexer_b200 import sml
@@ -91,3 +92,27 @@ def test_producers_reject_bad_arguments_without_cuda(L):
     assert "iq8" in sml.sml_last_error() and "iq_scale" in sml.sml_last_error()
     # empty batches need no buffers
     assert L.sml_indexer_q_quant(None, 0, None, None, None) == sml.SML_OK
+
+
+def test_cache_format_checks_without_cuda(L):
+    p = _problem()
+    lat = sml.Cache(0x10000, 4, 1, 0.0)          # plain E4M3 without a scale
+    code = L.sml_sparse_mla_decode(ctypes.byref(p), 0x1000, lat, 0x2000, 0x3000, 0x4000, 0x5000, None, 0, None)
+    assert code == sml.SML_ERR_INVALID_ARG and "latent.scale" in sml.sml_last_error()
+    lat = sml.Cache(0x10000, 4, 7, 1.0)          # unknown format
+    code = L.sml_sparse_mla_decode(ctypes.byref(p), 0x1000, lat, 0x2000, 0x3000, 0x4000, 0x5000, None, 0, None)
+    assert "latent.format" in sml.sml_last_error()
+    idx = sml.Cache(0x10000, 4, 1, 1.0)          # the indexer pool has one layout
+    code = L.sml_indexer_scores(ctypes.byref(p), 0x1000, 0x2000, 0x3000, idx, 0x4000, None, 0, None)
+    assert "index_cache.format" in sml.sml_last_error()
+
+
+def test_cache_descriptors_of_both_latent_forms():
+    ds = torch.zeros(3 * sml.LATENT_PAGE_BYTES, dtype=torch.uint8)
+    c = sml.latent_cache(ds)
+    assert (c.num_pages, c.format) == (3, sml.SML_LATENT_FP8_DS_MLA)
+    plain = torch.zeros(5 * sml.LATENT_E4M3_PAGE_BYTES, dtype=torch.uint8)
+    c = sml.latent_cache(sml.E4M3Latent(plain, 0.25))
+    assert (c.num_pages, c.format, c.scale) == (5, sml.SML_LATENT_E4M3, 0.25)
+    c = sml.cache(None, sml.INDEX_PAGE_BYTES)
+    assert (c.base, c.num_pages, c.format) == (None, 0, 0)

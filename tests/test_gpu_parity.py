@@ -254,3 +254,39 @@ def test_device_checks_set_status_bits():
                       idx, ln, out, lse, ws)
     assert sml.sml_read_device_status(ws)[0] == sml.SML_OK
     torch.cuda.synchronize()
+
+
+# --- the plain per-tensor E4M3 latent pool (576-B rows) ------------------------------
+
+@pytest.mark.parametrize("case", [0, 1, 2, 4])
+def test_plain_e4m3_latent_small_every_element(case):
+    L, Q, H, K, rope, ssmax, perm = SMALL[case]
+    wl = synth.make_workload(f"plain{case}", L, Q, H, topk=K, permuted=perm, ssmax=ssmax,
+                             layers=(("l0", rope, True, None),), extra_pages=3, latent_format="e4m3")
+    dw = DeviceWorkload(wl)
+    r = run_stages(dw)
+    parity.check_topk(wl, r["scores"], r["idx"], r["len"])
+    parity.check_attention(wl, 0, r["idx"], r["len"], r["out"], r["lse"])
+    r2 = run_layer(dw)
+    assert np.array_equal(r2["out"], r["out"]) and np.array_equal(r2["lse"], r["lse"], equal_nan=True)
+
+
+def test_plain_e4m3_latent_batched_decode_full():
+    base = synth.batched_decode()
+    wl = synth.make_workload("batched_decode_e4m3", base.ctx_len, np.ones(base.B, np.int32), 16,
+                             latent_format="e4m3")
+    dw = DeviceWorkload(wl)
+    r = run_stages(dw)
+    parity.check_topk(wl, r["scores"], r["idx"], r["len"])
+    parity.check_attention(wl, 0, r["idx"], r["len"], r["out"], r["lse"])
+
+
+def test_plain_e4m3_rejects_a_bad_scale():
+    wl = synth.make_workload("plain_bad", [300], [1], 16, topk=64, latent_format="e4m3")
+    dw = DeviceWorkload(wl)
+    p = dw.problem(0)
+    idx, ln, out, lse = dw.outputs()
+    bad = sml.E4M3Latent(dw.latent.pool, 0.0)
+    with pytest.raises(sml.SmlError) as e:
+        sml.sml_sparse_mla_decode(p, dw.layers[0].q, bad, idx, ln, out, lse, dw.workspace())
+    assert "latent.scale" in str(e.value)

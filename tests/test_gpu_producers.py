@@ -138,3 +138,21 @@ def test_whole_pools_of_a_workload_match_the_oracle():
     sml.sml_indexer_k_cache_write(bf16_dev(k), dev(slot), idx)
     assert np.array_equal(lat.cpu().numpy(), lat_want)
     assert np.array_equal(idx.cpu().numpy(), idx_want)
+
+
+@pytest.mark.parametrize("n,pages,skip,rope", [(10003, 160, 101, True), (300, 6, 7, False)])
+def test_plain_e4m3_latent_write_bit_exact(n, pages, skip, rope):
+    from oracle import formats as F
+    c = synth.producer_rows(6, f"pc/{n}", n, 512, spread=False)
+    kpe = synth.producer_rows(6, f"pkpe/{n}", n, 64, spread=False) if rope else None
+    slot = synth.producer_slots(6, f"pslot/{n}", n, pages, skip)
+    scale = 5.0 / 448.0      # some values saturate at +-448 codes
+    pool0 = synth.stream(6, f"ppool/{n}").integers(0, 256, pages * synth.PLAIN_PAGE, dtype=np.uint8)
+    want, bad = PR.write_latent_plain_e4m3(F.PlainE4M3Pool(pool0, scale), c, kpe, slot)
+    assert not bad
+    pool = dev(pool0)
+    sml.sml_latent_cache_write(bf16_dev(c), None if kpe is None else bf16_dev(kpe), dev(slot),
+                               sml.E4M3Latent(pool, want.scale), status_ws())
+    got = pool.cpu().numpy()
+    diff = np.nonzero(got != want.data)[0]
+    assert diff.size == 0, f"{diff.size} bytes differ, first at {diff[:8]}"
