@@ -90,7 +90,7 @@ void check_cache(Checker& c, sml_cache cache, const char* what, bool latent) {
 }
 
 struct Layout {
-  size_t header = 0, counters = 0, cand_key = 0, cand_idx = 0, part_out = 0, part_lse = 0,
+  size_t header = 0, counters = 0, cand_key = 0, cand_idx = 0, cand_cnt = 0, part_out = 0, part_lse = 0,
          scores = 0, total = 0;
 };
 
@@ -113,6 +113,8 @@ Layout layout(const sml_problem& p, int stage) {
     off += align_up(n * sizeof(uint32_t));
     L.cand_idx = off;
     off += align_up(n * sizeof(int32_t));
+    L.cand_cnt = off;
+    off += align_up((size_t)p.num_tokens * ch * sizeof(int32_t));
   }
   const size_t end_topk = off;
   int kps;
@@ -158,6 +160,7 @@ TopkWs topk_ws(const sml_problem& p, const Layout& L, void* ws) {
   t.counters = reinterpret_cast<int32_t*>(b + L.counters);
   t.cand_key = L.cand_key ? reinterpret_cast<uint32_t*>(b + L.cand_key) : nullptr;
   t.cand_idx = L.cand_idx ? reinterpret_cast<int32_t*>(b + L.cand_idx) : nullptr;
+  t.cand_cnt = L.cand_cnt ? reinterpret_cast<int32_t*>(b + L.cand_cnt) : nullptr;
   t.chunks = topk_chunks(p);
   return t;
 }

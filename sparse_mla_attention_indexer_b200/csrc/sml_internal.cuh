@@ -33,6 +33,7 @@ struct TopkWs {
   int32_t* counters;   // [T] arrival counters, zero between calls
   uint32_t* cand_key;  // [T, chunks, K]
   int32_t* cand_idx;   // [T, chunks, K]
+  int32_t* cand_cnt;   // [T, chunks] candidates per chunk
   int chunks;          // ceil(max_ctx / kTopkChunk)
 };
 

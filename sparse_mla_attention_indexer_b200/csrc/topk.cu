@@ -19,10 +19,14 @@
 //    key > tau and the lowest positions among keys == tau: the output is in
 //    ascending position order and ties go to the lower position;
 //  * rows longer than one chunk (16,384 positions) are cut into chunks, each
-//    selected by its own CTA into a candidate list; the last CTA of the row to
+//    turned by its own CTA into a candidate list; the last CTA of the row to
 //    finish (an arrival counter, no waiting) selects again over the
-//    concatenated candidates.  The global top-k is a subset of the union of
-//    the chunk top-ks, so the result is exact.
+//    concatenated candidates.  A chunk's candidates are its keys at or above a
+//    floor placed by a strided sample of the whole row (the same in every CTA
+//    of the row), or its own top k when more than k keys pass the floor or the
+//    sample gives none; a row whose candidates fall short of k (the sample
+//    misjudged) is selected again over all its positions.  Either way every
+//    key of the global top k is a candidate, so the result is exact.
 #include "ptx.cuh"
 #include "sml_internal.cuh"
 
@@ -33,6 +37,8 @@ constexpr int kBuckets = 2048;
 constexpr int kCandCap = 4096;
 constexpr int kSmallCand = 256;   // threshold by direct rank counting up to this many candidates
 constexpr int kSample = 1024;     // keys sampled to place the histogram floor
+constexpr int kMaxSegChunks = 4096;   // longest row (in chunks) whose candidates are floor-cut segments
+constexpr int kLevel2Keys = 2 * kTopkChunk;   // candidate keys the last CTA of a row holds in shared memory
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t b = __float_as_uint(f);
@@ -383,6 +389,118 @@ __device__ void select_topk(int n, int k, KeyAt key_at, Emit emit, SelectShared&
   __syncthreads();
 }
 
+// The row's floor from a strided sample of up to kSample keys, the same in
+// every CTA of the row so that all agree: the sample's ceil(mu + 4 sqrt(mu) +
+// 4)-th largest value (mu = k ns / n), found through a 256-bin coarse
+// histogram and then exactly among the samples of its bin, so that about
+// k (1 + a margin) keys of the row lie at or above it; -inf when the sample's
+// finite range is empty or the row is short.  All threads of the block call
+// it; the result is uniform.
+__device__ float row_floor(const float* row, int n, int k, SelectShared& sh) {
+  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int ns = min(kSample, n);
+  constexpr int kPer = kSample / kTopkThreads;
+  float sv[kPer];
+  float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int j = tid + u * nt;
+    sv[u] = NAN;
+    if (j < ns) {
+      sv[u] = key_value(order_key(__ldcg(row + (int)((long long)j * n / ns))));
+      if (isfinite(sv[u])) {
+        lo = fminf(lo, sv[u]);
+        hi = fmaxf(hi, sv[u]);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    sh.red_lo[warp] = lo;
+    sh.red_hi[warp] = hi;
+  }
+  for (int b = tid; b < 256; b += nt) sh.hist[b] = 0;
+  if (tid == 0) {
+    sh.bcast_f = -INFINITY;
+    sh.bcast[0] = 0;   // no bin found: no floor
+  }
+  __syncthreads();
+  lo = INFINITY;
+  hi = -INFINITY;
+  for (int w = 0; w < nt / 32; ++w) {
+    lo = fminf(lo, sh.red_lo[w]);
+    hi = fmaxf(hi, sh.red_hi[w]);
+  }
+  const float width = hi - lo;
+  if (!(hi > lo && width < INFINITY) || n <= 2 * k) return -INFINITY;
+  const float cscale = 254.f / width;
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const float v = sv[u];
+    if (tid + u * nt < ns) {
+      const int cb = !(v > -INFINITY) ? 0 : (v == INFINITY ? 255 : 1 + (int)fminf(fmaxf((v - lo) * cscale, 0.f), 253.f));
+      atomicAdd(&sh.hist[cb], 1);
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const float mu = (float)k * ns / (float)n;
+    const int need_s = min(ns, (int)ceilf(mu + 4.f * sqrtf(mu) + 4.f));
+    const int top = 255 - 8 * lane;   // 8 coarse bins per lane, descending
+    int local = 0;
+    for (int j = 0; j < 8; ++j) local += sh.hist[top - j];
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int above = incl - local;
+    if (above < need_s && need_s <= incl) {
+      for (int j = 0; j < 8; ++j) {
+        const int h = sh.hist[top - j];
+        if (need_s <= above + h) {
+          sh.bcast[0] = top - j;            // the bin
+          sh.bcast[1] = need_s - above;     // rank of the floor within it (1 = its largest)
+          break;
+        }
+        above += h;
+      }
+    }
+  }
+  if (tid == 0) sh.ncand = 0;
+  __syncthreads();
+  const int fb = sh.bcast[0], rank = sh.bcast[1];
+  if (fb <= 1) return -INFINITY;            // the floor would sit in the -inf / lowest bin
+  // the bin's samples into shared memory, then the one with `rank - 1` larger
+  // ones (ties: the value itself is the floor whichever copy is taken)
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const float v = sv[u];
+    if (tid + u * nt < ns && v > -INFINITY && v < INFINITY &&
+        1 + (int)fminf(fmaxf((v - lo) * cscale, 0.f), 253.f) == fb)
+      sh.cand[atomicAdd(&sh.ncand, 1)] = __float_as_uint(v);
+  }
+  __syncthreads();
+  const int m = sh.ncand;
+  for (int i = tid; i < m; i += nt) {
+    const float v = __uint_as_float(sh.cand[i]);
+    int gt = 0, ge = 0;
+    for (int j = 0; j < m; ++j) {
+      const float w = __uint_as_float(sh.cand[j]);
+      gt += w > v;
+      ge += w >= v;
+    }
+    if (gt < rank && rank <= ge) sh.bcast_f = v;   // every writer writes the same value
+  }
+  __syncthreads();
+  return sh.bcast_f;
+}
+
 __global__ void __launch_bounds__(kTopkThreads, 1)
 topk_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32_t* __restrict__ cu_q,
             const int32_t* __restrict__ ctx_len, const float* __restrict__ scores,
@@ -428,11 +546,60 @@ topk_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32_t* __re
     return;
   }
 
-  // Level 1: this chunk's top-k, as candidates in position order.
+  // Level 1: this chunk's candidates, in position order.  With a sampled
+  // floor, the chunk's keys at or above it when there are at most K of them;
+  // otherwise (and in rows too long for segment offsets in shared memory) the
+  // chunk's own top K.
+  constexpr int kW = kTopkThreads / 32;
   const size_t row_base = (size_t)t * ws.chunks * K;
   uint32_t* ck = ws.cand_key + row_base + (size_t)c * K;
   int32_t* ci = ws.cand_idx + row_base + (size_t)c * K;
-  select_topk(cn, K, smem_key, [&](int pos, int i) { ck[pos] = skeys[i]; ci[pos] = c0 + i; }, sh);
+  const float* full_row = scores + (size_t)t * max_ctx;
+  const bool segmented = nch <= kMaxSegChunks;
+  int count = -1;
+  if (segmented) {
+    const float fl = row_floor(full_row, n, K, sh);
+    if (fl > -INFINITY) {
+      const uint32_t fkey = order_key(fl);
+      const int lane = tid & 31, warp = tid >> 5;
+      const int seg = ((cn + kW - 1) / kW + 31) & ~31;
+      const int wb = min(cn, warp * seg), we = min(cn, wb + seg);
+      int cnt = 0;
+      for (int i0 = wb; i0 < we; i0 += 32) {
+        const int i = i0 + lane;
+        cnt += __popc(__ballot_sync(0xffffffffu, i < we && skeys[i] >= fkey));
+      }
+      if (lane == 0) sh.warp_a[warp] = cnt;
+      __syncthreads();
+      int total = 0, before = 0;
+      for (int w = 0; w < kW; ++w) {
+        total += sh.warp_a[w];
+        before += w < warp ? sh.warp_a[w] : 0;
+      }
+      if (total <= K) {
+        const unsigned below = (1u << lane) - 1u;
+        int off = before;
+        for (int i0 = wb; i0 < we; i0 += 32) {
+          const int i = i0 + lane;
+          const bool cand = i < we && skeys[i] >= fkey;
+          const unsigned m = __ballot_sync(0xffffffffu, cand);
+          if (cand) {
+            const int p = off + __popc(m & below);
+            ck[p] = skeys[i];
+            ci[p] = c0 + i;
+          }
+          off += __popc(m);
+        }
+        count = total;
+      }
+      __syncthreads();   // every warp has read warp_a before sh is reused
+    }
+  }
+  if (count < 0) {
+    select_topk(cn, K, smem_key, [&](int pos, int i) { ck[pos] = skeys[i]; ci[pos] = c0 + i; }, sh);
+    count = min(K, cn);
+  }
+  if (segmented && tid == 0) ws.cand_cnt[(size_t)t * ws.chunks + c] = count;
   __threadfence();  // this thread's candidates are visible device-wide ...
   __syncthreads();  // ... before the row's arrival counter moves
   if (tid == 0) {
@@ -443,20 +610,75 @@ topk_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32_t* __re
   if (!is_last) return;
   __threadfence();
 
-  // Level 2 (last CTA of the row): every chunk but the last holds exactly K
-  // candidates (a chunk has kTopkChunk >= K positions), so the candidates are
-  // contiguous and still in position order.
-  const int total = (nch - 1) * K + min(K, n - (nch - 1) * kTopkChunk);
+  // Level 2 (last CTA of the row).
   const uint32_t* tk = ws.cand_key + row_base;
   const int32_t* ti = ws.cand_idx + row_base;
-  if (total <= kTopkChunk) {
-#pragma unroll 16
-    for (int i = tid; i < total; i += nt) skeys[i] = __ldcg(tk + i);
-    __syncthreads();
-    select_topk(total, K, smem_key, [&](int pos, int i) { out[pos] = __ldcg(ti + i); }, sh);
-  } else {
+  if (!segmented) {
+    // every chunk but the last holds exactly K candidates (a chunk has
+    // kTopkChunk >= K positions), so they are contiguous and in position order
+    const int total = (nch - 1) * K + min(K, n - (nch - 1) * kTopkChunk);
     select_topk(total, K, [&](int i) { return __ldcg(tk + i); },
                 [&](int pos, int i) { out[pos] = __ldcg(ti + i); }, sh);
+  } else {
+    // segment starts (candidates before chunk c) into shared memory, after
+    // room for kLevel2Keys candidate keys
+    int* soff = reinterpret_cast<int*>(skeys + kLevel2Keys);
+    const int32_t* cnt = ws.cand_cnt + (size_t)t * ws.chunks;
+    int total = 0;
+    for (int base = 0; base < nch; base += nt) {
+      const int c2 = base + tid;
+      const int v = c2 < nch ? __ldcg(cnt + c2) : 0;
+      int tot;
+      const int incl = block_scan_incl(v, sh.warp_b, &tot);
+      if (c2 < nch) soff[c2] = total + incl - v;
+      total += tot;
+    }
+    if (tid == 0) soff[nch] = total;
+    __syncthreads();
+    if (total < K) {
+      // the sample misjudged (fewer than K keys at or above its floor): every
+      // position of the row
+      select_topk(n, K, [&](int i) { return order_key(__ldcg(full_row + i)); },
+                  [&](int pos, int i) { out[pos] = i; }, sh);
+    } else {
+      // candidate i lies in the last chunk whose segment starts at or before i
+      auto seg_of = [&](int i) {
+        int a = 0, b = nch - 1;
+        while (a < b) {
+          const int mid = (a + b + 1) >> 1;
+          if (soff[mid] <= i) a = mid;
+          else b = mid - 1;
+        }
+        return a;
+      };
+      if (total <= kLevel2Keys) {
+        // the keys into shared memory (one warp per chunk); positions are read
+        // from global memory for the K selected only
+        const int lane = tid & 31, warp = tid >> 5;
+        for (int c2 = warp; c2 < nch; c2 += kW) {
+          const int o = soff[c2], m2 = soff[c2 + 1] - o;
+          for (int j = lane; j < m2; j += 32) skeys[o + j] = __ldcg(tk + (size_t)c2 * K + j);
+        }
+        __syncthreads();
+        select_topk(total, K, smem_key,
+                    [&](int pos, int i) {
+                      const int g = seg_of(i);
+                      out[pos] = __ldcg(ti + (size_t)g * K + (i - soff[g]));
+                    },
+                    sh);
+      } else {
+      select_topk(total, K,
+                  [&](int i) {
+                    const int g = seg_of(i);
+                    return __ldcg(tk + (size_t)g * K + (i - soff[g]));
+                  },
+                  [&](int pos, int i) {
+                    const int g = seg_of(i);
+                    out[pos] = __ldcg(ti + (size_t)g * K + (i - soff[g]));
+                  },
+                  sh);
+      }
+    }
   }
   if (tid == 0) {
     idx_len[t] = K;  // n > kTopkChunk >= K
@@ -976,7 +1198,8 @@ cudaError_t launch_topk(const sml_problem& p, const float* scores, int32_t* idx,
                       p.num_requests, p.num_tokens, p.topk, p.max_ctx, p.max_pages, p.cu_q, p.ctx_len, scores, idx,
                       idx_len, status);
   }
-  const size_t smem = (size_t)kTopkChunk * sizeof(uint32_t);
+  // chunk keys, or (last CTA of a row) candidate keys, then segment starts
+  const size_t smem = (size_t)kLevel2Keys * sizeof(uint32_t) + (kMaxSegChunks + 1) * sizeof(int);
   cudaError_t e = set_max_smem(reinterpret_cast<const void*>(topk_kernel), smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(topk_kernel, dim3(ws.chunks, p.num_tokens), dim3(kTopkThreads), smem, stream, 0, p.num_requests,

@@ -156,6 +156,26 @@ def test_topk_two_level_rows_with_ties_across_chunks():
     _topk_case([coarse, exact], 100)
 
 
+def test_topk_long_rows_floor_paths():
+    """Rows over eight chunks: a sampled floor cuts each chunk's candidates.
+    Cover the floor's three outcomes: keys above it spread thinly (floor
+    segments), one chunk holding more than K of them (that chunk falls back to
+    its own top K), and a sample that misjudges (only the sampled positions are
+    large, so fewer than K candidates exist and the whole row is selected)."""
+    rng = np.random.default_rng(3)
+    n = 300_000
+    misjudged = np.zeros(n, dtype=np.float32)
+    pos = (np.arange(1024, dtype=np.int64) * n) // 1024          # the kernel's strided sample
+    misjudged[pos] = 10.0 + np.arange(1024, dtype=np.float32) * 1e-3
+    crowded = rng.standard_normal(200_000).astype(np.float32)
+    crowded[49152:65536] += 10.0                                 # one chunk holds every large key
+    ties = rng.standard_normal(500_000).astype(np.float32)
+    ties[rng.choice(500_000, 1000, replace=False)] = 4.0         # ties near the threshold
+    spread = rng.standard_normal(1_048_576).astype(np.float32)
+    _topk_case([misjudged, crowded, ties, spread], 2048)
+    _topk_case([misjudged, crowded, ties], 7)
+
+
 # --- the benchmark workloads at full size -----------------------------------------
 
 def test_batched_decode_full():
