@@ -813,7 +813,15 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
   const float* row = scores + (size_t)t * max_ctx;
 
   // 1. this chunk's keys into shared memory; the row's sample straight from
-  //    global memory (every CTA takes the same sample, so all agree on it).
+  //    global memory (every CTA takes the same sample, so all agree on it),
+  //    its loads issued together with the chunk's.
+  const int ns = min(kSample, n);
+  float sraw[kSample / kTopkThreads];
+#pragma unroll
+  for (int u = 0; u < kSample / kTopkThreads; ++u) {
+    const int j = tid + u * nt;
+    sraw[u] = j < ns ? __ldcg(row + (int)((long long)j * n / ns)) : NAN;
+  }
   if ((reinterpret_cast<uintptr_t>(row + c0) & 15) == 0) {
     // 16-B loads, all of a thread's issued before any is used
     const float4* src = reinterpret_cast<const float4*>(row + c0);
@@ -836,7 +844,6 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
 #pragma unroll 8
     for (int i = tid; i < cn; i += nt) keys[i] = order_key(__ldcg(row + c0 + i));
   }
-  const int ns = min(kSample, n);
   float sv[kSample / kTopkThreads];
   float lo = INFINITY, hi = -INFINITY;
 #pragma unroll
@@ -844,7 +851,7 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
     const int j = tid + u * nt;
     sv[u] = NAN;
     if (j < ns) {
-      sv[u] = key_value(order_key(__ldcg(row + (int)((long long)j * n / ns))));
+      sv[u] = key_value(order_key(sraw[u]));
       if (isfinite(sv[u])) {
         lo = fminf(lo, sv[u]);
         hi = fmaxf(hi, sv[u]);
