@@ -80,6 +80,7 @@ struct __align__(1024) Smem {
   float halpha[kHC];             // this tile's exp(m_old - m_new)
   float hf[kHC];                 // this tile's rescale factor of O
   float hinv[kHC];               // 1 / sigma_h (0 while unset)
+  float hosc[kHC];               // epilogue: sigma_h / l_h, the output scale of head h
   float scw[2][4];               // per-warp max of the tile's scales (double-buffered by tile)
   int32_t rowid[kMaxSplit];      // pool row (page * 64 + row) of each key, -1 = masked
   uint64_t e_full[2], e_free[2];
@@ -649,30 +650,41 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
     ok = softmax_all(ok && warp_wait(&S.pv_done, (ntiles - 1) & 1, abort));
     if (!ok) *abort = 1;
     ptx::tc_fence_after();
-    // Row sums over the 128 key lanes, then the output: sigma_h (hi + mid + lo) / l_h.
+    // Row sums over the 128 key lanes, then each head's output scale
+    // sigma_h / l_h and its log-sum-exp.
     column_reduce<false>(S, row, lrow);
+    if (row < kHC) {
+      const float lsum = S.hstat[row];
+      S.hosc[row] = lsum > 0.f ? S.hsig[row] / lsum : 0.f;
+      P.ws.part_lse[slot0 + (size_t)row * P.ws.splits] = lsum > 0.f ? S.hm[row] + logf(lsum) : -INFINITY;
+    }
+  }
+
+  // Output, sigma_h (hi + mid + lo) / l_h per head, by every warp but the MMA
+  // issuer (the gather warps are idle by now): unit (block b, TMEM lane
+  // quarter q) goes to a warp whose quarter is q.  The named barrier orders
+  // the last PV (the softmax warps waited for it) and S.hosc before the reads;
+  // every path of warps 0-14, a timed-out one included, reaches it.
+  if (warp != kWarpMma) {
+    asm volatile("bar.sync 3, %0;" ::"n"(32 * kWarpMma) : "memory");
+    ptx::tc_fence_after();
+    const int q = warp & 3;
+    const int nq = (kWarpMma - 1 - q) / 4 + 1;   // warps 0..14 with quarter q
     float osc[kHC];
 #pragma unroll
-    for (int h = 0; h < kHC; ++h) {
-      const float ls = S.hstat[h];
-      osc[h] = ls > 0.f ? S.hsig[h] / ls : 0.f;
-    }
+    for (int h = 0; h < kHC; ++h) osc[h] = S.hosc[h];
 #pragma unroll 1
-    for (int b = 0; b < 4; ++b) {
+    for (int b = warp >> 2; b < 4; b += nq) {
       uint32_t ov[32], ow[16];
       ptx::tmem_ld32(T0 + kColO + kOStride * b + lane_off, ov);
       ptx::tmem_ld16(T0 + kColO + kOStride * b + 32 + lane_off, ow);
       ptx::tmem_wait_ld(ov, ow);
-      const int dim = 128 * b + row;
+      const int dim = 128 * b + 32 * q + lane;
 #pragma unroll
       for (int h = 0; h < kHC; ++h) {
         const float o = __uint_as_float(ov[h]) + __uint_as_float(ov[kHC + h]) + __uint_as_float(ow[h]);
         P.ws.part_out[(slot0 + (size_t)h * P.ws.splits) * SML_LATENT_DIM + dim] = o * osc[h];
       }
-    }
-    if (row < kHC) {
-      const float lsum = S.hstat[row];
-      P.ws.part_lse[slot0 + (size_t)row * P.ws.splits] = lsum > 0.f ? S.hm[row] + logf(lsum) : -INFINITY;
     }
   }
 
