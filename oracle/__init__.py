@@ -13,9 +13,11 @@ Modules:
   dsa     -- indexer scores, visible lengths, exact top-k
   mla     -- absorbed-query attention, sparse and dense MLA, LSE merge, one layer
   producers -- FP8 quantisation and the cache writes just before the step
+  dcp     -- the step with the cache sharded by token over ranks (decode
+             context parallelism): candidates, stable merge, LSE combine
 
 Every function is pinned by tests under ``tests/`` (``-m "not gpu"``) to
 values the pages print, closed forms, invariants, library routines and brute
 force on tiny inputs; none is "parity unpinned".
 """
-from . import dsa, formats, mla, producers  # noqa: F401
+from . import dcp, dsa, formats, mla, producers  # noqa: F401

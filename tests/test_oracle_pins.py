@@ -580,3 +580,57 @@ def test_plain_e4m3_writer_round_trip_and_untouched_rows():
     assert np.array_equal(a[~touched], b[~touched])
     nope, _ = PR.write_latent_plain_e4m3(pool0, c[:1], None, np.array([3], dtype=np.int32))
     assert not nope.data[3 * 576 + 512: 4 * 576].any()
+
+
+# --- decode context parallelism: the cache sharded by token over ranks ----------------
+
+from oracle import dcp  # noqa: E402
+
+
+def _dcp_rows():
+    rng = np.random.default_rng(12)
+    vals = np.array([-1.5, -0.0, 0.0, 0.25, 2.0, np.inf, -np.inf, np.nan], dtype=np.float32)
+    rows = [rng.choice(vals, size=n).astype(np.float32) for n in (1, 9, 300, 5000)]
+    rows.append(np.zeros(3000, dtype=np.float32))                              # ties across every rank
+    rows.append(np.round(rng.standard_normal(7000) * 3).astype(np.float32))    # heavy ties
+    rows.append(rng.standard_normal(20000).astype(np.float32))
+    return rows
+
+
+@pytest.mark.parametrize("R,I", [(1, 1), (2, 1), (3, 1), (8, 1), (2, 64), (8, 64), (5, 100)])
+def test_dcp_selection_is_the_unsharded_topk(R, I):
+    for row in _dcp_rows():
+        for k in (1, 7, 64, 2048):
+            got = dcp.select(row, R, I, k)
+            assert np.array_equal(got, dsa.topk_row(row, k)), (R, I, k, len(row))
+
+
+def test_dcp_candidates_hold_the_global_topk_and_at_most_k_each():
+    row = np.round(np.random.default_rng(13).standard_normal(9000) * 2).astype(np.float32)
+    k = 700
+    want = set(dsa.topk_row(row, k).tolist())
+    union = set()
+    for r in range(4):
+        s, p = dcp.rank_candidates(row, r, 4, 1, k)
+        assert len(p) <= k and np.all(dcp.owner(p, 4, 1) == r)
+        assert np.array_equal(s, row[p])
+        union |= set(p.tolist())
+    assert want <= union
+
+
+def test_dcp_attention_is_the_unsharded_sparse_mla(small):
+    wl = small
+    v = wl.view(0)
+    scores = dsa.indexer_scores(v, v.iq8, v.iq_scale, v.iw, wl.index_cache)
+    for R, I in ((2, 1), (3, 64), (8, 64)):
+        for t in range(wl.T):
+            sel = dcp.select(scores[t], R, I, wl.topk)
+            assert np.array_equal(sel, dsa.topk_row(scores[t], wl.topk))
+            out, lse, per_rank = dcp.attention(v, wl.latent, t, sel, R, I)
+            ref_o, ref_l = mla.token_attention(v, wl.latent, t, sel)
+            assert np.allclose(out, ref_o, rtol=1e-12, atol=1e-12)
+            assert np.allclose(lse, ref_l, rtol=1e-12, atol=1e-12)
+            # a rank holding none of the selected tokens has an empty row
+            holders = set(dcp.owner(sel, R, I).tolist())
+            for r in range(R):
+                assert (r in holders) == bool(np.all(np.isfinite(per_rank[r])))
