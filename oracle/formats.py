@@ -93,12 +93,14 @@ def _le_f32(raw: np.ndarray) -> np.ndarray:
 
 def latent_rows(cache, pages: np.ndarray, rows: np.ndarray):
     """Read latent rows (physical page, row in page) from an fp8_ds_mla pool
-    (uint8 bytes) or a ``PlainE4M3Pool``.
+    (uint8 bytes), a ``PlainE4M3Pool`` or a ``Bf16Pool``.
 
     Returns (c_hat [n, 512] = e4m3 * block scale, k_pe [n, 64]) in float64.
     """
     if isinstance(cache, PlainE4M3Pool):
         return plain_e4m3_rows(cache, pages, rows)
+    if isinstance(cache, Bf16Pool):
+        return bf16_rows(cache, pages, rows)
     pages = np.asarray(pages, dtype=np.int64)
     rows = np.asarray(rows, dtype=np.int64)
     start = pages * LATENT_PAGE_BYTES + rows * LATENT_ROW_BYTES
@@ -133,6 +135,26 @@ class PlainE4M3Pool(NamedTuple):
     the pool's fp32 scale."""
     data: np.ndarray
     scale: float
+
+
+BF16_PAGE_BYTES = PAGE_TOKENS * BF16_ROW_BYTES                       # 73,728
+
+
+class Bf16Pool(NamedTuple):
+    """A latent pool in bf16 (blog, section "ROCm 实现细节", paragraph "FP8 潜在
+    缓存": 1,152 B per token per layer in bf16).  Reading: a row is [512 x bf16
+    latent][64 x bf16 RoPE key], little-endian, a page 64 rows back to back."""
+    data: np.ndarray
+
+
+def bf16_rows(pool: Bf16Pool, pages: np.ndarray, rows: np.ndarray):
+    """Read latent rows from a bf16 pool: (c_hat [n, 512], k_pe [n, 64]) in float64."""
+    pages = np.asarray(pages, dtype=np.int64)
+    rows = np.asarray(rows, dtype=np.int64)
+    start = pages * BF16_PAGE_BYTES + rows * BF16_ROW_BYTES
+    raw = pool.data[start[:, None] + np.arange(BF16_ROW_BYTES)[None, :]]
+    v = decode_bf16(np.ascontiguousarray(raw).view("<u2"))
+    return v[:, :LATENT_DIM], v[:, LATENT_DIM:]
 
 
 def plain_e4m3_rows(pool: PlainE4M3Pool, pages: np.ndarray, rows: np.ndarray):

@@ -38,7 +38,8 @@ Readings (the pages print no quantiser):
 
 Byte layouts: those of ``formats`` (fp8_ds_mla row [512 x e4m3][4 x fp32]
 [64 x bf16]; plain E4M3 row [576 x e4m3] under one pool scale that the caller
-gives; indexer page [64 x 128 B keys][64 x fp32 scales]).
+gives; bf16 row [576 x bf16]; indexer page [64 x 128 B keys][64 x fp32
+scales]).
 """
 from __future__ import annotations
 
@@ -158,3 +159,20 @@ def write_latent_plain_e4m3(pool: F.PlainE4M3Pool, c_bits: np.ndarray, kpe_bits,
         start = p * F.PLAIN_E4M3_PAGE_BYTES + r * F.PLAIN_E4M3_ROW_BYTES
         out[start: start + F.PLAIN_E4M3_ROW_BYTES] = row
     return F.PlainE4M3Pool(out, float(s)), bad
+
+
+def write_latent_bf16(pool: F.Bf16Pool, c_bits: np.ndarray, kpe_bits, slot: np.ndarray):
+    """Latent rows (bf16 bits [n, 512]) and RoPE keys (bf16 bits [n, 64], or
+    None: zeros) into a copy of a bf16 pool, stored as given.  Returns (new
+    pool, any slot out of range)."""
+    out = np.array(pool.data, dtype=np.uint8, copy=True)
+    num_pages = out.size // F.BF16_PAGE_BYTES
+    ids, pages, rows, bad = _slots(slot, num_pages)
+    for i, p, r in zip(ids, pages, rows):
+        row = np.zeros(F.LATENT_DIM + F.ROPE_DIM, dtype="<u2")
+        row[:F.LATENT_DIM] = np.asarray(c_bits[i], dtype=np.uint16)
+        if kpe_bits is not None:
+            row[F.LATENT_DIM:] = np.asarray(kpe_bits[i], dtype=np.uint16)
+        start = p * F.BF16_PAGE_BYTES + r * F.BF16_ROW_BYTES
+        out[start: start + F.BF16_ROW_BYTES] = row.view(np.uint8)
+    return F.Bf16Pool(out), bad

@@ -634,3 +634,50 @@ def test_dcp_attention_is_the_unsharded_sparse_mla(small):
             holders = set(dcp.owner(sel, R, I).tolist())
             for r in range(R):
                 assert (r in holders) == bool(np.all(np.isfinite(per_rank[r])))
+
+
+# --- the bf16 latent pool (1,152 B per token) ----------------------------------------
+
+def test_bf16_row_layout_from_independent_packing():
+    assert F.BF16_ROW_BYTES == 1152
+    vals = [((i * 37) % 255 - 127) / 16.0 for i in range(576)]   # at most 7 significant bits: exact in bf16
+    raw = b"".join(struct.pack("<f", v)[2:] for v in vals)      # bf16 = top half of the fp32
+    pool = bytearray(2 * 64 * 1152)
+    page, row = 1, 5
+    off = page * 64 * 1152 + row * 1152
+    pool[off: off + 1152] = raw
+    c, pe = F.bf16_rows(F.Bf16Pool(np.frombuffer(bytes(pool), dtype=np.uint8)), [page], [row])
+    assert np.array_equal(c[0], np.array(vals[:512])) and np.array_equal(pe[0], np.array(vals[512:]))
+
+
+def test_bf16_pool_gives_the_attention_of_an_equal_fp8_ds_mla_pool(small):
+    """E4M3 codes times a power-of-two block scale are bf16 values, so a bf16
+    pool can hold exactly the rows of an fp8_ds_mla pool: same rows, same
+    attention."""
+    wl = small
+    n_rows = wl.num_pages * 64
+    pages = np.arange(wl.num_pages).repeat(64)
+    rows = np.tile(np.arange(64), wl.num_pages)
+    rng = synth.stream(14, "bf16_vs_ds")
+    codes = (rng.integers(0, 0x7F, size=(n_rows, 512)) | (rng.integers(0, 2, (n_rows, 512)) << 7)).astype(np.uint8)
+    scale = np.float32(2.0 ** -6)
+    ds = np.zeros((n_rows, F.LATENT_ROW_BYTES), dtype=np.uint8)
+    ds[:, :512] = codes
+    ds[:, 512:528] = np.full((n_rows, 4), scale, dtype="<f4").view(np.uint8)
+    pe_bits = synth.to_bf16_bits(rng.standard_normal((n_rows, 64)).astype(np.float32))
+    ds[:, 528:] = pe_bits.astype("<u2").view(np.uint8).reshape(n_rows, 128)
+    c_vals = (F.decode_e4m3(codes) * float(scale)).astype(np.float32)
+    c_bits = synth.to_bf16_bits(c_vals)
+    assert np.array_equal(F.decode_bf16(c_bits), c_vals.astype(np.float64))      # exact in bf16
+    b16, bad = PR.write_latent_bf16(F.Bf16Pool(np.zeros(wl.num_pages * F.BF16_PAGE_BYTES, np.uint8)),
+                                    c_bits, pe_bits, np.arange(n_rows, dtype=np.int32))
+    assert not bad
+    c1, p1 = F.latent_rows(b16, pages, rows)
+    c2, p2 = F.latent_rows(ds.reshape(-1), pages, rows)
+    assert np.array_equal(c1, c2) and np.array_equal(p1, p2)
+    v = wl.view(0)
+    idx = np.tile(np.arange(64), (wl.T, 1))
+    ln = np.minimum(64, dsa.visible_lengths(wl.cu_q, wl.ctx_len))
+    o1, l1 = mla.sparse_mla(v, b16, idx, ln)
+    o2, l2 = mla.sparse_mla(v, ds.reshape(-1), idx, ln)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
