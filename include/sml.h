@@ -15,6 +15,9 @@
  *                          the producers just before the step: FP8
  *                          quantisation of new tokens into the two caches,
  *                          and of the indexer queries
+ *   sml_dcp_merge_candidates, sml_dcp_split_selection, sml_lse_combine
+ *                          decode context parallelism: the steps between the
+ *                          ranks' own top-k and sparse MLA
  *
  * Sources: vLLM blog "vLLM 首日支持 Mistral Large 4：1T 参数 MoE 多模态模型",
  * highlights list (MLA with KV LoRA rank 512 and RoPE dim 64; a DSA indexer
@@ -263,6 +266,59 @@ int sml_latent_cache_write(const void* c, const void* k_pe, const int32_t* slot,
  * inputs of sml_indexer_scores.  The indexer's SSMax factor is not folded in
  * here; sml_indexer_scores applies it. */
 int sml_indexer_q_quant(const void* iq, int32_t num_tokens, void* iq8, float* iq_scale, void* stream);
+
+/* ---- decode context parallelism (DCP): the cache sharded by token --------
+ *
+ * vLLM blog "vLLM 首日支持 Mistral Large 4", section "长上下文：解码和预填充的上下文
+ * 并行", paragraph "DCP" and the list after it: the cache is sharded by token
+ * over R ranks; every rank runs the indexer and top-k over its own tokens; the
+ * candidates are exchanged as (score, id) pairs and merged with a stable
+ * top-k; each rank attends over the selected tokens it holds; the partial
+ * outputs are combined by their log-sum-exp.  Reading: token s of a request
+ * lives on rank (s / I) % R at local position (s / (I R)) I + s % I for an
+ * interleave I (I = 64 keeps a page on one rank, so a rank's shard is a local
+ * block table over the same pool).  Every rank's problem is the batch with
+ * its local lengths; the merge compares scores across ranks, so the layers
+ * must run with ssmax = 0 (the SSMax factor would differ per rank).  One
+ * query token per request.  The calls below are the steps between the ranks'
+ * own sml_indexer_scores / sml_topk and their own sml_sparse_mla_decode; the
+ * caller moves the arrays between GPUs. */
+#define SML_DCP_MAX_RANKS 8
+
+/* The ranks' top-k results (host struct; the pointers are device pointers). */
+typedef struct sml_dcp_ranks {
+  int32_t num_ranks;                             /* R, 1..SML_DCP_MAX_RANKS */
+  int32_t interleave;                            /* I >= 1 */
+  const float* scores[SML_DCP_MAX_RANKS];        /* rank r's score matrix [T, score_stride[r]] */
+  int64_t score_stride[SML_DCP_MAX_RANKS];       /* its row stride (that rank's max_ctx) */
+  const int32_t* idx[SML_DCP_MAX_RANKS];         /* rank r's top-k [T, topk], local positions, ascending */
+  const int32_t* idx_len[SML_DCP_MAX_RANKS];     /* [T] */
+} sml_dcp_ranks;
+
+/* Merge: for query t, every rank's candidates (score, global position) in
+ * ascending global position: merged_scores / merged_pos [T, R * topk] (row
+ * stride R * topk), merged_len [T].  sml_topk over them (a problem of T
+ * requests of one token, ctx_len = merged_len, max_ctx = R * topk) selects the
+ * global top-k, ties to the lower global position.  workspace (NULL or >= 256
+ * B) gets SML_FAULT_TOPK_LEN / SML_FAULT_INDEX for bad lengths / positions. */
+int sml_dcp_merge_candidates(const sml_dcp_ranks* ranks, int32_t num_tokens, int32_t topk, float* merged_scores,
+                             int32_t* merged_pos, int32_t* merged_len, void* workspace, void* stream);
+
+/* Split: the selection sel [T, topk] (indices into the merged rows,
+ * ascending) / sel_len [T] back to every rank's compacted list of the
+ * selected tokens it holds: local_idx[r] [T, topk] (local positions,
+ * ascending, -1 padded), local_len[r] [T].  local_idx / local_len are host
+ * arrays of num_ranks device pointers. */
+int sml_dcp_split_selection(int32_t num_ranks, int32_t interleave, int32_t num_tokens, int32_t topk,
+                            const int32_t* sel, const int32_t* sel_len, const int32_t* merged_pos,
+                            int32_t* const* local_idx, int32_t* const* local_len, void* workspace, void* stream);
+
+/* LSE combine of num_parts partial attentions, each normalised by its own
+ * sum: part_out[r] [T, H, 512] (16-B aligned), part_lse[r] [T, H] (host arrays
+ * of device pointers) -> out [T, H, 512], lse [T, H].  A part with lse = -inf
+ * drops out. */
+int sml_lse_combine(int32_t num_parts, int32_t num_tokens, int32_t num_heads, const float* const* part_out,
+                    const float* const* part_lse, float* out, float* lse, void* stream);
 
 /* Synchronise `stream`, then return SML_OK, SML_ERR_DEVICE_FAULT or
  * SML_ERR_TIMEOUT from the workspace's sticky status word (its SML_FAULT_*

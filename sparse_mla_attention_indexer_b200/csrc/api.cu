@@ -394,6 +394,82 @@ int sml_indexer_q_quant(const void* iq, int32_t num_tokens, void* iq8, float* iq
   return e == cudaSuccess ? SML_OK : cuda_fail(e, "sml_indexer_q_quant");
 }
 
+// ---- decode context parallelism -------------------------------------------------------
+
+int sml_dcp_merge_candidates(const sml_dcp_ranks* ranks, int32_t num_tokens, int32_t topk, float* merged_scores,
+                             int32_t* merged_pos, int32_t* merged_len, void* workspace, void* stream) {
+  Checker c;
+  c.check(ranks != nullptr, SML_ERR_INVALID_ARG, "ranks is NULL");
+  c.check(num_tokens >= 0, SML_ERR_INVALID_ARG, "num_tokens < 0");
+  c.check(topk >= 1 && topk <= SML_MAX_TOPK, SML_ERR_UNSUPPORTED, "topk not in [1, 2048]");
+  c.check(workspace == nullptr || aligned(workspace, 256), SML_ERR_WORKSPACE, "workspace not 256-B aligned");
+  if (ranks) {
+    c.check(ranks->num_ranks >= 1 && ranks->num_ranks <= SML_DCP_MAX_RANKS, SML_ERR_UNSUPPORTED,
+            "num_ranks not in [1, SML_DCP_MAX_RANKS]");
+    c.check(ranks->interleave >= 1, SML_ERR_INVALID_ARG, "interleave < 1");
+    const int R = ranks->num_ranks >= 1 && ranks->num_ranks <= SML_DCP_MAX_RANKS ? ranks->num_ranks : 0;
+    for (int r = 0; r < R && num_tokens > 0; ++r) {
+      c.check(ranks->scores[r] != nullptr, SML_ERR_INVALID_ARG, "ranks->scores[r] is NULL");
+      c.check(ranks->idx[r] != nullptr, SML_ERR_INVALID_ARG, "ranks->idx[r] is NULL");
+      c.check(ranks->idx_len[r] != nullptr, SML_ERR_INVALID_ARG, "ranks->idx_len[r] is NULL");
+      c.check(ranks->score_stride[r] >= 1 && ranks->score_stride[r] <= (1 << 30), SML_ERR_INVALID_ARG,
+              "ranks->score_stride[r] not in [1, 2^30]");
+    }
+  }
+  const bool any = num_tokens > 0;
+  c.check(!any || merged_scores != nullptr, SML_ERR_INVALID_ARG, "merged_scores is NULL");
+  c.check(!any || merged_pos != nullptr, SML_ERR_INVALID_ARG, "merged_pos is NULL");
+  c.check(!any || merged_len != nullptr, SML_ERR_INVALID_ARG, "merged_len is NULL");
+  if (c.done("sml_dcp_merge_candidates") != SML_OK) return c.code;
+  cudaError_t e = launch_dcp_merge(*ranks, num_tokens, topk, merged_scores, merged_pos, merged_len,
+                                   workspace ? status_of(workspace) : nullptr, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SML_OK : cuda_fail(e, "sml_dcp_merge_candidates");
+}
+
+int sml_dcp_split_selection(int32_t num_ranks, int32_t interleave, int32_t num_tokens, int32_t topk,
+                            const int32_t* sel, const int32_t* sel_len, const int32_t* merged_pos,
+                            int32_t* const* local_idx, int32_t* const* local_len, void* workspace, void* stream) {
+  Checker c;
+  c.check(num_ranks >= 1 && num_ranks <= SML_DCP_MAX_RANKS, SML_ERR_UNSUPPORTED,
+          "num_ranks not in [1, SML_DCP_MAX_RANKS]");
+  c.check(interleave >= 1, SML_ERR_INVALID_ARG, "interleave < 1");
+  c.check(num_tokens >= 0, SML_ERR_INVALID_ARG, "num_tokens < 0");
+  c.check(topk >= 1 && topk <= SML_MAX_TOPK, SML_ERR_UNSUPPORTED, "topk not in [1, 2048]");
+  c.check(workspace == nullptr || aligned(workspace, 256), SML_ERR_WORKSPACE, "workspace not 256-B aligned");
+  const bool any = num_tokens > 0;
+  c.check(!any || (sel && sel_len && merged_pos), SML_ERR_INVALID_ARG, "sel, sel_len or merged_pos is NULL");
+  c.check(!any || (local_idx && local_len), SML_ERR_INVALID_ARG, "local_idx or local_len is NULL");
+  if (any && local_idx && local_len && num_ranks >= 1 && num_ranks <= SML_DCP_MAX_RANKS)
+    for (int r = 0; r < num_ranks; ++r)
+      c.check(local_idx[r] && local_len[r], SML_ERR_INVALID_ARG, "local_idx[r] or local_len[r] is NULL");
+  if (c.done("sml_dcp_split_selection") != SML_OK) return c.code;
+  cudaError_t e = launch_dcp_split(num_ranks, interleave, num_tokens, topk, sel, sel_len, merged_pos, local_idx,
+                                   local_len, workspace ? status_of(workspace) : nullptr,
+                                   static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SML_OK : cuda_fail(e, "sml_dcp_split_selection");
+}
+
+int sml_lse_combine(int32_t num_parts, int32_t num_tokens, int32_t num_heads, const float* const* part_out,
+                    const float* const* part_lse, float* out, float* lse, void* stream) {
+  Checker c;
+  c.check(num_parts >= 1 && num_parts <= SML_DCP_MAX_RANKS, SML_ERR_UNSUPPORTED,
+          "num_parts not in [1, SML_DCP_MAX_RANKS]");
+  c.check(num_tokens >= 0, SML_ERR_INVALID_ARG, "num_tokens < 0");
+  c.check(num_heads >= 1 && num_heads <= 65535, SML_ERR_INVALID_ARG, "num_heads not in [1, 65535]");
+  const bool any = num_tokens > 0;
+  c.check(!any || (part_out && part_lse), SML_ERR_INVALID_ARG, "part_out or part_lse is NULL");
+  if (any && part_out && part_lse && num_parts >= 1 && num_parts <= SML_DCP_MAX_RANKS)
+    for (int r = 0; r < num_parts; ++r)
+      c.check(part_out[r] && aligned(part_out[r], 16) && part_lse[r], SML_ERR_INVALID_ARG,
+              "part_out[r] NULL or not 16-B aligned, or part_lse[r] NULL");
+  c.check(!any || (out && aligned(out, 16)), SML_ERR_INVALID_ARG, "out NULL or not 16-B aligned");
+  c.check(!any || lse, SML_ERR_INVALID_ARG, "lse is NULL");
+  if (c.done("sml_lse_combine") != SML_OK) return c.code;
+  cudaError_t e = launch_lse_combine(num_parts, num_tokens, num_heads, part_out, part_lse, out, lse,
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SML_OK : cuda_fail(e, "sml_lse_combine");
+}
+
 int sml_read_device_status(void* workspace, int clear, int32_t* bits, void* stream) {
   Checker c;
   c.check(workspace != nullptr, SML_ERR_WORKSPACE, "workspace is NULL");

@@ -155,6 +155,13 @@ cudaError_t launch_indexer_k_write(const void* k, const int32_t* slot, int n, vo
                                    int32_t* status, cudaStream_t stream);
 cudaError_t launch_latent_write(const void* c, const void* kpe, const int32_t* slot, int n, const sml_cache& cache,
                                 int32_t* status, cudaStream_t stream);
+cudaError_t launch_dcp_merge(const sml_dcp_ranks& rk, int T, int K, float* mscore, int32_t* mpos, int32_t* mlen,
+                             int32_t* status, cudaStream_t stream);
+cudaError_t launch_dcp_split(int R, int I, int T, int K, const int32_t* sel, const int32_t* sel_len,
+                             const int32_t* mpos, int32_t* const* local_idx, int32_t* const* local_len,
+                             int32_t* status, cudaStream_t stream);
+cudaError_t launch_lse_combine(int R, int T, int H, const float* const* part_out, const float* const* part_lse,
+                               float* out, float* lse, cudaStream_t stream);
 cudaError_t launch_indexer_q_quant(const void* iq, int T, void* iq8, float* iq_scale, cudaStream_t stream);
 
 }  // namespace sml

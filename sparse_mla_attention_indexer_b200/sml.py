@@ -75,6 +75,17 @@ class Cache(ctypes.Structure):
                 ("scale", ctypes.c_float)]
 
 
+SML_DCP_MAX_RANKS = 8
+
+
+class DcpRanks(ctypes.Structure):
+    _fields_ = [("num_ranks", ctypes.c_int32), ("interleave", ctypes.c_int32),
+                ("scores", ctypes.c_void_p * SML_DCP_MAX_RANKS),
+                ("score_stride", ctypes.c_int64 * SML_DCP_MAX_RANKS),
+                ("idx", ctypes.c_void_p * SML_DCP_MAX_RANKS),
+                ("idx_len", ctypes.c_void_p * SML_DCP_MAX_RANKS)]
+
+
 class E4M3Latent(NamedTuple):
     """A latent pool in the plain per-tensor E4M3 format (576-B rows) and its scale;
     a bare uint8 tensor is an fp8_ds_mla pool."""
@@ -107,12 +118,18 @@ def lib() -> ctypes.CDLL:
         L.sml_indexer_k_cache_write.argtypes = [vp, vp, ctypes.c_int32, Cache, vp, vp]
         L.sml_latent_cache_write.argtypes = [vp, vp, vp, ctypes.c_int32, Cache, vp, vp]
         L.sml_indexer_q_quant.argtypes = [vp, ctypes.c_int32, vp, vp, vp]
+        i32p = ctypes.c_int32
+        L.sml_dcp_merge_candidates.argtypes = [ctypes.POINTER(DcpRanks), i32p, i32p, vp, vp, vp, vp, vp]
+        L.sml_dcp_split_selection.argtypes = [i32p, i32p, i32p, i32p, vp, vp, vp, ctypes.POINTER(vp),
+                                              ctypes.POINTER(vp), vp, vp]
+        L.sml_lse_combine.argtypes = [i32p, i32p, i32p, ctypes.POINTER(vp), ctypes.POINTER(vp), vp, vp, vp]
         L.sml_status_string.argtypes = [i32]
         for name in ("sml_status_string", "sml_last_error", "sml_version"):
             getattr(L, name).restype = ctypes.c_char_p
         for name in ("sml_workspace_init", "sml_indexer_scores", "sml_topk", "sml_sparse_mla_decode",
                      "sml_sparse_mla_decode_noalloc", "sml_run_layer", "sml_read_device_status",
-                     "sml_indexer_k_cache_write", "sml_latent_cache_write", "sml_indexer_q_quant"):
+                     "sml_indexer_k_cache_write", "sml_latent_cache_write", "sml_indexer_q_quant",
+                     "sml_dcp_merge_candidates", "sml_dcp_split_selection", "sml_lse_combine"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -241,6 +258,44 @@ def sml_latent_cache_write(c, k_pe, slot, latent, workspace=None, stream=None):
 def sml_indexer_q_quant(iq, iq8, iq_scale, stream=None):
     """Indexer queries iq [T, 64, 128] bf16 -> iq8 (e4m3 codes, uint8) and iq_scale [T] fp32."""
     _check(lib().sml_indexer_q_quant(_p(iq), _numel(iq_scale), _p(iq8), _p(iq_scale), _s(stream)))
+
+
+def _ptrs(tensors):
+    arr = (ctypes.c_void_p * max(1, len(tensors)))()
+    for i, t in enumerate(tensors):
+        arr[i] = _p(t)
+    return arr
+
+
+def sml_dcp_merge_candidates(scores, idx, idx_len, interleave, topk, merged_scores, merged_pos, merged_len,
+                             workspace=None, stream=None):
+    """Ranks' top-k results (lists of per-rank tensors: scores [T, stride_r],
+    idx [T, topk], idx_len [T]) -> candidates in global position order."""
+    rk = DcpRanks()
+    rk.num_ranks = len(scores)
+    rk.interleave = interleave
+    for r, (sc, ix, ln) in enumerate(zip(scores, idx, idx_len)):
+        rk.scores[r] = _p(sc)
+        rk.score_stride[r] = sc.shape[1]
+        rk.idx[r] = _p(ix)
+        rk.idx_len[r] = _p(ln)
+    _check(lib().sml_dcp_merge_candidates(ctypes.byref(rk), _numel(merged_len), topk, _p(merged_scores),
+                                          _p(merged_pos), _p(merged_len), _p(workspace), _s(stream)))
+
+
+def sml_dcp_split_selection(interleave, topk, sel, sel_len, merged_pos, local_idx, local_len, workspace=None,
+                            stream=None):
+    """Global selection (indices into the merged rows) -> each rank's compacted local list."""
+    _check(lib().sml_dcp_split_selection(len(local_idx), interleave, _numel(sel_len), topk, _p(sel), _p(sel_len),
+                                         _p(merged_pos), _ptrs(local_idx), _ptrs(local_len), _p(workspace),
+                                         _s(stream)))
+
+
+def sml_lse_combine(part_out, part_lse, out, lse, stream=None):
+    """LSE combine of per-rank partial attentions (lists of tensors [T, H, 512] / [T, H])."""
+    T, H = lse.shape
+    _check(lib().sml_lse_combine(len(part_out), T, H, _ptrs(part_out), _ptrs(part_lse), _p(out), _p(lse),
+                                 _s(stream)))
 
 
 def sml_read_device_status(workspace, clear: bool = True, stream=None):

@@ -116,3 +116,22 @@ def test_cache_descriptors_of_both_latent_forms():
     assert (c.num_pages, c.format, c.scale) == (5, sml.SML_LATENT_E4M3, 0.25)
     c = sml.cache(None, sml.INDEX_PAGE_BYTES)
     assert (c.base, c.num_pages, c.format) == (None, 0, 0)
+
+
+def test_dcp_entry_points_reject_bad_arguments_without_cuda(L):
+    rk = sml.DcpRanks()
+    rk.num_ranks = 9
+    rk.interleave = 0
+    code = L.sml_dcp_merge_candidates(ctypes.byref(rk), 4, 2048, None, None, None, None, None)
+    assert code in (sml.SML_ERR_INVALID_ARG, sml.SML_ERR_UNSUPPORTED)
+    msg = sml.sml_last_error()
+    for part in ("num_ranks", "interleave", "merged_scores"):
+        assert part in msg, msg
+    ptrs = (ctypes.c_void_p * 2)(None, None)
+    code = L.sml_dcp_split_selection(2, 64, 3, 2048, 0x1000, 0x2000, 0x3000, ptrs, ptrs, None, None)
+    assert code == sml.SML_ERR_INVALID_ARG and "local_idx[r]" in sml.sml_last_error()
+    outs = (ctypes.c_void_p * 2)(0x1004, 0x2000)
+    lses = (ctypes.c_void_p * 2)(0x3000, 0x4000)
+    code = L.sml_lse_combine(2, 3, 16, outs, lses, 0x5000, 0x6000, None)
+    assert code == sml.SML_ERR_INVALID_ARG and "16-B aligned" in sml.sml_last_error()
+    assert L.sml_lse_combine(2, 0, 16, None, None, None, None, None) == sml.SML_OK
