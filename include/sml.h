@@ -189,8 +189,17 @@ int sml_topk(const sml_problem* p, const float* scores, int32_t* idx, int32_t* i
  *   idx      [T, topk] int32 logical positions (any order; -1 padding ignored)
  *   idx_len  [T] int32 number of valid entries at the front of each idx row
  *   out      [T, H, 512] fp32;  lse [T, H] fp32 (natural log; -inf if empty)
- * Products run on tensor cores in fp16 (dequantised latent, probabilities)
- * with fp32 accumulation; softmax in fp32. */
+ * Arithmetic: both products run on the tensor cores as E4M3 x E4M3 with fp32
+ * accumulation, straight from the cached E4M3 codes (the latent is never
+ * dequantised).  The bf16 query of each head is split exactly into two E4M3
+ * terms, q = s_h (hi + lo), s_h the power of two >= amax_h / 448: exact for
+ * every query element at or above 2^-6 s_h, E4M3's smallest normal step (a
+ * bf16 has 8 significant bits, hi takes 4, lo the other 4); smaller elements
+ * keep an absolute error below 2^-10 s_h (half of E4M3's subnormal step).
+ * The RoPE part (fp8_ds_mla) runs as bf16 x bf16.  The softmax is fp32; each
+ * weight p_i * block scale is split into three E4M3 terms whose sum carries
+ * 12 significant bits, under a per-head power-of-two scale that keeps the
+ * dominant weights in E4M3's normal range. */
 int sml_sparse_mla_decode(const sml_problem* p, const void* q, sml_cache latent,
                           const int32_t* idx, const int32_t* idx_len, float* out, float* lse,
                           void* workspace, size_t ws_bytes, void* stream);
@@ -223,11 +232,21 @@ int sml_run_layer(const sml_problem* p, const void* q, const void* iq8, const fl
  *     call's contents (nothing in it needs to start at zero).  Calls that can
  *     overlap on the GPU (different streams, or several host threads) race on
  *     it: serialise them.
- *   - There is no workspace, so there is no device status word: out-of-range
- *     pages or positions are still masked, but not reported. */
+ *   - There is no workspace, so the device checks (out-of-range pages or
+ *     positions, a bounded wait that gave up) set bits in a status word built
+ *     into the library beside the scratch array: one per device, shared by
+ *     every call on it and sticky until cleared.  Read it with
+ *     sml_noalloc_read_status. */
 int sml_sparse_mla_decode_noalloc(const sml_problem* p, const void* q, sml_cache latent,
                                   const int32_t* idx, const int32_t* idx_len, float* out, float* lse,
                                   void* stream);
+
+/* The status word of sml_sparse_mla_decode_noalloc on the current device, as
+ * sml_read_device_status reads a workspace's: synchronise `stream`, then
+ * return SML_OK, SML_ERR_DEVICE_FAULT or SML_ERR_TIMEOUT (the SML_FAULT_*
+ * bits go to *bits when bits is a host pointer); clear != 0 resets the word.
+ * Allocates nothing.  (The pages have no counterpart.) */
+int sml_noalloc_read_status(int clear, int32_t* bits, void* stream);
 
 /* ---- producers: quantise new tokens and write the caches the step reads ----
  *
@@ -300,7 +319,11 @@ typedef struct sml_dcp_ranks {
  * stride R * topk), merged_len [T].  sml_topk over them (a problem of T
  * requests of one token, ctx_len = merged_len, max_ctx = R * topk) selects the
  * global top-k, ties to the lower global position.  workspace (NULL or >= 256
- * B) gets SML_FAULT_TOPK_LEN / SML_FAULT_INDEX for bad lengths / positions. */
+ * B) gets SML_FAULT_TOPK_LEN / SML_FAULT_INDEX for bad lengths / positions; a
+ * slot that no valid candidate fills holds (NaN, -1), which ranks below every
+ * score and which sml_dcp_split_selection skips (and reports).  Global
+ * positions are int32: every score_stride[r] * num_ranks must fit, else
+ * SML_ERR_UNSUPPORTED. */
 int sml_dcp_merge_candidates(const sml_dcp_ranks* ranks, int32_t num_tokens, int32_t topk, float* merged_scores,
                              int32_t* merged_pos, int32_t* merged_len, void* workspace, void* stream);
 

@@ -414,6 +414,8 @@ int sml_dcp_merge_candidates(const sml_dcp_ranks* ranks, int32_t num_tokens, int
       c.check(ranks->idx_len[r] != nullptr, SML_ERR_INVALID_ARG, "ranks->idx_len[r] is NULL");
       c.check(ranks->score_stride[r] >= 1 && ranks->score_stride[r] <= (1 << 30), SML_ERR_INVALID_ARG,
               "ranks->score_stride[r] not in [1, 2^30]");
+      c.check(ranks->score_stride[r] * (int64_t)R <= INT32_MAX, SML_ERR_UNSUPPORTED,
+              "ranks->score_stride[r] * num_ranks exceeds int32 (global positions are int32)");
     }
   }
   const bool any = num_tokens > 0;

@@ -32,13 +32,16 @@ struct RankOut {
   int32_t* len[SML_DCP_MAX_RANKS];
 };
 
-__device__ __forceinline__ int global_pos(int local, int rank, int R, int I) {
-  return ((local / I) * R + rank) * I + local % I;
+// The host checks that every rank's score stride times R fits in int32, so a
+// valid local position's global position does; the arithmetic runs in int64
+// all the same, so that an invalid one cannot wrap into range.
+__device__ __forceinline__ long long global_pos(int local, int rank, int R, int I) {
+  return ((long long)(local / I) * R + rank) * I + local % I;
 }
 
 // Candidates of query t whose global position is below g on rank r (the
 // rank's list is ascending in local, hence in global, position).
-__device__ __forceinline__ int count_below(const int32_t* list, int n, int g, int r, int R, int I) {
+__device__ __forceinline__ int count_below(const int32_t* list, int n, long long g, int r, int R, int I) {
   int a = 0, b = n;
   while (a < b) {
     const int mid = (a + b) >> 1;
@@ -68,6 +71,14 @@ dcp_merge_kernel(RankArrays ra, int R, int I, int K, float* __restrict__ mscore,
     total += v;
   }
   const size_t row = (size_t)t * R * K;
+  // Every slot of the merged row starts as (NaN, -1): a NaN ranks below every
+  // score in the top-k, and the split skips position -1.  Valid ascending
+  // lists overwrite every slot; an invalid entry (reported) leaves its slot so.
+  for (int m = threadIdx.x; m < total; m += kMergeThreads) {
+    mscore[row + m] = __int_as_float(0x7fc00000);
+    mpos[row + m] = -1;
+  }
+  __syncthreads();
   for (int r = 0; r < R; ++r) {
     const int32_t* list = ra.idx[r] + (size_t)t * K;
     for (int i = threadIdx.x; i < n[r]; i += kMergeThreads) {
@@ -76,12 +87,14 @@ dcp_merge_kernel(RankArrays ra, int R, int I, int K, float* __restrict__ mscore,
         raise_fault(status, SML_FAULT_INDEX);
         continue;
       }
-      const int g = global_pos(l, r, R, I);
+      const long long g = global_pos(l, r, R, I);
       int m = i;
       for (int r2 = 0; r2 < R; ++r2)
         if (r2 != r) m += count_below(ra.idx[r2] + (size_t)t * K, n[r2], g, r2, R, I);
-      mscore[row + m] = __ldg(ra.scores[r] + (size_t)t * ra.stride[r] + l);
-      mpos[row + m] = g;
+      if (m < total) {
+        mscore[row + m] = __ldg(ra.scores[r] + (size_t)t * ra.stride[r] + l);
+        mpos[row + m] = (int32_t)g;
+      }
     }
   }
   if (threadIdx.x == 0) mlen[t] = total;
@@ -108,12 +121,12 @@ dcp_split_kernel(int R, int I, int K, const int32_t* __restrict__ sel, const int
     int owner = -1, local = 0;
     if (i < n) {
       const int m = __ldg(sel + (size_t)t * K + i);
-      if (m >= 0 && m < mstride) {
-        const int g = __ldg(mpos + (size_t)t * mstride + m);
+      const int g = m >= 0 && m < mstride ? __ldg(mpos + (size_t)t * mstride + m) : -1;
+      if (g >= 0) {
         owner = (g / I) % R;
-        local = (g / (I * R)) * I + g % I;
+        local = (int)(((long long)g / ((long long)I * R)) * I + g % I);
       } else {
-        raise_fault(status, SML_FAULT_INDEX);
+        raise_fault(status, SML_FAULT_INDEX);   // a selection outside the row, or an unfilled merge slot
       }
     }
     for (int r = 0; r < R; ++r) {
@@ -139,7 +152,7 @@ __global__ void __launch_bounds__(128)
 lse_combine_kernel(PartArrays pa, int R, int H, float* __restrict__ out, float* __restrict__ lse) {
   ptx::griddep_wait();
   if (threadIdx.x == 0) ptx::griddep_launch_dependents();
-  const int h = blockIdx.x, t = blockIdx.y;
+  const int t = blockIdx.x, h = blockIdx.y;   // tokens on x: gridDim.y is limited to 65,535
   const size_t th = (size_t)t * H + h;
   float mx = -INFINITY;
   for (int r = 0; r < R; ++r) mx = fmaxf(mx, __ldg(pa.lse[r] + th));
@@ -204,7 +217,7 @@ cudaError_t launch_lse_combine(int R, int T, int H, const float* const* part_out
     pa.out[r] = part_out[r];
     pa.lse[r] = part_lse[r];
   }
-  return launch_pdl(lse_combine_kernel, dim3(H, T), dim3(128), 0, stream, 0, pa, R, H, out, lse);
+  return launch_pdl(lse_combine_kernel, dim3(T, H), dim3(128), 0, stream, 0, pa, R, H, out, lse);
 }
 
 }  // namespace sml

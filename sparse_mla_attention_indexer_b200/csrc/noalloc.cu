@@ -15,28 +15,40 @@ namespace sml {
 // libsml.so holds these bytes until the process exits.
 constexpr size_t kNoallocScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+// The sticky device status word of this entry point (SML_FAULT_* bits), in
+// place of the one a workspace would hold; zero when the library loads.
+static __device__ __align__(256) int32_t g_noalloc_status;
 
 namespace {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
+struct DeviceAddrs {
+  void* scratch;
+  int32_t* status;
+};
+DeviceAddrs g_addr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device, looked up once
-// per device (the host-side name of the array is not a device address).
-cudaError_t scratch_address(void** out) {
+// Device addresses of the scratch array and the status word on the current
+// device, looked up once per device (the host-side names of the arrays are not
+// device addresses).
+cudaError_t device_addresses(DeviceAddrs* out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_addr[dev].scratch) {
     void* p = nullptr;
+    void* st = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
+    e = cudaGetSymbolAddress(&st, g_noalloc_status);
+    if (e != cudaSuccess) return e;
+    g_addr[dev].scratch = p;
+    g_addr[dev].status = static_cast<int32_t*>(st);
   }
-  *out = g_scratch_ptr[dev];
+  *out = g_addr[dev];
   return cudaSuccess;
 }
 
@@ -91,15 +103,14 @@ extern "C" int sml_sparse_mla_decode_noalloc(const sml_problem* p, const void* q
     set_last_error(std::string("sml_sparse_mla_decode_noalloc: ") + msg);
     return code;
   }
-  void* base = nullptr;
-  cudaError_t e = scratch_address(&base);
+  DeviceAddrs addr{};
+  cudaError_t e = device_addresses(&addr);
   if (e == cudaSuccess) {
-    char* b = static_cast<char*>(base);
+    char* b = static_cast<char*>(addr.scratch);
     const size_t slots = (size_t)p->num_tokens * p->num_heads * ws.splits;
     ws.part_out = reinterpret_cast<float*>(b);
     ws.part_lse = reinterpret_cast<float*>(b + align_up(slots * SML_LATENT_DIM * sizeof(float)));
-    // No status word: the device checks still mask bad positions and pages.
-    e = launch_sparse_mla(*p, static_cast<const uint16_t*>(q), latent, idx, idx_len, out, lse, ws, nullptr,
+    e = launch_sparse_mla(*p, static_cast<const uint16_t*>(q), latent, idx, idx_len, out, lse, ws, addr.status,
                           static_cast<cudaStream_t>(stream));
   }
   if (e != cudaSuccess) {
@@ -108,4 +119,22 @@ extern "C" int sml_sparse_mla_decode_noalloc(const sml_problem* p, const void* q
   }
   set_last_error("");
   return SML_OK;
+}
+
+extern "C" int sml_noalloc_read_status(int clear, int32_t* bits, void* stream) {
+  DeviceAddrs addr{};
+  cudaError_t e = device_addresses(&addr);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t word = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&word, addr.status, sizeof word, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess && clear) e = cudaMemsetAsync(addr.status, 0, sizeof word, st);
+  if (e != cudaSuccess) {
+    set_last_error(std::string("sml_noalloc_read_status: ") + cudaGetErrorString(e));
+    return SML_ERR_CUDA;
+  }
+  set_last_error("");
+  if (bits) *bits = word;
+  if (word & SML_FAULT_TIMEOUT) return SML_ERR_TIMEOUT;
+  return word ? SML_ERR_DEVICE_FAULT : SML_OK;
 }

@@ -115,6 +115,7 @@ def lib() -> ctypes.CDLL:
         L.sml_sparse_mla_decode_noalloc.argtypes = [pp, vp, Cache, vp, vp, vp, vp, vp]
         L.sml_run_layer.argtypes = [pp, vp, vp, vp, vp, Cache, Cache, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sml_read_device_status.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_int32), vp]
+        L.sml_noalloc_read_status.argtypes = [i32, ctypes.POINTER(ctypes.c_int32), vp]
         L.sml_indexer_k_cache_write.argtypes = [vp, vp, ctypes.c_int32, Cache, vp, vp]
         L.sml_latent_cache_write.argtypes = [vp, vp, vp, ctypes.c_int32, Cache, vp, vp]
         L.sml_indexer_q_quant.argtypes = [vp, ctypes.c_int32, vp, vp, vp]
@@ -128,6 +129,7 @@ def lib() -> ctypes.CDLL:
             getattr(L, name).restype = ctypes.c_char_p
         for name in ("sml_workspace_init", "sml_indexer_scores", "sml_topk", "sml_sparse_mla_decode",
                      "sml_sparse_mla_decode_noalloc", "sml_run_layer", "sml_read_device_status",
+                     "sml_noalloc_read_status",
                      "sml_indexer_k_cache_write", "sml_latent_cache_write", "sml_indexer_q_quant",
                      "sml_dcp_merge_candidates", "sml_dcp_split_selection", "sml_lse_combine"):
             getattr(L, name).restype = ctypes.c_int
@@ -232,6 +234,16 @@ def sml_sparse_mla_decode_noalloc(problem, q, latent, idx, idx_len, out, lse, st
     _check(lib().sml_sparse_mla_decode_noalloc(ctypes.byref(problem), _p(q),
                                                latent_cache(latent), _p(idx),
                                                _p(idx_len), _p(out), _p(lse), _s(stream)))
+
+
+def sml_noalloc_read_status(clear: bool = False, stream=None):
+    """(status code, SML_FAULT_* bits) of the no-allocation entry point's own
+    status word on the current device; synchronises the stream."""
+    bits = ctypes.c_int32(0)
+    code = lib().sml_noalloc_read_status(int(clear), ctypes.byref(bits), _s(stream))
+    if code == SML_ERR_CUDA:
+        _check(code)
+    return code, bits.value
 
 
 def sml_run_layer(problem, q, iq8, iq_scale, iw, latent, index_cache, reuse_idx, reuse_len,

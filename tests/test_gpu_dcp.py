@@ -10,6 +10,7 @@ import torch
 
 from sparse_mla_attention_indexer_b200 import sml, synth
 from sparse_mla_attention_indexer_b200.device import DeviceWorkload
+from oracle import dcp as odcp
 from tests import parity
 
 pytestmark = pytest.mark.gpu
@@ -98,7 +99,26 @@ def run_dcp(dw, wl, R, I):
     for t in range(T):
         gsel[t, :sel_len_h[t]] = pos_h[t, sel_h[t, :sel_len_h[t]]]
     return dict(sel=gsel, sel_len=sel_len_h, out=out.cpu().numpy(), lse=lse.cpu().numpy(),
-                local_len=np.stack([x.cpu().numpy() for x in local_len]))
+                local_len=np.stack([x.cpu().numpy() for x in local_len]),
+                rank_scores=[x["scores"].cpu().numpy() for x in ranks])
+
+
+def global_rows(wl, rank_scores, R, I):
+    """Each query's visible score row in global positions, assembled from the
+    ranks' own score rows (token s of a request is local position
+    (s // (I R)) I + s % I on rank (s // I) % R)."""
+    n_all = parity.dsa.visible_lengths(wl.cu_q, wl.ctx_len)
+    rows = []
+    for t in range(wl.T):
+        s = np.arange(int(n_all[t]))
+        rank = (s // I) % R
+        local = (s // (I * R)) * I + s % I
+        row = np.empty(len(s), dtype=np.float32)
+        for r in range(R):
+            m = rank == r
+            row[m] = rank_scores[r][t, local[m]]
+        rows.append(row)
+    return rows
 
 
 @pytest.mark.parametrize("R,I,K", [(2, 64, 2048), (4, 64, 2048), (8, 128, 2048), (3, 64, 128)])
@@ -115,7 +135,15 @@ def test_dcp_equals_the_unsharded_step(R, I, K):
     sml.sml_topk(p, scores, idx, ln, ws)
     assert sml.sml_read_device_status(ws)[0] == sml.SML_OK
     ref_idx, ref_len = idx.cpu().numpy(), ln.cpu().numpy()
+    parity.check_topk(wl, scores.cpu().numpy(), ref_idx, ref_len)
     got = run_dcp(dw, wl, R, I)
+    # the oracle's DCP selection (per-rank candidates, stable merge) over the
+    # ranks' own score rows
+    for t, row in enumerate(global_rows(wl, got["rank_scores"], R, I)):
+        want = odcp.select(row, R, I, K)
+        assert got["sel_len"][t] == len(want), f"token {t}: len"
+        assert np.array_equal(got["sel"][t, :len(want)], want), f"token {t}: selection differs from the oracle"
+    # and the unsharded step's selection
     assert np.array_equal(got["sel_len"], ref_len)
     for t in range(wl.T):
         assert np.array_equal(got["sel"][t, :ref_len[t]], ref_idx[t, :ref_len[t]]), f"token {t}"
