@@ -43,11 +43,15 @@ from sparse_mla_attention_indexer_b200 import sml, synth  # noqa: E402
 from sparse_mla_attention_indexer_b200.device import DeviceWorkload  # noqa: E402
 
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 FLUSH_BYTES = 256 << 20
 # dram__bytes_read.sum + dram__bytes_write.sum of one indexer launch on this
 # workload, from the ncu capture summarised in profiles/ (None = not captured
 # for the current kernel).
 INDEXER_NCU_TRAFFIC_BYTES = 164_824_320
+# The same for one sparse-MLA launch (the merge not included); None once the
+# kernel has changed since the counters were taken.
+MLA_NCU_TRAFFIC_BYTES = None
 
 
 def dist_env():
@@ -58,32 +62,18 @@ def dist_env():
 
 
 def peaks():
+    """Roofline denominators: the driver's measured HBM copy bandwidth and
+    bf16 dense GEMM rate (burst: every kernel here is timed alone), else the
+    pool's fallback figures.  FP8 dense = 2 x bf16 (the nominal ratio,
+    4.5 / 2.25 PFLOP/s); it is not measured separately."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
+        hbm, bf16, kind = float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
-
-
-def workload_units(wl):
-    """Algorithmic bytes of the indexer scan and gathered tokens of the attention."""
-    from_ctx = 0
-    n_sum = 0
-    cu = wl.cu_q
-    for r in range(wl.B):
-        Q = int(cu[r + 1] - cu[r])
-        L = int(wl.ctx_len[r])
-        from_ctx += L                      # every visible cache token read once per request
-        n_sum += sum(L - Q + j + 1 for j in range(Q))
-    idx_bytes = from_ctx * 132 + n_sum * 4 + wl.T * (64 * 128 + 4 + 64 * 4)
-    gathered = sum(min(wl.topk, n) for n in _visible(wl))
-    rope = wl.layers[0].rope_dim
-    mla_bytes = gathered * (656 if rope else 528)
-    mla_flops = gathered * 2 * wl.num_heads * ((512 + rope) + 512)
-    return dict(indexer_bytes=idx_bytes, gathered=gathered, mla_bytes=mla_bytes, mla_flops=mla_flops,
-                topk_bytes=n_sum * 4)
+        hbm, bf16, kind = FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+    return dict(hbm_gbs=hbm, bf16_tflops=bf16, fp8_tflops=2.0 * bf16, source=kind)
 
 
 def _visible(wl):
@@ -93,6 +83,38 @@ def _visible(wl):
         L = int(wl.ctx_len[r])
         out += [L - Q + j + 1 for j in range(Q)]
     return out
+
+
+def layer_units(wl, i):
+    """Algorithmic work of layer i of a workload (one stage call each):
+
+    * indexer: 132 B per visible cache token read once per request (keys and
+      scales), 4 B per score written, and the query inputs (64 x 128 E4M3
+      codes, a scale and 64 head weights per query token); FLOPs 2 * 64 * 128
+      per (query token, visible position);
+    * top-k: 4 B per visible score read;
+    * sparse MLA: 656 B per selected row (528 for a NoPE layer, which skips
+      the RoPE key), and 2 * H * ((512 + rope_dim) + 512) FLOPs per selected
+      row (QK^T and PV).  Rows are counted once per query that selects them:
+      the same row selected by two queries counts twice."""
+    lay = wl.layers[i]
+    vis = _visible(wl)
+    from_ctx = int(np.sum(wl.ctx_len.astype(np.int64)))
+    n_sum = int(np.sum(vis))
+    gathered = int(sum(min(wl.topk, n) for n in vis))
+    rope = lay.rope_dim
+    u = dict(gathered=gathered,
+             mla_bytes=gathered * (656 if rope else 528),
+             mla_flops=gathered * 2 * wl.num_heads * ((512 + rope) + 512))
+    if lay.reuse_from is None:
+        u.update(indexer_bytes=from_ctx * 132 + n_sum * 4 + wl.T * (64 * 128 + 4 + 64 * 4),
+                 indexer_flops=n_sum * 2 * 64 * 128, topk_bytes=n_sum * 4)
+    return u
+
+
+def workload_units(wl):
+    """Layer 0's units (the one-layer workloads)."""
+    return layer_units(wl, 0)
 
 
 class ClockSampler:
@@ -147,102 +169,138 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def time_ours(args, wl, rank):
-    dw = DeviceWorkload(wl)
-    p = dw.problem(0)
-    lay = dw.layers[0]
-    ws = dw.workspace(sml.SML_STAGE_LAYER)
-    idx, ln, out, lse = dw.outputs()
-    scores = dw.scores()
-    flush = L2Flush()
+_cudart = None
+
+
+def _record(e, st, capturing):
+    """Record event e on stream st; during graph capture the runtime's
+    "external" record flag makes it a timing node of the graph."""
+    global _cudart
+    if not capturing:
+        e.record(st)
+        return
+    if _cudart is None:
+        _cudart = ctypes.CDLL("libcudart.so.12")
+        _cudart.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
+    rc = _cudart.cudaEventRecordWithFlags(ctypes.c_void_p(e.cuda_event), ctypes.c_void_p(st.cuda_stream), 1)
+    if rc != 0:
+        raise RuntimeError(f"cudaEventRecordWithFlags failed: {rc}")
+
+
+class Step:
+    """The stage calls of one step of a workload, in order: per layer, the
+    indexer and the top-k (unless the layer reuses an earlier layer's top-k),
+    then the sparse MLA (with its merge).  Every layer has its own outputs;
+    the score matrix and the workspace are shared."""
+
+    def __init__(self, wl):
+        self.wl = wl
+        self.dw = dw = DeviceWorkload(wl)
+        self.ws = dw.workspace(sml.SML_STAGE_LAYER)
+        self.scores = dw.scores()
+        self.outs = [dw.outputs() for _ in dw.layers]
+        self.calls = []                     # (label, layer, fn(stream))
+        multi = len(dw.layers) > 1
+        for i, lay in enumerate(dw.layers):
+            p = dw.problem(i)
+            idx, ln, out, lse = self.outs[i]
+            tag = f"{wl.layers[i].name or i}." if multi else ""
+            if lay.reuse_from is None:
+                self.calls.append((tag + "indexer", i, self._indexer(p, lay)))
+                self.calls.append((tag + "topk", i, self._topk(p, idx, ln)))
+                use = (idx, ln)
+            else:
+                use = self.outs[lay.reuse_from][:2]
+            self.calls.append((tag + "sparse_mla_and_merge", i, self._mla(p, lay, use, out, lse)))
+
+    def _indexer(self, p, lay):
+        return lambda st: sml.sml_indexer_scores(p, lay.iq8, lay.iq_scale, lay.iw, self.dw.index_cache,
+                                                 self.scores, self.ws, st)
+
+    def _topk(self, p, idx, ln):
+        return lambda st: sml.sml_topk(p, self.scores, idx, ln, self.ws, st)
+
+    def _mla(self, p, lay, use, out, lse):
+        return lambda st: sml.sml_sparse_mla_decode(p, lay.q, self.dw.latent, use[0], use[1], out, lse,
+                                                    self.ws, st)
+
+    def check_status(self):
+        code, bits = sml.sml_read_device_status(self.ws)
+        if code != sml.SML_OK:
+            raise RuntimeError(f"device status {code} bits {bits:#x}")
+
+
+def time_step(step: Step, steps: int, warmup: int, flush):
+    """Time a workload's step as a CUDA-graph replay (events around it, after
+    an L2 flush), and its stages from a second graph with an event between
+    every two calls.  Returns (step ms [steps], stage ms [steps, calls])."""
     stream = torch.cuda.current_stream()
+    n = len(step.calls)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
 
-    # One step = the three stage calls, captured once into a CUDA graph.  The
-    # kernels are launched with programmatic stream serialization, so in the
-    # graph each may start while the one before it drains; events between the
-    # stages would cut those edges, so the step is timed from events around
-    # the replay, and a second graph with an event between stages gives the
-    # per-stage times (its own loop after the timed one).
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-    cudart = ctypes.CDLL("libcudart.so.12")
-    cudart.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
+    def run(st, capturing=False, events=False):
+        for j, (_, _, fn) in enumerate(step.calls):
+            if events:
+                _record(ev[j], st, capturing)
+            fn(st)
+        if events:
+            _record(ev[n], st, capturing)
 
-    def record(e, st, capturing):
-        # events recorded during capture become timing nodes only with the
-        # runtime's "external" record flag
-        if capturing:
-            rc = cudart.cudaEventRecordWithFlags(ctypes.c_void_p(e.cuda_event), ctypes.c_void_p(st.cuda_stream), 1)
-            if rc != 0:
-                raise RuntimeError(f"cudaEventRecordWithFlags failed: {rc}")
-        else:
-            e.record(st)
-
-    def step(st, capturing=False, events=False):
-        if events:
-            record(ev[0], st, capturing)
-        sml.sml_indexer_scores(p, lay.iq8, lay.iq_scale, lay.iw, dw.index_cache, scores, ws, st)
-        if events:
-            record(ev[1], st, capturing)
-        sml.sml_topk(p, scores, idx, ln, ws, st)
-        if events:
-            record(ev[2], st, capturing)
-        sml.sml_sparse_mla_decode(p, lay.q, dw.latent, idx, ln, out, lse, ws, st)
-        if events:
-            record(ev[3], st, capturing)
-
-    step(stream, events=True)          # first calls outside capture (per-device set-up, events created)
+    # The kernels are launched with programmatic stream serialization, so in
+    # the graph each may start while the one before it drains; events between
+    # the stages would cut those edges, so the step is timed around the
+    # replay and the per-stage graph is timed in a loop of its own.
+    run(stream, events=True)       # first calls outside capture (per-device set-up)
     torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
+    step.check_status()
+    graph, graph_ev = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        step(torch.cuda.current_stream(), capturing=True)
-    graph_ev = torch.cuda.CUDAGraph()
+        run(torch.cuda.current_stream(), capturing=True)
     with torch.cuda.graph(graph_ev):
-        step(torch.cuda.current_stream(), capturing=True, events=True)
-    for _ in range(args.warmup):
+        run(torch.cuda.current_stream(), capturing=True, events=True)
+    for _ in range(warmup):
         flush()
         graph.replay()
         flush()
         graph_ev.replay()
     torch.cuda.synchronize()
-    code, bits = sml.sml_read_device_status(ws)
-    if code != sml.SML_OK:
-        raise RuntimeError(f"device status {code} bits {bits:#x}")
-
+    step.check_status()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     step_ms = []
     barrier()
     torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clocks:
-        for _ in range(args.steps):
-            flush()
-            t0.record(stream)
-            graph.replay()
-            t1.record(stream)
-            torch.cuda.synchronize()
-            step_ms.append(t0.elapsed_time(t1))
-        barrier()
+    for _ in range(steps):
+        flush()
+        t0.record(stream)
+        graph.replay()
+        t1.record(stream)
         torch.cuda.synchronize()
-    # per-stage breakdown (the same steps with events between the stages)
+        step_ms.append(t0.elapsed_time(t1))
+    barrier()
+    torch.cuda.synchronize()
     rows = []
-    for _ in range(args.steps):
+    for _ in range(steps):
         flush()
         graph_ev.replay()
         torch.cuda.synchronize()
-        rows.append([ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]), ev[2].elapsed_time(ev[3]),
-                     ev[0].elapsed_time(ev[3])])
-    per = np.array(rows)
-    per = np.concatenate([per, np.array(step_ms)[:, None]], axis=1)
+        rows.append([ev[j].elapsed_time(ev[j + 1]) for j in range(n)])
     del graph, graph_ev
-    code, bits = sml.sml_read_device_status(ws)
-    if code != sml.SML_OK:
-        raise RuntimeError(f"device status {code} bits {bits:#x}")
+    step.check_status()
+    return np.array(step_ms), np.array(rows)
 
-    # End to end through the one-call entry point from pinned host memory:
-    # per step, copy the step's inputs (queries, indexer queries, batch
-    # metadata) host -> device, run the layer, read the outputs back.  The
-    # inputs sit in one pinned buffer and one device buffer (the tensors are
-    # views into it at 256-B aligned offsets), and the outputs likewise, so a
-    # step is one copy each way.
+
+def time_e2e(step: Step, steps: int, warmup: int, flush):
+    """End to end through the one-call entry point from pinned host memory:
+    per step, copy the step's inputs (queries, indexer queries, batch
+    metadata) host -> device, run the layer, read the outputs back.  The
+    inputs sit in one pinned buffer and one device buffer (the tensors are
+    views into it at 256-B aligned offsets), and the outputs likewise, so a
+    step is one copy each way.  Returns (ms, h2d bytes, d2h bytes)."""
+    dw, wl = step.dw, step.wl
+    lay = dw.layers[0]
+    idx, ln, out, lse = step.outs[0]
+    stream = torch.cuda.current_stream()
+
     def packed(tensors, device):
         offs, total = [], 0
         for t in tensors:
@@ -262,49 +320,55 @@ def time_ours(args, wl, rank):
     d_outb, (o_out, o_lse, o_idx, o_len) = packed([out, lse, idx, ln], "cuda")
     h_out = torch.empty_like(d_outb, device="cpu").pin_memory()
     q_v, iq8_v, iqs_v, iw_v, cu_v, ctx_v, bt_v = dv
-    wlx = dw.wl
-    p_e2e = sml.make_problem(num_heads=wlx.num_heads, topk=wlx.topk, rope_dim=lay.rope_dim, cu_q=cu_v,
-                             ctx_len=ctx_v, block_table=bt_v, max_ctx=wlx.max_ctx, ssmax=wlx.ssmax,
-                             sm_scale=wlx.sm_scale, ssmax_s=wlx.ssmax_s, ssmax_s_index=wlx.ssmax_s_index,
-                             num_tokens=wlx.T)
-    h2d = h_in.numel()
-    d2h = h_out.numel()
+    p_e2e = sml.make_problem(num_heads=wl.num_heads, topk=wl.topk, rope_dim=lay.rope_dim, cu_q=cu_v,
+                             ctx_len=ctx_v, block_table=bt_v, max_ctx=wl.max_ctx, ssmax=wl.ssmax,
+                             sm_scale=wl.sm_scale, ssmax_s=wl.ssmax_s, ssmax_s_index=wl.ssmax_s_index,
+                             num_tokens=wl.T)
     e2e_ms = []
-    for i in range(args.warmup + args.steps):
+    for i in range(warmup + steps):
         flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         d_in.copy_(h_in, non_blocking=True)
         sml.sml_run_layer(p_e2e, q_v, iq8_v, iqs_v, iw_v, dw.latent, dw.index_cache, None, None,
-                          o_idx, o_len, o_out, o_lse, ws, stream)
+                          o_idx, o_len, o_out, o_lse, step.ws, stream)
         h_out.copy_(d_outb, non_blocking=True)
         e1.record(stream)
         stream.synchronize()
-        if i >= args.warmup:
+        if i >= warmup:
             e2e_ms.append(e0.elapsed_time(e1))
-    # The same attention over a plain per-tensor E4M3 latent pool (576-B rows)
-    # with the same block table and selection: one graph of the MLA call.
+    step.check_status()
+    return float(np.mean(e2e_ms)), h_in.numel(), h_out.numel()
+
+
+def time_plain_pool(step: Step, steps: int, warmup: int, flush):
+    """The same attention over a plain per-tensor E4M3 latent pool (576-B
+    rows) with the same block table and selection: one graph of the MLA call."""
+    dw, wl = step.dw, step.wl
+    p = dw.problem(0)
+    lay = dw.layers[0]
+    idx, ln, out, lse = step.outs[0]
+    stream = torch.cuda.current_stream()
     plain = torch.from_numpy(synth.plain_pool(0, wl.name + "/plain_pool", wl.num_pages)).cuda()
     lat_plain = sml.E4M3Latent(plain, synth.PLAIN_SCALE)
-    g_plain = torch.cuda.CUDAGraph()
-    sml.sml_sparse_mla_decode(p, lay.q, lat_plain, idx, ln, out, lse, ws, stream)
+    g = torch.cuda.CUDAGraph()
+    sml.sml_sparse_mla_decode(p, lay.q, lat_plain, idx, ln, out, lse, step.ws, stream)
     torch.cuda.synchronize()
-    with torch.cuda.graph(g_plain):
-        sml.sml_sparse_mla_decode(p, lay.q, lat_plain, idx, ln, out, lse, ws, torch.cuda.current_stream())
-    plain_ms = []
-    for i in range(args.warmup + args.steps):
+    with torch.cuda.graph(g):
+        sml.sml_sparse_mla_decode(p, lay.q, lat_plain, idx, ln, out, lse, step.ws, torch.cuda.current_stream())
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = []
+    for i in range(warmup + steps):
         flush()
         t0.record(stream)
-        g_plain.replay()
+        g.replay()
         t1.record(stream)
         torch.cuda.synchronize()
-        if i >= args.warmup:
-            plain_ms.append(t0.elapsed_time(t1))
-    del g_plain
-    code, bits = sml.sml_read_device_status(ws)
-    if code != sml.SML_OK:
-        raise RuntimeError(f"device status {code} bits {bits:#x}")
-    return per, clocks.summary(), float(np.mean(e2e_ms)), h2d, d2h, float(np.mean(plain_ms))
+        if i >= warmup:
+            ms.append(t0.elapsed_time(t1))
+    del g
+    step.check_status()
+    return float(np.mean(ms))
 
 
 # Algorithmic bytes per new token of the producers: bf16 inputs and the int32
@@ -428,6 +492,70 @@ def config_of(wl, args, n_gpus):
                   "(the write-backs finish before the timed region)", "parallelism": f"replicas x{n_gpus}"}
 
 
+def mla_roofline(u, ms, pk, traffic=None):
+    """Sparse MLA (+ merge) against the slower of its FLOPs at the bf16 tensor
+    peak and its gathered bytes at the HBM peak.  The algorithmic contraction
+    is a bf16 query against dequantised latent rows, so bf16 is its dtype
+    (the kernel itself runs it as exact E4M3 x E4M3 products); the fraction
+    against the FP8 peak is given too."""
+    t_bytes = u["mla_bytes"] / (pk["hbm_gbs"] * 1e9)
+    t_flops = u["mla_flops"] / (pk["bf16_tflops"] * 1e12)
+    sec = ms / 1e3
+    hbm = t_bytes >= t_flops
+    achieved = u["mla_bytes"] / sec / 1e9 if hbm else u["mla_flops"] / sec / 1e12
+    peak = pk["hbm_gbs"] if hbm else pk["bf16_tflops"]
+    return {"kernel": "sparse MLA + LSE merge", "bound": "hbm" if hbm else "tensor", "achieved": achieved,
+            "peak": peak, "unit": "GB/s" if hbm else "TFLOP/s", "frac": achieved / peak,
+            "roofline_us": max(t_bytes, t_flops) * 1e6, "measured_us": ms * 1e3,
+            "gbs": u["mla_bytes"] / sec / 1e9, "tflops": u["mla_flops"] / sec / 1e12,
+            "frac_of_fp8_peak": u["mla_flops"] / sec / 1e12 / pk["fp8_tflops"],
+            "algorithmic_bytes_per_launch": u["mla_bytes"], "algorithmic_flops_per_launch": u["mla_flops"],
+            "peak_source": pk["source"], "traffic": traffic}
+
+
+def indexer_roofline(u, ms, pk, traffic=None):
+    """Indexer scores against the slower of its bytes at the HBM peak and its
+    FP8 products at the FP8 tensor peak (2 x the measured bf16 rate)."""
+    sec = ms / 1e3
+    t_bytes = u["indexer_bytes"] / (pk["hbm_gbs"] * 1e9)
+    t_flops = u["indexer_flops"] / (pk["fp8_tflops"] * 1e12)
+    hbm = t_bytes >= t_flops
+    gbs = u["indexer_bytes"] / sec / 1e9
+    tflops = u["indexer_flops"] / sec / 1e12
+    achieved, peak = (gbs, pk["hbm_gbs"]) if hbm else (tflops, pk["fp8_tflops"])
+    return {"kernel": "indexer scores", "bound": "hbm" if hbm else "tensor", "achieved": achieved, "peak": peak,
+            "unit": "GB/s" if hbm else "TFLOP/s", "frac": achieved / peak, "gbs": gbs,
+            "frac_of_hbm": gbs / pk["hbm_gbs"], "frac_of_8000_gbs": gbs / 8000.0, "tflops": tflops,
+            "frac_of_fp8_peak": tflops / pk["fp8_tflops"], "roofline_us": max(t_bytes, t_flops) * 1e6,
+            "measured_us": ms * 1e3, "algorithmic_bytes_per_launch": u["indexer_bytes"],
+            "algorithmic_flops_per_launch": u["indexer_flops"], "peak_source": pk["source"], "traffic": traffic}
+
+
+def workload_report(wl, step, step_ms, stage_ms, pk):
+    """Per-workload figures: step time, rates, and every stage with its roofline."""
+    ms = float(step_ms.mean())
+    st = {label: float(stage_ms[:, j].mean()) for j, (label, _, _) in enumerate(step.calls)}
+    layers = {}
+    gathered = 0
+    for j, (label, i, _) in enumerate(step.calls):
+        u = layer_units(wl, i)
+        name = wl.layers[i].name or str(i)
+        d = layers.setdefault(name, {})
+        t = st[label]
+        if label.endswith("indexer"):
+            d["indexer"] = indexer_roofline(u, t, pk)
+        elif label.endswith("topk"):
+            d["topk"] = {"measured_us": t * 1e3, "gbs": u["topk_bytes"] / (t / 1e3) / 1e9,
+                         "algorithmic_bytes_per_launch": u["topk_bytes"]}
+        else:
+            d["sparse_mla"] = mla_roofline(u, t, pk)
+            gathered += u["gathered"]
+    return {"ms_per_step": ms, "queries_per_s": wl.T / (ms / 1e3), "gathered_tokens_per_s": gathered / (ms / 1e3),
+            "query_tokens": wl.T, "requests": wl.B, "mla_heads": wl.num_heads, "ssmax": bool(wl.ssmax),
+            "ctx_tokens_total": int(wl.ctx_len.sum()), "stage_ms": st,
+            "step_with_stage_events_ms": float(stage_ms.sum(axis=1).mean()), "layers": layers}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -435,6 +563,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="batched_decode", choices=sorted(synth.SUITE))
+    ap.add_argument("--workloads", default="all",
+                    help="the other workloads to time for the 'workloads' object: 'all', 'none' or a "
+                         "comma-separated list")
     args = ap.parse_args()
     world, rank, local = dist_env()
     metric = "sparse-MLA decode queries/s (indexer + top-2048 + sparse MLA, one layer)"
@@ -464,24 +595,48 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     else:
         torch.cuda.set_device(0)
+    pk = peaks()
+    if args.workloads == "all":
+        others = [w for w in synth.SUITE if w != args.workload]
+    elif args.workloads == "none":
+        others = []
+    else:
+        others = [w for w in args.workloads.split(",") if w and w != args.workload]
     wl = synth.SUITE[args.workload](seed=0)
     units = workload_units(wl)
-    per, clocks, e2e_ms, h2d, d2h, plain_ms = time_ours(args, wl, rank)
-    ms_step = max_over_ranks(float(per[:, 4].mean()))
-    ms_staged = max_over_ranks(float(per[:, 3].mean()))
-    ms_idx = max_over_ranks(float(per[:, 0].mean()))
-    ms_topk = max_over_ranks(float(per[:, 1].mean()))
-    ms_mla = max_over_ranks(float(per[:, 2].mean()))
+    flush = L2Flush()
+    step = Step(wl)
+    reports = {}
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        step_ms, stage_ms = time_step(step, args.steps, args.warmup, flush)
+        e2e_ms, h2d, d2h = time_e2e(step, args.steps, args.warmup, flush)
+        plain_ms = time_plain_pool(step, args.steps, args.warmup, flush)
+        reports[wl.name] = workload_report(wl, step, step_ms, stage_ms, pk)
+        del step
+        # the other workloads, each its own step (every rank alike)
+        for name in others:
+            w = synth.SUITE[name](seed=0)
+            s2 = Step(w)
+            sm2, st2 = time_step(s2, args.steps, args.warmup, flush)
+            reports[name] = workload_report(w, s2, sm2, st2, pk)
+            del s2, w
+            torch.cuda.empty_cache()
+    clk = clocks.summary()
+    ms_step = max_over_ranks(float(step_ms.mean()))
+    ms_idx = max_over_ranks(float(stage_ms[:, 0].mean()))
+    ms_topk = max_over_ranks(float(stage_ms[:, 1].mean()))
+    ms_mla = max_over_ranks(float(stage_ms[:, 2].mean()))
+    ms_staged = max_over_ranks(float(stage_ms.sum(axis=1).mean()))
     e2e_ms = max_over_ranks(e2e_ms)
-    peak, peak_kind = peaks()
-    producers = time_producers(wl.T, args.steps, peak) if rank == 0 else None
+    producers = time_producers(wl.T, args.steps, pk["hbm_gbs"]) if rank == 0 else None
     cb = cpu_baseline(wl) if rank == 0 and world == 1 else None
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank != 0:
         return
     qps = whole_job_rate(world, wl.T, ms_step)
-    idx_gbs = units["indexer_bytes"] / (ms_idx / 1e3) / 1e9
+    idx_rf = indexer_roofline(units, ms_idx, pk, INDEXER_NCU_TRAFFIC_BYTES)
+    mla_rf = mla_roofline(units, ms_mla, pk, MLA_NCU_TRAFFIC_BYTES)
     line = {
         "metric": metric, "value": qps, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -490,18 +645,17 @@ def main():
         "gathered_tokens_per_s": whole_job_rate(world, units["gathered"], ms_step),
         "stage_ms": {"indexer": ms_idx, "topk": ms_topk, "sparse_mla_and_merge": ms_mla,
                      "step_with_stage_events": ms_staged},
-        "indexer_hbm_gbs": idx_gbs, "indexer_frac_of_8000_gbs": idx_gbs / 8000.0,
-        "mla_hbm_gbs": units["mla_bytes"] / (ms_mla / 1e3) / 1e9,
-        "mla_tflops": units["mla_flops"] / (ms_mla / 1e3) / 1e12,
-        "roofline": {"kernel": "indexer scores", "bound": "hbm", "achieved": idx_gbs, "peak": peak,
-                     "unit": "GB/s", "frac": idx_gbs / peak, "peak_source": peak_kind,
-                     "algorithmic_bytes_per_launch": units["indexer_bytes"],
-                     "traffic": INDEXER_NCU_TRAFFIC_BYTES},
-        "clocks": clocks,
+        "indexer_hbm_gbs": idx_rf["gbs"], "indexer_frac_of_8000_gbs": idx_rf["frac_of_8000_gbs"],
+        "roofline": {k: idx_rf[k] for k in ("kernel", "bound", "achieved", "peak", "unit", "frac", "peak_source",
+                                            "algorithmic_bytes_per_launch", "traffic")},
+        "mla_roofline": mla_rf,
+        "peaks": pk,
+        "clocks": clk,
         "e2e": {"value": whole_job_rate(world, wl.T, e2e_ms), "unit": "queries/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "entry_point": "sml_run_layer"},
         "gpu_launches": args.steps * 4,
         "cpu_baseline": cb,
+        "workloads": reports,
         "producers": producers,
         "latent_e4m3_576": {"sparse_mla_and_merge_ms": plain_ms,
                             "hbm_gbs": units["gathered"] * 576 / (plain_ms / 1e3) / 1e9,

@@ -78,6 +78,7 @@ class Layer:
     iq_scale: np.ndarray | None = None  # float32 [T]
     iw: np.ndarray | None = None        # float32 [T, 64]
     reuse_from: int | None = None
+    name: str = ""                      # the layer's tag in its workload ("rope", "nope", ...)
 
 
 @dataclass
@@ -250,6 +251,7 @@ def make_workload(name: str, ctx_len, q_count, num_heads: int, topk: int = 2048,
     T = int(cu_q[-1])
     for tag, rope_dim, with_idx, reuse in layers:
         wl.layers.append(make_layer(seed, name + "/" + tag, T, num_heads, rope_dim, with_idx, reuse))
+        wl.layers[-1].name = tag
     return wl
 
 
