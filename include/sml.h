@@ -15,7 +15,8 @@
  *                          the producers just before the step: FP8
  *                          quantisation of new tokens into the two caches,
  *                          and of the indexer queries
- *   sml_dcp_merge_candidates, sml_dcp_split_selection, sml_lse_combine
+ *   sml_dcp_pack_candidates, sml_dcp_merge_candidates,
+ *   sml_dcp_split_selection, sml_lse_combine
  *                          decode context parallelism: the steps between the
  *                          ranks' own top-k and sparse MLA
  *
@@ -51,8 +52,9 @@
  * [cu_q[r], cu_q[r+1]) (Q_r = cu_q[r+1] - cu_q[r] >= 1) and L_r = ctx_len[r]
  * cached tokens, its own query tokens included (L_r >= Q_r).  Query j (0-based)
  * of request r sees positions [0, n_t) with n_t = L_r - Q_r + j + 1 (causal
- * within the request).  Logical position s of request r lives in physical
- * page block_table[r * max_pages + s / 64], row s % 64.
+ * within the request), unless sml_problem.vis_len gives n_t.  Logical
+ * position s of request r lives in physical page
+ * block_table[r * max_pages + s / 64], row s % 64.
  */
 #ifndef SML_H_
 #define SML_H_
@@ -117,6 +119,15 @@ typedef struct sml_problem {
   const int32_t* cu_q;         /* [B + 1], cu_q[0] = 0, non-decreasing */
   const int32_t* ctx_len;      /* [B], L_r */
   const int32_t* block_table;  /* [B * max_pages], physical page ids */
+  /* Optional per-token overrides (NULL = the causal rule; a zero-initialised
+   * struct keeps it).  vis_len [T]: n_t itself, in [0, L_r] and
+   * non-decreasing within a request (n_t = 0: nothing visible; with it the
+   * only length rule on L_r is 0 <= L_r <= max_ctx).  ssmax_len [T]: the n of
+   * every SSMax factor s * ln(n), >= 1 (default n_t).  Decode context
+   * parallelism sets both: a rank sees its own share of each query's
+   * context, but every rank scales by the global length. */
+  const int32_t* vis_len;
+  const int32_t* ssmax_len;
 } sml_problem;
 
 /* Latent cache formats (sml_cache.format of a latent pool; an indexer pool
@@ -291,17 +302,19 @@ int sml_indexer_q_quant(const void* iq, int32_t num_tokens, void* iq8, float* iq
  * vLLM blog "vLLM 首日支持 Mistral Large 4", section "长上下文：解码和预填充的上下文
  * 并行", paragraph "DCP" and the list after it: the cache is sharded by token
  * over R ranks; every rank runs the indexer and top-k over its own tokens; the
- * candidates are exchanged as (score, id) pairs and merged with a stable
- * top-k; each rank attends over the selected tokens it holds; the partial
- * outputs are combined by their log-sum-exp.  Reading: token s of a request
- * lives on rank (s / I) % R at local position (s / (I R)) I + s % I for an
- * interleave I (I = 64 keeps a page on one rank, so a rank's shard is a local
- * block table over the same pool).  Every rank's problem is the batch with
- * its local lengths; the merge compares scores across ranks, so the layers
- * must run with ssmax = 0 (the SSMax factor would differ per rank).  One
- * query token per request.  The calls below are the steps between the ranks'
- * own sml_indexer_scores / sml_topk and their own sml_sparse_mla_decode; the
- * caller moves the arrays between GPUs. */
+ * candidates are exchanged as packed (score, id) pairs and merged with a
+ * stable top-k; each rank attends over the selected tokens it holds; the
+ * partial outputs are combined by their log-sum-exp.  Reading: token s of a
+ * request lives on rank (s / I) % R at local position (s / (I R)) I + s % I
+ * for an interleave I (I = 64 keeps a page on one rank, so a rank's shard is a
+ * local block table over the same pool).  A rank's problem is the batch with
+ * its local context lengths, sml_problem.vis_len = each query's local visible
+ * count (its tokens among the query's n_t) and sml_problem.ssmax_len = the
+ * global n_t, so that scores compare across ranks with SSMax on and any
+ * number of query tokens per request.  The calls below are the steps between
+ * the ranks' own sml_indexer_scores / sml_topk and their own
+ * sml_sparse_mla_decode; the caller moves the arrays between GPUs (the Python
+ * package's dcp module does it with torch.distributed). */
 #define SML_DCP_MAX_RANKS 8
 
 /* The ranks' top-k results (host struct; the pointers are device pointers). */
@@ -312,7 +325,18 @@ typedef struct sml_dcp_ranks {
   int64_t score_stride[SML_DCP_MAX_RANKS];       /* its row stride (that rank's max_ctx) */
   const int32_t* idx[SML_DCP_MAX_RANKS];         /* rank r's top-k [T, topk], local positions, ascending */
   const int32_t* idx_len[SML_DCP_MAX_RANKS];     /* [T] */
+  int32_t packed;  /* 1: scores[r] is [T, topk], entry i the score of candidate i (from
+                      sml_dcp_pack_candidates; score_stride ignored); 0: score matrices */
 } sml_dcp_ranks;
+
+/* Pack one rank's candidates for the exchange: cand_scores [T, topk] with
+ * entry i = scores[t, idx[t, i]] for i < idx_len[t], NaN past it (a NaN ranks
+ * below every score).  A position outside [0, score_stride) or a length
+ * outside [0, topk] gives NaN and sets SML_FAULT_INDEX / SML_FAULT_TOPK_LEN in
+ * workspace (NULL or >= 256 B). */
+int sml_dcp_pack_candidates(int32_t num_tokens, int32_t topk, const float* scores, int64_t score_stride,
+                            const int32_t* idx, const int32_t* idx_len, float* cand_scores, void* workspace,
+                            void* stream);
 
 /* Merge: for query t, every rank's candidates (score, global position) in
  * ascending global position: merged_scores / merged_pos [T, R * topk] (row

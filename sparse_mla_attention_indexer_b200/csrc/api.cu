@@ -117,9 +117,7 @@ Layout layout(const sml_problem& p, int stage) {
     off += align_up((size_t)p.num_tokens * ch * sizeof(int32_t));
   }
   const size_t end_topk = off;
-  int kps;
-  const int S = mla_splits(p, &kps);
-  const size_t slots = (size_t)p.num_tokens * p.num_heads * S;
+  const size_t slots = mla_slots(mla_plan(p), p.num_tokens) * 16;   // 16 heads per slot
   L.part_out = off;
   off += align_up(slots * SML_LATENT_DIM * sizeof(float));
   L.part_lse = off;
@@ -168,7 +166,7 @@ TopkWs topk_ws(const sml_problem& p, const Layout& L, void* ws) {
 MlaWs mla_ws(const sml_problem& p, const Layout& L, void* ws) {
   char* b = static_cast<char*>(ws);
   MlaWs m;
-  m.splits = mla_splits(p, &m.keys_per_split);
+  m.plan = mla_plan(p);
   m.part_out = reinterpret_cast<float*>(b + L.part_out);
   m.part_lse = reinterpret_cast<float*>(b + L.part_lse);
   return m;
@@ -408,10 +406,12 @@ int sml_dcp_merge_candidates(const sml_dcp_ranks* ranks, int32_t num_tokens, int
             "num_ranks not in [1, SML_DCP_MAX_RANKS]");
     c.check(ranks->interleave >= 1, SML_ERR_INVALID_ARG, "interleave < 1");
     const int R = ranks->num_ranks >= 1 && ranks->num_ranks <= SML_DCP_MAX_RANKS ? ranks->num_ranks : 0;
+    c.check(ranks->packed == 0 || ranks->packed == 1, SML_ERR_INVALID_ARG, "ranks->packed not 0 or 1");
     for (int r = 0; r < R && num_tokens > 0; ++r) {
       c.check(ranks->scores[r] != nullptr, SML_ERR_INVALID_ARG, "ranks->scores[r] is NULL");
       c.check(ranks->idx[r] != nullptr, SML_ERR_INVALID_ARG, "ranks->idx[r] is NULL");
       c.check(ranks->idx_len[r] != nullptr, SML_ERR_INVALID_ARG, "ranks->idx_len[r] is NULL");
+      if (ranks->packed) continue;   // positions past int32 are reported by the kernel
       c.check(ranks->score_stride[r] >= 1 && ranks->score_stride[r] <= (1 << 30), SML_ERR_INVALID_ARG,
               "ranks->score_stride[r] not in [1, 2^30]");
       c.check(ranks->score_stride[r] * (int64_t)R <= INT32_MAX, SML_ERR_UNSUPPORTED,
@@ -426,6 +426,23 @@ int sml_dcp_merge_candidates(const sml_dcp_ranks* ranks, int32_t num_tokens, int
   cudaError_t e = launch_dcp_merge(*ranks, num_tokens, topk, merged_scores, merged_pos, merged_len,
                                    workspace ? status_of(workspace) : nullptr, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SML_OK : cuda_fail(e, "sml_dcp_merge_candidates");
+}
+
+int sml_dcp_pack_candidates(int32_t num_tokens, int32_t topk, const float* scores, int64_t score_stride,
+                            const int32_t* idx, const int32_t* idx_len, float* cand_scores, void* workspace,
+                            void* stream) {
+  Checker c;
+  c.check(num_tokens >= 0, SML_ERR_INVALID_ARG, "num_tokens < 0");
+  c.check(topk >= 1 && topk <= SML_MAX_TOPK, SML_ERR_UNSUPPORTED, "topk not in [1, 2048]");
+  c.check(score_stride >= 1 && score_stride <= (1 << 30), SML_ERR_INVALID_ARG, "score_stride not in [1, 2^30]");
+  c.check(workspace == nullptr || aligned(workspace, 256), SML_ERR_WORKSPACE, "workspace not 256-B aligned");
+  const bool any = num_tokens > 0;
+  c.check(!any || (scores && idx && idx_len && cand_scores), SML_ERR_INVALID_ARG,
+          "scores, idx, idx_len or cand_scores is NULL");
+  if (c.done("sml_dcp_pack_candidates") != SML_OK) return c.code;
+  cudaError_t e = launch_dcp_pack(num_tokens, topk, scores, score_stride, idx, idx_len, cand_scores,
+                                  workspace ? status_of(workspace) : nullptr, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SML_OK : cuda_fail(e, "sml_dcp_pack_candidates");
 }
 
 int sml_dcp_split_selection(int32_t num_ranks, int32_t interleave, int32_t num_tokens, int32_t topk,

@@ -25,6 +25,7 @@ struct RankArrays {
   const int32_t* idx[SML_DCP_MAX_RANKS];
   const int32_t* len[SML_DCP_MAX_RANKS];
   int64_t stride[SML_DCP_MAX_RANKS];
+  int packed;   // scores[r] is [T, K], aligned with idx[r]
 };
 
 struct RankOut {
@@ -83,16 +84,17 @@ dcp_merge_kernel(RankArrays ra, int R, int I, int K, float* __restrict__ mscore,
     const int32_t* list = ra.idx[r] + (size_t)t * K;
     for (int i = threadIdx.x; i < n[r]; i += kMergeThreads) {
       const int l = __ldg(list + i);
-      if (l < 0 || l >= ra.stride[r]) {
+      const long long g = l >= 0 ? global_pos(l, r, R, I) : -1;
+      if (l < 0 || (!ra.packed && l >= ra.stride[r]) || g > INT32_MAX) {
         raise_fault(status, SML_FAULT_INDEX);
         continue;
       }
-      const long long g = global_pos(l, r, R, I);
       int m = i;
       for (int r2 = 0; r2 < R; ++r2)
         if (r2 != r) m += count_below(ra.idx[r2] + (size_t)t * K, n[r2], g, r2, R, I);
       if (m < total) {
-        mscore[row + m] = __ldg(ra.scores[r] + (size_t)t * ra.stride[r] + l);
+        mscore[row + m] = ra.packed ? __ldg(ra.scores[r] + (size_t)t * K + i)
+                                    : __ldg(ra.scores[r] + (size_t)t * ra.stride[r] + l);
         mpos[row + m] = (int32_t)g;
       }
     }
@@ -138,6 +140,30 @@ dcp_split_kernel(int R, int I, int K, const int32_t* __restrict__ sel, const int
   for (int r = 0; r < R; ++r) {
     for (int i = cnt[r] + lane; i < K; i += 32) out.idx[r][(size_t)t * K + i] = -1;
     if (lane == 0) out.len[r][t] = cnt[r];
+  }
+}
+
+// cand[t, i] = scores[t, idx[t, i]] for i < len[t], NaN past it and for a
+// position outside the row.
+__global__ void __launch_bounds__(256)
+dcp_pack_kernel(int K, const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ idx,
+                const int32_t* __restrict__ len, float* __restrict__ cand, int32_t* status) {
+  ptx::griddep_wait();
+  if (threadIdx.x == 0) ptx::griddep_launch_dependents();
+  const int t = blockIdx.x;
+  int n = __ldg(len + t);
+  if (n < 0 || n > K) {
+    if (threadIdx.x == 0) raise_fault(status, SML_FAULT_TOPK_LEN);
+    n = max(0, min(n, K));
+  }
+  for (int i = threadIdx.x; i < K; i += blockDim.x) {
+    float v = __int_as_float(0x7fc00000);
+    if (i < n) {
+      const int l = __ldg(idx + (size_t)t * K + i);
+      if (l >= 0 && l < stride) v = __ldg(scores + (size_t)t * stride + l);
+      else raise_fault(status, SML_FAULT_INDEX);
+    }
+    cand[(size_t)t * K + i] = v;
   }
 }
 
@@ -192,8 +218,15 @@ cudaError_t launch_dcp_merge(const sml_dcp_ranks& rk, int T, int K, float* mscor
     ra.len[r] = rk.idx_len[r];
     ra.stride[r] = rk.score_stride[r];
   }
+  ra.packed = rk.packed;
   return launch_pdl(dcp_merge_kernel, dim3(T), dim3(kMergeThreads), 0, stream, 0, ra, rk.num_ranks, rk.interleave, K,
                     mscore, mpos, mlen, status);
+}
+
+cudaError_t launch_dcp_pack(int T, int K, const float* scores, int64_t stride, const int32_t* idx,
+                            const int32_t* len, float* cand, int32_t* status, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  return launch_pdl(dcp_pack_kernel, dim3(T), dim3(256), 0, stream, 0, K, scores, stride, idx, len, cand, status);
 }
 
 cudaError_t launch_dcp_split(int R, int I, int T, int K, const int32_t* sel, const int32_t* sel_len,

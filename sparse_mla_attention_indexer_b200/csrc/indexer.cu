@@ -67,6 +67,7 @@ struct __align__(1024) Smem {
   float ksc[kStages][kTile];
   float w[kEpiGroups][kGroup * SML_INDEX_HEADS]; // per epilogue warpgroup: head weights of the group
   float qf[kEpiGroups][kGroup];                  // per epilogue warpgroup: sq_t * c_t per query
+  int nv[kEpiGroups][kGroup];                    // per epilogue warpgroup: n_t per query
   uint64_t full[kStages], empty[kStages];
   uint64_t qfull[2], qempty[2];
   uint64_t accfull[C::kAccBufs], accempty[C::kAccBufs];
@@ -84,6 +85,8 @@ struct Params {
   const int32_t* cu_q;
   const int32_t* ctx_len;
   const int32_t* block_table;
+  const int32_t* vis_len;     // optional n_t per token (non-decreasing within a request)
+  const int32_t* ssmax_len;   // optional SSMax n per token
   const float* iq_scale;
   const float* iw;
   const uint8_t* index_base;
@@ -100,12 +103,13 @@ struct Walker {
   Req rq;
 
   __device__ void load_req() {
-    rq = load_request(P->cu_q, P->ctx_len, r, P->T, P->max_ctx, P->max_pages);
+    rq = load_request(P->cu_q, P->ctx_len, r, P->T, P->max_ctx, P->max_pages, P->vis_len != nullptr);
     ngroups = rq.ok ? (rq.Q + kGroup - 1) / kGroup : 0;
   }
   __device__ int group_tiles() const {
     const int last = min(rq.Q, kGroup * g + kGroup);   // the group's queries: [4g, last)
-    const int n_last = rq.L - rq.Q + last;             // visible length of its last query
+    bool bad = false;                                  // (reported by the epilogue)
+    const int n_last = visible_len(P->vis_len, rq, rq.q0 + last - 1, &bad);   // the largest of the group's
     return (n_last + kTile - 1) / kTile;
   }
   __device__ int qg() const { return min(kGroup, rq.Q - kGroup * g); }
@@ -419,6 +423,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     const int et = threadIdx.x - 64 - 128 * eg; // 0..127 within the warpgroup
     float* wsm = S.w[eg];
     float* qfs = S.qf[eg];
+    int* nvs = S.nv[eg];
     Walker<kGroup> w{&P};
     if (beg < end) w.start(S.sched[2], S.sched[3]);
     int last_r = -1, last_g = -1;
@@ -435,9 +440,13 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         for (int i = et; i < qg * SML_INDEX_HEADS; i += 128)
           wsm[i] = __ldg(P.iw + (size_t)(w.rq.q0 + j0) * SML_INDEX_HEADS + i);
         if (et < qg) {
-          const int n = w.rq.L - w.rq.Q + j0 + et + 1;
-          const float c = P.ssmax ? P.s_index * logf((float)n) : 1.f;
-          qfs[et] = __ldg(P.iq_scale + w.rq.q0 + j0 + et) * c;
+          const int t = w.rq.q0 + j0 + et;
+          bool bad = false;
+          const int n = visible_len(P.vis_len, w.rq, t, &bad);
+          if (bad) raise_fault(P.status, SML_FAULT_LENGTHS);
+          const float c = P.ssmax ? P.s_index * logf((float)ssmax_len_of(P.ssmax_len, t, n)) : 1.f;
+          qfs[et] = __ldg(P.iq_scale + t) * c;
+          nvs[et] = n;
         }
         if (eg == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
         else asm volatile("bar.sync 2, 128;" ::: "memory");
@@ -463,8 +472,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
           s0 = fmaf(wj[i], fmaxf(__uint_as_float(v0[i]), 0.f), s0);
           s1 = fmaf(wj[32 + i], fmaxf(__uint_as_float(v1[i]), 0.f), s1);
         }
-        const int n = w.rq.L - w.rq.Q + j0 + j + 1;
-        if (row_ok && s < n) P.scores[(size_t)(w.rq.q0 + j0 + j) * P.max_ctx + s] = (s0 + s1) * qfs[j] * sk;
+        if (row_ok && s < nvs[j]) P.scores[(size_t)(w.rq.q0 + j0 + j) * P.max_ctx + s] = (s0 + s1) * qfs[j] * sk;
       }
       ptx::tc_fence_before();
       __syncwarp();
@@ -576,6 +584,8 @@ cudaError_t launch_indexer(const sml_problem& p, const uint8_t* iq8, const float
   P.cu_q = p.cu_q;
   P.ctx_len = p.ctx_len;
   P.block_table = p.block_table;
+  P.vis_len = p.vis_len;
+  P.ssmax_len = p.ssmax_len;
   P.iq_scale = iq_scale;
   P.iw = iw;
   P.index_base = index_base;

@@ -1,41 +1,55 @@
-// Absorbed-query sparse MLA over a paged fp8_ds_mla latent cache on the sm_100a
-// tensor cores, split over the selected keys, then a log-sum-exp merge.
+// Absorbed-query sparse MLA over a paged fp8_ds_mla (or plain E4M3) latent
+// cache on the sm_100a tensor cores, split over the selected keys, then a
+// log-sum-exp merge.
 //
 // vLLM blog "vLLM 首日支持 Mistral Large 4": highlights list (MLA, KV LoRA
 // rank 512, RoPE dim 64, top-2048 keys per query); section "实现细节 / 模型架构"
 // (sparse MLA over the fp8_ds_mla latent cache; NoPE = RoPE dim 0 on the same
 // cache; SSMax on the MLA query); section "长上下文" (partial results merged by
-// their LSE).  For token t, head h over the selected set S_t:
+// their LSE); section "ROCm 实现细节", paragraph "FP8 潜在缓存" (the plain
+// per-tensor E4M3 cache, 576 B per token).  For token t, head h over the
+// selected set S_t:
 //   z_i = sm_scale * c_t * (q_nope . c_hat_i + q_pe . k_pe_i)
 //   out = sum_i softmax(z)_i c_hat_i,   lse = ln sum_i exp(z_i)
 // with c_hat_i = e4m3 latent x its 128-element block scale.
 //
-// One CTA = (query token, group of 16 heads, split of up to 512 selected keys),
-// in tiles of 128 keys; keys are the MMA M dimension of QK^T and its K
-// dimension of PV, the 16 heads N (an MMA costs at least ~45 cycles whatever
-// its N, and 16 heads as M would waste 3/4 of the smallest M).  Both products
-// run on kind::f8f6f4 straight from the gathered E4M3 latent tile: nothing of
-// the latent is ever converted.
-//   * warps 4-14 gather the selected 656-B rows, eight rows per warp batch
-//     (16-B register loads, one row per warp instruction), into
-//     128-B-swizzled tiles: E4M3 latent, bf16 RoPE key, block scales aside;
-//     two tile buffers.  Random rows need many loads in flight per SM, hence
-//     many gather warps and deep batches;
-//   * warp 15 issues the MMAs:
-//       S_b^T = C_b . [Qhi_b; Qlo_b]^T  (K-major; N = 32: both query terms),
-//       S_pe^T = K_pe . Q_pe^T          (kind::f16, bf16),
+// Work: a unit is (query token, group of 16 heads, tile of 128 selected keys).
+// One persistent CTA per SM takes an equal contiguous range of the units
+// (token-major), so every SM holds the same number of tiles whatever the
+// batch; where its range crosses a (token, head group) boundary it writes one
+// partial result per (token, head group), and a merge kernel combines the
+// partials by their LSE.  Keys are the MMA M dimension of QK^T and the K
+// dimension of PV, the 16 heads N (16 heads as M would waste 3/4 of the
+// smallest M); both products run on kind::f8f6f4 straight from the gathered
+// E4M3 tile: the latent is never converted.
+//   * warps 9-23 fill the two tile buffers: they turn the tile's selected
+//     positions into pool rows (block table, bounds checks), then copy the
+//     rows with 16-B cp.async straight into place, 128-B-swizzled, a masked
+//     row as zeros; the copies arrive on the buffer's barrier by themselves,
+//     so the loaders go on to the next tile at once.  (Random 656-B rows are
+//     bound by the requests in flight per SM: measured on B200, cp.async
+//     from many warps reaches about 20 GB/s per SM whatever the shared-memory
+//     size, while register loads lose a quarter of that rate when the
+//     kernel's shared memory leaves L1 small, and TMA tile::gather4 reaches
+//     about half of it.);
+//   * warp 8 issues the MMAs (one thread):
+//       S_b^T = C_b . [Qhi_b; Qlo_b]^T   (K-major; N = 32: both query terms),
+//       S_pe^T = K_pe . Q_pe^T           (bf16; plain E4M3: both terms),
 //       O_b^T += C_b^T . [Bhi_b; Bmid_b; Blo_b]^T  (C_b^T read MN-major from
-//       the same tile; N = 48: the three weight terms);
-//     the next tile's QK^T goes in ahead of this tile's PV, as soon as its
-//     rows have landed and the softmax has read S;
-//   * warps 0-3 (one thread per key) run the softmax on S^T and build the
-//     weights B_b[i, h] = p_ih scale_ib / sigma_h as three E4M3 terms whose
-//     sum carries 12 significant bits (finer than fp16); sigma_h is a per-head
+//       the same tile; N = 48: the three weight terms),
+//     each as soon as its inputs are ready: a tile's PV (which frees its
+//     buffer) does not wait for the next tile's QK^T, nor the reverse;
+//   * warps 0-7 (two per TMEM lane quarter: keys 32q..32q+31, heads 8 hh..
+//     8 hh + 7) stage each (token, head group)'s query, run the softmax on
+//     S^T and build the weights B_b[i, h] = p_ih scale_ib / sigma_h as three
+//     E4M3 terms whose sum carries 12 significant bits; sigma_h is a per-head
 //     power of two that keeps the terms in range, raised (and O rescaled,
-//     exactly) only when a tile would overflow; at the end they read O^T back
-//     (one thread per latent dim) and write the split's output and LSE.
+//     exactly) only when a tile would overflow; at the end of a (token, head
+//     group) they read O^T back and write its partial output and LSE.
 // The query is split exactly into two E4M3 terms sharing a power-of-two scale
 // per head; products of E4M3 values are exact and accumulate in fp32.
+// Every wait is bounded; a wait that gives up sets SML_FAULT_TIMEOUT and the
+// CTA winds down (no trap).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -47,44 +61,47 @@
 namespace sml {
 namespace {
 
-constexpr int kHC = 16;          // heads per CTA
+constexpr int kHC = 16;          // heads per unit
 constexpr int kKT = 128;         // keys per tile
-constexpr int kMaxSplit = 512;   // keys per split (4 tiles)
-constexpr int kThreads = 512;    // warps 0-3 softmax, 4-14 gather, 15 MMA
-constexpr int kGatherWarps = 11;
-constexpr int kBatchRows = 8;                     // rows per gather batch (16 loads in flight per thread)
-constexpr int kBatchesPerTile = 128 / kBatchRows;  // >= kGatherWarps: every gather warp has a batch in every tile
-static_assert(kBatchesPerTile >= kGatherWarps, "a gather warp without a batch in a tile would never signal it");
-constexpr int kWarpMma = 15;
-constexpr float kLazyRescale = 8.f;   // nats
+constexpr int kSoftmaxThreads = 256;   // warps 0-7
+constexpr int kWarpMma = 8;
+constexpr int kWarpLoad = 9;           // warps 9-23 copy the rows
+constexpr int kLoadWarps = 15;
+constexpr int kLoadThreads = 32 * kLoadWarps;
+constexpr int kThreads = 32 * (kWarpLoad + kLoadWarps);   // 768: six warpgroups
+// Registers: the kernel launches with kRegsLaunch per thread; the two softmax
+// warpgroups then raise theirs to kRegsSoftmax and the other four (MMA and
+// loaders) lower theirs to kRegsOther.  setmaxnreg.inc draws on what the
+// block launched with, so the shares must add up to it exactly.
+constexpr int kRegsLaunch = 80, kRegsSoftmax = 112, kRegsOther = 64;
+static_assert(kThreads * kRegsLaunch == 256 * kRegsSoftmax + (kThreads - 256) * kRegsOther,
+              "warpgroup register shares must add up to the launch allocation");
+static_assert(kThreads % 128 == 0 && kWarpMma == 8, "roles are whole warpgroups: 0-1 softmax, 2-5 the rest");
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLazyRescale = 8.f * kLog2e;   // 8 nats, in the log2 units the softmax runs in
 
 // TMEM columns
 constexpr uint32_t kColS = 0;       // S_b^T (lanes = keys): 32 columns per block b (hi | lo query term)
-constexpr uint32_t kColSpe = 128;   // S_pe^T
+constexpr uint32_t kColSpe = 128;   // S_pe^T: 16 columns (bf16), or 32 (plain E4M3: hi | lo)
 constexpr uint32_t kColO = 256;     // O_b^T (lanes = dims of block b): 48 columns (hi | mid | lo) ...
 constexpr uint32_t kOStride = 64;   // ... at kColO + kOStride b
 constexpr int kPBytes = kKT * 3 * kHC;   // one block's weight terms: 128 keys x 48 E4M3
+constexpr int kLatBlock = kKT * 128;     // one 128-dim latent block of a tile
 
 struct __align__(1024) Smem {
-  uint8_t lat[2][4][kKT * 128];  // [buffer][block b][128 keys x 128 B] E4M3, SW128
-  uint8_t pe[2][kKT * 128];      // [buffer][128 keys x 64 bf16], SW128
+  uint8_t lat[2][4][kLatBlock];  // [buffer][block b][128 keys x 128 B] E4M3, SW128
+  uint8_t pe[2][kKT * 128];      // [buffer][128 keys x 128 B] RoPE key (64 bf16, or 64 E4M3 + 64 zeros), SW128
   uint8_t q8[4][2 * kHC * 128];  // [block] 32 rows x 128 B, SW128: rows 0-15 high term, 16-31 low term
-  uint8_t qpe[kHC * 128];        // query RoPE bf16 [16 heads x 64], SW128
+  uint8_t qpe[2 * kHC * 128];    // RoPE query, SW128: bf16 rows 0-15; plain E4M3: rows 0-15 high, 16-31 low
   uint8_t pb[4][kPBytes];        // weight terms of block b, MN-major 8-key x 16-B core matrices
-  float xch[kKT * kHC];          // softmax column-reduction exchange
-  float sc[2][kKT][4];           // [buffer][key][block] scales of the staged tile
+  float sc[2][kKT][4];            // [buffer][key] the four block scales of the staged row
+  float xmax[2][2][4][12];       // [tile parity][head half][key quarter]: 8 head maxima, largest scale
+  float xsum[2][4][8];           // [head half][key quarter][head]: row-sum exchange
   float qs[kHC];                 // power-of-two query scale per head
-  float hstat[kHC];              // per-head row sum (epilogue)
-  float hm[kHC];                 // per-head running max m_h
-  float hsig[kHC];               // per-head weight scale sigma_h (a power of two; 0 = not set yet)
-  float halpha[kHC];             // this tile's exp(m_old - m_new)
-  float hf[kHC];                 // this tile's rescale factor of O
-  float hinv[kHC];               // 1 / sigma_h (0 while unset)
-  float hosc[kHC];               // epilogue: sigma_h / l_h, the output scale of head h
-  float scw[2][4];               // per-warp max of the tile's scales (double-buffered by tile)
-  int32_t rowid[kMaxSplit];      // pool row (page * 64 + row) of each key, -1 = masked
-  uint64_t e_full[2], e_free[2];
-  uint64_t q_ready, s_full, s_free, p_full, pv_done, drain;
+  int32_t rowid[4][kKT];         // [tile % 4] pool row of each key, -1 = masked
+  uint64_t full[2], lat_free[2];
+  uint64_t q_ready, s_full, s_free, p_full, pv_done, o_free, drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -95,6 +112,8 @@ struct Params {
   const int32_t* cu_q;
   const int32_t* ctx_len;
   const int32_t* block_table;
+  const int32_t* vis_len;     // optional n_t per token
+  const int32_t* ssmax_len;   // optional SSMax n per token
   const uint16_t* q;
   const uint8_t* latent;
   int64_t latent_pages;
@@ -110,17 +129,14 @@ __device__ __forceinline__ uint32_t sw128(uint32_t base, int row, int chunk) {
   return base + (row >> 3) * 1024 + (row & 7) * 128 + ((chunk ^ (row & 7)) << 4);
 }
 
-// 16-B global load that does not allocate in L1 (each row is read once).
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+__device__ __forceinline__ void st_shared_v2(uint32_t addr, uint32_t a, uint32_t b) {
+  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
+}
+__device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t a) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
 }
 
 // Round two floats to E4M3 (nearest even, saturating); the codes, low byte = a.
@@ -133,11 +149,6 @@ __device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t two) {
   return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
-// Two floats that are bf16 values -> their bf16 bits, low half = a.
-__device__ __forceinline__ uint32_t bf16x2_bits(float a, float b) {
-  return (__float_as_uint(a) >> 16) | (__float_as_uint(b) & 0xffff0000u);
-}
-
 // x (two values) -> E4M3 codes of the nearest value and the exact residual.
 __device__ __forceinline__ uint32_t split_e4m3x2(float& x0, float& x1) {
   const uint32_t c = f2_to_e4m3x2(x0, x1);
@@ -147,157 +158,246 @@ __device__ __forceinline__ uint32_t split_e4m3x2(float& x0, float& x1) {
   return c;
 }
 
+// x rounded to 4 significant bits, nearest even, by integer arithmetic on
+// its fp32 bits: the E4M3 value nearest to x wherever x is in E4M3's normal
+// range (|x| in [2^-6, 448]).  Below 2^-6 the result is finer than E4M3's
+// subnormal step 2^-9, and the code the conversion then picks is within
+// 2^-10 of it.
+__device__ __forceinline__ float round_e4m3_normal(float x) {
+  const uint32_t b = __float_as_uint(x);
+  return __uint_as_float((b + 0x7ffffu + ((b >> 20) & 1u)) & 0xfff00000u);
+}
+
+// Three E4M3 terms of two weights (each at most 448), low byte = first
+// weight: x = hi + mid + lo to 12 significant bits; the residuals are exact
+// in fp32.
+__device__ __forceinline__ void split3_e4m3x2(float x0, float x1, uint32_t& hi, uint32_t& mid, uint32_t& lo) {
+  const float h0 = round_e4m3_normal(x0), h1 = round_e4m3_normal(x1);
+  const float r0 = x0 - h0, r1 = x1 - h1;
+  const float m0 = round_e4m3_normal(r0), m1 = round_e4m3_normal(r1);
+  hi = f2_to_e4m3x2(h0, h1);
+  mid = f2_to_e4m3x2(m0, m1);
+  lo = f2_to_e4m3x2(r0 - m0, r1 - m1);
+}
+
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort) {
   const bool ok = ptx::mbar_wait(bar, parity, abort);
   return __all_sync(0xffffffffu, ok);
 }
 
-// AND of a flag over the four softmax warps (named barrier 1): every wait
-// outcome is made uniform across them before the next named barrier, so a
-// timed-out wait ends all four together instead of leaving three behind.
+// AND of a flag over the 256 softmax threads (named barrier 3).  Every wait
+// outcome reaches this before the next named barrier of the softmax warps, so
+// a wait that gave up ends all eight warps together instead of leaving some
+// blocked at a barrier.
 __device__ __forceinline__ bool softmax_all(bool ok) {
   uint32_t r;
   asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}"
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 3, 256, p;\n selp.u32 %0, 1, 0, q;\n}"
       : "=r"(r)
       : "r"((uint32_t)ok)
       : "memory");
   return r != 0;
 }
 
-// Softmax exchange buffer: [128 keys][16] floats, columns XOR-swizzled by key.
-__device__ __forceinline__ float* xbuf(Smem& S, int key, int col) {
-  return S.xch + key * kHC + (col ^ (key & 15));
-}
-
-// Sum (or max) over the 128 keys of 16 per-key values (warps 0-3); every
-// softmax thread reads the 16 results from S.hstat afterwards.  Shared writes
-// made before the call are visible to all four warps after it.
-template <bool kMax>
-__device__ __forceinline__ void column_reduce(Smem& S, int row, const float (&v)[kHC]) {
-#pragma unroll
-  for (int h = 0; h < kHC; ++h) *xbuf(S, row, h) = v[h];
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-  const int hh = row >> 3, part = row & 7;   // head hh, keys part + 8 j
-  float acc = kMax ? -INFINITY : 0.f;
-#pragma unroll
-  for (int j = 0; j < kKT / 8; ++j) {
-    const float x = *xbuf(S, part + 8 * j, hh);
-    acc = kMax ? fmaxf(acc, x) : acc + x;
-  }
-#pragma unroll
-  for (int o = 1; o < 8; o <<= 1) {
-    const float y = __shfl_xor_sync(0xffffffffu, acc, o);
-    acc = kMax ? fmaxf(acc, y) : acc + y;
-  }
-  if (part == 0) S.hstat[hh] = acc;
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-}
-
-// Per-tile softmax statistics (warps 0-3).  Max over the 128 keys of z; then
-// the thread owning head h updates, for that head, the lazily raised running
-// max m_h and the weight scale sigma_h: the tile's weights are at most
-// exp(tmax_h - m_h) * SC (SC = largest block scale in the tile) and must stay
-// <= 448 sigma_h; sigma_h is reset to the next power of two >= U_h / 448
-// (U_h below) whenever U_h leaves [28, 448] sigma_h.  O holds
-// sum(weights / sigma), so both changes rescale it by
-// f_h = exp(m_old - m_new) * sigma_old / sigma_new (exact for the sigma
-// part).  Returns whether any f_h != 1.
-__device__ __forceinline__ bool tile_stats(Smem& S, int row, const float (&z)[kHC], int tile) {
-#pragma unroll
-  for (int h = 0; h < kHC; ++h) *xbuf(S, row, h) = z[h];
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-  const int hh = row >> 3, part = row & 7;
-  float tm = -INFINITY;
-#pragma unroll
-  for (int j = 0; j < kKT / 8; ++j) tm = fmaxf(tm, *xbuf(S, part + 8 * j, hh));
-#pragma unroll
-  for (int o = 1; o < 8; o <<= 1) tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, o));
-  uint32_t changed = 0;
-  if (part == 0) {
-    const float* w = S.scw[tile & 1];
-    const float SC = fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3]));
-    float m = S.hm[hh], sig = S.hsig[hh];
-    float alpha = 1.f;
-    if (tm > m + kLazyRescale || (m == -INFINITY && tm != -INFINITY)) {
-      alpha = m == -INFINITY ? 0.f : expf(m - tm);
-      m = tm;
-    }
-    // Weights that matter are ~SC (p ~ 1 against the running max) or, in a
-    // tile above the running max, up to exp(tmax - m) SC; sigma keeps the
-    // largest of them within [28, 448] sigma, so the dominant weights keep all
-    // 12 bits of the three-term split, and moves only when they leave it.
-    const float U = tm == -INFINITY ? 0.f : fmaxf(expf(tm - m), 1.f) * SC;
-    float beta = 1.f;
-    if (U > 0.f && (U > 448.f * sig || U < 28.f * sig)) {
-      int e = 0;
-      frexpf(U * (1.f / 448.f), &e);   // U / 448 < 2^e
-      const float ns = ldexpf(1.f, e);
-      beta = sig > 0.f ? sig / ns : 1.f;
-      sig = ns;
-    }
-    S.hm[hh] = m;
-    S.hsig[hh] = sig;
-    S.halpha[hh] = alpha;
-    S.hf[hh] = alpha * beta;
-    S.hinv[hh] = sig > 0.f ? 1.f / sig : 0.f;
-    changed = alpha * beta != 1.f;
-  }
-  uint32_t any;
+// AND of a flag over the loader threads (named barrier 4); also orders their
+// shared-memory writes before it against reads after it.
+__device__ __forceinline__ bool loader_all(bool ok) {
+  uint32_t r;
   asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}"
-      : "=r"(any)
-      : "r"(changed)
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 4, %2, p;\n selp.u32 %0, 1, 0, q;\n}"
+      : "=r"(r)
+      : "r"((uint32_t)ok), "n"(kLoadThreads)
       : "memory");
-  return any != 0;
+  return r != 0;
+}
+
+// 2^x (the hardware approximation; relative error about 2^-22).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// The four warps of one head half (named barrier 1 + half).
+__device__ __forceinline__ void half_sync(int half) {
+  if (half == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
+  else asm volatile("bar.sync 2, 128;" ::: "memory");
+}
+
+__device__ __forceinline__ long long unit_begin(const MlaPlan& m, int c) { return m.units * c / m.ctas; }
+// The CTA whose range holds unit u.
+__device__ __forceinline__ int cta_of(const MlaPlan& m, long long u) {
+  return (int)(((u + 1) * m.ctas - 1) / m.units);
+}
+
+// One (token, head group) of a CTA's range: tiles [j0, j0 + nj) of it, of
+// which the first ne hold selected keys (tile j holds keys [128 j, 128 j +
+// 128) of the token's selection, len of them valid).
+struct Seg {
+  int tg, t, g, j0, nj, ne;
+  int r, n, len, nss;   // request, visible length, selected count, SSMax n
+  bool req_ok, len_bad;
+  size_t slot;
+};
+
+// Warp-collective (the request lookup is a 32-way search).
+__device__ Seg segment_at(const Params& P, long long u, long long e) {
+  const MlaPlan& m = P.ws.plan;
+  Seg s;
+  s.tg = (int)(u / m.tpt);
+  s.j0 = (int)(u % m.tpt);
+  const long long seg_end = min(e, (long long)(s.tg + 1) * m.tpt);
+  s.nj = (int)(seg_end - u);
+  s.t = s.tg / m.hg;
+  s.g = s.tg % m.hg;
+  s.r = request_of_warp(P.cu_q, P.B, s.t);
+  const Req rq = load_request(P.cu_q, P.ctx_len, s.r, P.T, P.max_ctx, P.max_pages, P.vis_len != nullptr);
+  s.req_ok = rq.ok && s.t >= rq.q0 && s.t - rq.q0 < rq.Q;
+  bool bad_n = false;
+  s.n = s.req_ok ? visible_len(P.vis_len, rq, s.t, &bad_n) : 0;
+  s.req_ok = s.req_ok && !bad_n;
+  s.nss = ssmax_len_of(P.ssmax_len, s.t, s.n);
+  const int len = s.req_ok ? __ldg(P.idx_len + s.t) : 0;
+  const int len_max = min(P.K, s.n);
+  s.len_bad = len < 0 || len > len_max;
+  s.len = max(0, min(len, len_max));
+  const int tiles = (s.len + kKT - 1) / kKT;
+  s.ne = max(0, min(s.nj, tiles - s.j0));
+  s.slot = (size_t)s.tg * m.smax + (blockIdx.x - cta_of(m, (long long)s.tg * m.tpt));
+  return s;
+}
+
+// A cursor over the non-empty tiles of a CTA's range, in order: tile jj of
+// segment s (the seg-th non-empty (token, head group) of the range), the
+// k-th tile overall.  Warp-collective, like segment_at.
+struct Cur {
+  long long u;   // the unit after segment s
+  Seg s;
+  int jj, seg, k;
+  bool valid;
+};
+
+__device__ __forceinline__ void cur_seek(Cur& c, const Params& P, long long ue) {
+  while (c.u < ue) {
+    c.s = segment_at(P, c.u, ue);
+    c.u += c.s.nj;
+    if (c.s.ne > 0) {
+      c.jj = 0;
+      c.valid = true;
+      return;
+    }
+  }
+  c.valid = false;
+}
+
+__device__ __forceinline__ void cur_start(Cur& c, const Params& P, long long ub, long long ue) {
+  c.u = ub;
+  c.seg = 0;
+  c.k = 0;
+  cur_seek(c, P, ue);
+}
+
+__device__ __forceinline__ void cur_next(Cur& c, const Params& P, long long ue) {
+  ++c.k;
+  if (++c.jj < c.s.ne) return;
+  ++c.seg;
+  cur_seek(c, P, ue);
+}
+
+// Stage the query of (token t, head group g) for QK^T (the 256 softmax
+// threads; thread = head h, part p of 16).  Nope part: q = s_h (hi + lo), hi
+// and lo E4M3 and s_h a power of two >= amax_h / 448, so q / s_h, its
+// rounding to hi and the residual lo are exact in fp32, and lo is exact in
+// E4M3 (a bf16 has 8 significant bits, hi takes 4, the residual the other 4)
+// down to E4M3's subnormal step.  RoPE part: copied as bf16; for a plain E4M3
+// pool split the same way (its products are E4M3 x E4M3).
+template <bool kPlain>
+__device__ __forceinline__ void stage_query(const Params& P, Smem& S, int t, int g, int tid) {
+  const int h = tid >> 4, p = tid & 15;
+  const int Dq = SML_LATENT_DIM + P.rope_dim;
+  const uint16_t* qh = P.q + ((size_t)t * P.H + g * kHC + h) * Dq;
+  uint4 v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = __ldg(reinterpret_cast<const uint4*>(qh + 32 * p) + i);
+  uint2 pv = make_uint2(0u, 0u);
+  if (P.rope_dim) pv = __ldg(reinterpret_cast<const uint2*>(qh + SML_LATENT_DIM + 4 * p));
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[k] << 16)), fabsf(__uint_as_float(w[k] & 0xffff0000u))));
+  }
+  if (kPlain) {
+    amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(pv.x << 16)), fabsf(__uint_as_float(pv.x & 0xffff0000u))));
+    amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(pv.y << 16)), fabsf(__uint_as_float(pv.y & 0xffff0000u))));
+  }
+#pragma unroll
+  for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  int e2 = 0;
+  if (amax > 0.f) frexpf(amax / 448.f, &e2);   // amax / 448 < 2^e2
+  const float inv = ldexpf(1.f, -e2);
+  if (p == 0) S.qs[h] = ldexpf(1.f, e2);
+  // dims [32 p, 32 p + 32) -> block p / 4, 16-B chunks 2 (p % 4) and 2 (p % 4) + 1
+  const int b = p >> 2;
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint4 vv = v[2 * c + (k >> 1)];
+      const uint32_t wa = (k & 1) ? vv.z : vv.x, wb = (k & 1) ? vv.w : vv.y;
+      float x0 = __uint_as_float(wa << 16) * inv, x1 = __uint_as_float(wa & 0xffff0000u) * inv;
+      float x2 = __uint_as_float(wb << 16) * inv, x3 = __uint_as_float(wb & 0xffff0000u) * inv;
+      const uint32_t h01 = split_e4m3x2(x0, x1), h23 = split_e4m3x2(x2, x3);
+      hw[k] = h01 | (h23 << 16);
+      lw[k] = f2_to_e4m3x2(x0, x1) | (f2_to_e4m3x2(x2, x3) << 16);
+    }
+    const int chunk = 2 * (p & 3) + c;
+    st_shared_v4(sw128(ptx::smem_u32(S.q8[b]), h, chunk), hw[0], hw[1], hw[2], hw[3]);
+    st_shared_v4(sw128(ptx::smem_u32(S.q8[b]), h + kHC, chunk), lw[0], lw[1], lw[2], lw[3]);
+  }
+  if (P.rope_dim) {
+    const uint32_t qb = ptx::smem_u32(S.qpe);
+    if (kPlain) {
+      // 4 E4M3 codes per term: bytes 4 p .. 4 p + 3 of rows h (high) and h + 16 (low)
+      float x0 = __uint_as_float(pv.x << 16) * inv, x1 = __uint_as_float(pv.x & 0xffff0000u) * inv;
+      float x2 = __uint_as_float(pv.y << 16) * inv, x3 = __uint_as_float(pv.y & 0xffff0000u) * inv;
+      const uint32_t h01 = split_e4m3x2(x0, x1), h23 = split_e4m3x2(x2, x3);
+      const uint32_t lo = f2_to_e4m3x2(x0, x1) | (f2_to_e4m3x2(x2, x3) << 16);
+      st_shared_b32(sw128(qb, h, p >> 2) + 4 * (p & 3), h01 | (h23 << 16));
+      st_shared_b32(sw128(qb, h + kHC, p >> 2) + 4 * (p & 3), lo);
+    } else {
+      // 4 bf16: bytes 8 p .. 8 p + 7 of row h
+      st_shared_v2(sw128(qb, h, p >> 1) + 8 * (p & 1), pv.x, pv.y);
+    }
+  }
 }
 
 // kPlain: the latent pool is plain E4M3 (576-B rows under one scale); else
-// fp8_ds_mla.  A template parameter, so that each gather loop is compiled for
-// its own row layout.
+// fp8_ds_mla.  A template parameter, so that each path is compiled for its
+// own row layout.
 template <bool kPlain>
-__global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params P) {
+__global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const Params P) {
   extern __shared__ uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x, hg = blockIdx.y, t = blockIdx.z;
-  ptx::griddep_wait();   // the selection comes from the previous kernel
-
-  // ---- this split's key range (uniform across the CTA) ----
-  const int r = request_of_warp(P.cu_q, P.B, t);
-  const Req rq = load_request(P.cu_q, P.ctx_len, r, P.T, P.max_ctx, P.max_pages);
-  const bool req_ok = rq.ok && t >= rq.q0 && t - rq.q0 < rq.Q;
-  const int n = req_ok ? rq.L - rq.Q + (t - rq.q0) + 1 : 0;
-  int len = req_ok ? __ldg(P.idx_len + t) : 0;
-  const int len_max = min(P.K, n);
-  if (len < 0 || len > len_max) {
-    if (split == 0 && hg == 0 && threadIdx.x == 0) raise_fault(P.status, SML_FAULT_TOPK_LEN);
-    len = max(0, min(len, len_max));
-  }
-  if (!req_ok && split == 0 && hg == 0 && threadIdx.x == 0) raise_fault(P.status, SML_FAULT_LENGTHS);
-  const int kb = split * P.ws.keys_per_split;
-  const int ke = min(len, kb + P.ws.keys_per_split);
-  const size_t slot0 = ((size_t)t * P.H + hg * kHC) * P.ws.splits + split;   // + h * splits
-  if (kb >= ke) {
-    // No selected key in this split: an empty partial (lse = -inf drops out of the merge).
-    for (int e = threadIdx.x; e < kHC * SML_LATENT_DIM; e += kThreads)
-      P.ws.part_out[(slot0 + (size_t)(e / SML_LATENT_DIM) * P.ws.splits) * SML_LATENT_DIM + e % SML_LATENT_DIM] = 0.f;
-    if (threadIdx.x < kHC) P.ws.part_lse[slot0 + (size_t)threadIdx.x * P.ws.splits] = -INFINITY;
-    return;
-  }
-  const int nkeys = ke - kb;
-  const int ntiles = (nkeys + kKT - 1) / kKT;
+  const MlaPlan& plan = P.ws.plan;
+  const long long ub = unit_begin(plan, blockIdx.x), ue = unit_begin(plan, blockIdx.x + 1);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(&S.e_full[i], kGatherWarps);   // one arrival per gather warp
-      ptx::mbar_init(&S.e_free[i], 1);   // PV of the tile done (it is the tile's last reader)
+      // every loader thread's copies (asynchronous arrivals) + one ordinary arrival
+      ptx::mbar_init(&S.full[i], kLoadThreads + 1);
+      ptx::mbar_init(&S.lat_free[i], 1);   // PV of the tile done (its last reader)
     }
-    ptx::mbar_init(&S.q_ready, 4);
+    ptx::mbar_init(&S.q_ready, 8);
     ptx::mbar_init(&S.s_full, 1);
-    ptx::mbar_init(&S.s_free, 4);
-    ptx::mbar_init(&S.p_full, 4);
+    ptx::mbar_init(&S.s_free, 8);
+    ptx::mbar_init(&S.p_full, 8);
     ptx::mbar_init(&S.pv_done, 1);
+    ptx::mbar_init(&S.o_free, 8);
     ptx::mbar_init(&S.drain, 1);
     S.abort = 0;
     ptx::fence_mbar_init();
@@ -312,380 +412,463 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
   // This CTA holds its tensor memory now, so a dependent grid scheduled on the
   // same SM cannot starve it of columns.
   if (threadIdx.x == 0) ptx::griddep_launch_dependents();
+  ptx::griddep_wait();   // the selection comes from the previous kernel
   volatile int* abort = &S.abort;
   const uint32_t T0 = S.tmem_base;
-  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
 
-  if (warp >= 4 && warp < 4 + kGatherWarps) {
-    // ================= gather warps: row offsets, then rows -> swizzled tiles =================
-    constexpr int kGT = 32 * kGatherWarps;
-    const int ct = threadIdx.x - 128;   // 0 .. kGT - 1
-    // Pool rows of the split's keys.
-    for (int k = ct; k < kMaxSplit; k += kGT) {
-      int32_t id = -1;
-      if (k < nkeys) {
-        const int pos = __ldg(P.idx + (size_t)t * P.K + kb + k);
-        if (pos >= 0 && pos < n) {
-          const int ph = __ldg(P.block_table + (size_t)r * P.max_pages + pos / SML_PAGE_TOKENS);
-          if (ph >= 0 && ph < P.latent_pages)
-            id = ph * SML_PAGE_TOKENS + pos % SML_PAGE_TOKENS;
-          else
-            raise_fault(P.status, SML_FAULT_PAGE);
-        } else {
-          raise_fault(P.status, SML_FAULT_INDEX);
-        }
-      }
-      S.rowid[k] = id;
-    }
-    asm volatile("bar.sync 2, %0;" ::"n"(kGT) : "memory");
-    // Rows -> tiles in batches of kBatchRows rows per warp (a tile is
-    // kKT / kBatchRows batches; batch i goes to warp i % kGatherWarps): the
-    // batch's loads go into registers first (lane l: 16-B latent chunk l, then
-    // lane 0 the four scales and lanes 1-8 the RoPE key), then the warp waits
-    // for the tile's buffer to be free and stores them 128-B-swizzled, so the
-    // loads are in flight while the buffer drains.  A masked row is zeros.  A
-    // warp signals a tile after storing its last batch of it.
-    const int gw = warp - 4;
-    const int nb_total = ntiles * kBatchesPerTile;
+  // Each role moves its warpgroup's register share first (the lowering ones
+  // free what the raising ones take; every warpgroup takes exactly one branch).
+  if (warp >= kWarpLoad) {
+    // ================= loaders: pool rows, then row copies =================
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+    const int lt = threadIdx.x - 32 * kWarpLoad;   // 0 .. kLoadThreads - 1
+    constexpr int kRow = kPlain ? SML_LATENT_E4M3_ROW_BYTES : SML_LATENT_ROW_BYTES;
+    // A row as 16-B chunks: 0-31 the 512-B latent (chunk c: block c / 8,
+    // 16-B column c % 8); fp8_ds_mla, 32 the four block scales and 33-40 the
+    // bf16 RoPE key; plain E4M3, 32-35 the 64 RoPE codes (the only bytes of
+    // the row the RoPE MMA reads).  The tile's chunks are numbered row-major
+    // and dealt out to the loader threads in order (chunk lt + kLoadThreads
+    // i), so a warp's 32 chunks are mostly of one row.
+    const int parts = kPlain ? (P.rope_dim ? 36 : 32) : (P.rope_dim ? 41 : 33);
+    const int drow = kLoadThreads / parts, dpart = kLoadThreads - drow * parts;
+    const int row0 = lt / parts, part0 = lt - row0 * parts;
+    int k = 0;   // tiles so far
     bool ok = true;
-    for (int bi = gw; bi < nb_total; bi += kGatherWarps) {
-      const int tile = bi / kBatchesPerTile, buf = tile & 1;
-      const int row0 = (bi % kBatchesPerTile) * kBatchRows;
-      uint4 va[kBatchRows], vb[kBatchRows];
-      uint32_t live = 0;   // bit u: row u of the batch is a selected row (plain E4M3 only)
-#pragma unroll
-      for (int u = 0; u < kBatchRows; ++u) {
-        const int32_t id = S.rowid[tile * kKT + row0 + u];
-        const uint8_t* src =
-            P.latent + (size_t)(id >= 0 ? id : 0) * (kPlain ? SML_LATENT_E4M3_ROW_BYTES : SML_LATENT_ROW_BYTES);
-        va[u] = make_uint4(0u, 0u, 0u, 0u);
-        vb[u] = make_uint4(0u, 0u, 0u, 0u);
-        if (id >= 0) {
-          if (kPlain) live |= 1u << u;
-          va[u] = ldg_stream(src + 16 * lane);
-          // fp8_ds_mla: lane 0 the four block scales, lanes 1-8 the bf16 RoPE
-          // key; plain E4M3: lanes 0-3 the 64 RoPE codes
-          if (kPlain ? (lane < 4 && P.rope_dim) : (lane == 0 || (lane <= 8 && P.rope_dim)))
-            vb[u] = ldg_stream(src + SML_LATENT_DIM + 16 * lane);
-        }
+    for (long long u = ub; ok && u < ue;) {
+      const Seg s = segment_at(P, u, ue);
+      u += s.nj;
+      if (lt == 0) {
+        if (!s.req_ok) raise_fault(P.status, SML_FAULT_LENGTHS);
+        else if (s.len_bad) raise_fault(P.status, SML_FAULT_TOPK_LEN);
       }
-      // first batch of this tile for this warp: the buffer must be free (PV of tile - 2 done)
-      if (tile >= 2 && bi - kGatherWarps < tile * kBatchesPerTile &&
-          !warp_wait(&S.e_free[buf], ((tile >> 1) - 1) & 1, abort)) {
-        ok = false;
-        break;
-      }
-      const uint32_t lat_l = ptx::smem_u32(S.lat[buf][lane >> 3]);
-      const uint32_t pe_b = ptx::smem_u32(S.pe[buf]);
-      const uint32_t sc_b = ptx::smem_u32(&S.sc[buf][0][0]);
-#pragma unroll
-      for (int u = 0; u < kBatchRows; ++u) {
-        const int row = row0 + u;
-        st_shared_v4(sw128(lat_l, row, lane & 7), va[u].x, va[u].y, va[u].z, va[u].w);
-        if (kPlain) {
-          // one scale for every block (zero for a masked row); RoPE codes
-          // widened to bf16 (exact: E4M3 values are bf16 values)
-          if (lane == 0) {
-            const uint32_t sb = (live >> u) & 1 ? __float_as_uint(P.latent_scale) : 0u;
-            st_shared_v4(sc_b + row * 16, sb, sb, sb, sb);
-          }
-          if (lane < 4 && P.rope_dim) {
-            const uint32_t w[4] = {vb[u].x, vb[u].y, vb[u].z, vb[u].w};
-            uint32_t o[8];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float2 lo = e4m3x2_to_f2(w[k]), hi = e4m3x2_to_f2(w[k] >> 16);
-              o[2 * k] = bf16x2_bits(lo.x, lo.y);
-              o[2 * k + 1] = bf16x2_bits(hi.x, hi.y);
+      for (int jj = 0; jj < s.ne; ++jj, ++k) {
+        const int j = s.j0 + jj, buf = k & 1;
+        int32_t* rowid = S.rowid[k & 3];   // last used by tile k - 4, whose softmax is done
+        // pool row of the tile's key lt (loaded before the buffer is free)
+        if (lt < kKT) {
+          int rid = -1;
+          const int key = j * kKT + lt;
+          if (key < s.len) {
+            const int pos = __ldg(P.idx + (size_t)s.t * P.K + key);
+            if (pos >= 0 && pos < s.n) {
+              const int ph = __ldg(P.block_table + (size_t)s.r * P.max_pages + pos / SML_PAGE_TOKENS);
+              if (ph >= 0 && ph < P.latent_pages) rid = ph * SML_PAGE_TOKENS + pos % SML_PAGE_TOKENS;
+              else raise_fault(P.status, SML_FAULT_PAGE);
+            } else {
+              raise_fault(P.status, SML_FAULT_INDEX);
             }
-            st_shared_v4(sw128(pe_b, row, 2 * lane), o[0], o[1], o[2], o[3]);
-            st_shared_v4(sw128(pe_b, row, 2 * lane + 1), o[4], o[5], o[6], o[7]);
           }
-        } else if (lane == 0) {
-          st_shared_v4(sc_b + row * 16, vb[u].x, vb[u].y, vb[u].z, vb[u].w);
-        } else if (lane <= 8 && P.rope_dim) {
-          st_shared_v4(sw128(pe_b, row, lane - 1), vb[u].x, vb[u].y, vb[u].z, vb[u].w);
+          rowid[lt] = rid;
         }
-      }
-      if (bi + kGatherWarps >= (tile + 1) * kBatchesPerTile) {   // this warp's last batch of the tile
-        ptx::fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&S.e_full[buf]);
+        // the buffer's last tile (k - 2) has been read by its PV
+        if (k >= 2) ok = warp_wait(&S.lat_free[buf], ((k >> 1) - 1) & 1, abort);
+        ok = loader_all(ok);   // the tile's row ids written, and the wait's outcome shared
+        if (!ok) break;
+        // the row ids are generic writes the softmax reads: released by this
+        // arrival (after the barrier above); the copies arrive by themselves
+        if (lt == 0) ptx::mbar_arrive(&S.full[buf]);
+        const uint32_t lat0 = ptx::smem_u32(S.lat[buf][0]);
+        const uint32_t pe0 = ptx::smem_u32(S.pe[buf]);
+        const uint32_t sc0 = ptx::smem_u32(&S.sc[buf][0][0]);
+        int row = row0, part = part0;
+        for (; row < kKT; row += drow, part += dpart) {
+          if (part >= parts) {
+            part -= parts;
+            ++row;
+            if (row >= kKT) break;
+          }
+          const int id = rowid[row];
+          const uint8_t* src = P.latent + (size_t)(id >= 0 ? id : 0) * kRow + 16 * part;
+          uint32_t dst;
+          if (part < 32) dst = sw128(lat0 + (part >> 3) * kLatBlock, row, part & 7);
+          else if (kPlain) dst = sw128(pe0, row, part - 32);
+          else if (part == 32) dst = sc0 + 16 * row;
+          else dst = sw128(pe0, row, part - 33);
+          ptx::cp_async16(dst, src, id >= 0 ? 16u : 0u);   // a masked row is zero-filled, nothing read
+        }
+        // This thread's copies arrive on the buffer's barrier once they have
+        // landed (generic-proxy writes: the MMA thread fences them for its
+        // async-proxy reads after it sees the barrier complete).
+        ptx::cp_async_arrive_noinc(&S.full[buf]);
       }
     }
     if (!ok) *abort = 1;
+    ptx::cp_async_wait_all();   // nothing in flight when the CTA's shared memory goes away
+    __syncwarp();
   } else if (warp == kWarpMma) {
     // ================= MMA issuer =================
-    if (lane == 0) {
-      const uint32_t id_qk = ptx::idesc_f16(2 * kHC, 0, 0, 0);   // E4M3 x E4M3, both K-major, N = 32
-      const uint32_t id_pe = ptx::idesc_f16(kHC, 1, 0, 0);       // bf16, N = 16
-      const uint32_t id_pv = ptx::idesc_f16(3 * kHC, 0, 1, 1);   // E4M3 x E4M3, both MN-major, N = 48
-      auto issue_qk = [&](int buf) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+    const uint32_t id_qk = ptx::idesc_f16(2 * kHC, 0, 0, 0);   // E4M3 x E4M3, both K-major, N = 32
+    const uint32_t id_pe = ptx::idesc_f16(kHC, 1, 0, 0);       // bf16, N = 16
+    const uint32_t id_pv = ptx::idesc_f16(3 * kHC, 0, 1, 1);   // E4M3 x E4M3, both MN-major, N = 48
+    auto issue_qk = [&](int buf) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {   // 32 latent dims per step
+      for (int kk = 0; kk < 4; ++kk) {   // 32 latent dims per step
 #pragma unroll
-          for (int b = 0; b < 4; ++b)
-            ptx::mma_f8f6f4_ss(T0 + kColS + 32 * b, ptx::sdesc_sw128(ptx::smem_u32(S.lat[buf][b]) + 32 * k),
-                               ptx::sdesc_sw128(ptx::smem_u32(S.q8[b]) + 32 * k), id_qk, k > 0);
-          if (P.rope_dim)
-            ptx::mma_f16_ss(T0 + kColSpe, ptx::sdesc_sw128(ptx::smem_u32(S.pe[buf]) + 32 * k),
-                            ptx::sdesc_sw128(ptx::smem_u32(S.qpe) + 32 * k), id_pe, k > 0);
+        for (int b = 0; b < 4; ++b)
+          ptx::mma_f8f6f4_ss(T0 + kColS + 32 * b, ptx::sdesc_sw128(ptx::smem_u32(S.lat[buf][b]) + 32 * kk),
+                             ptx::sdesc_sw128(ptx::smem_u32(S.q8[b]) + 32 * kk), id_qk, kk > 0);
+        if (P.rope_dim) {
+          if (!kPlain)
+            ptx::mma_f16_ss(T0 + kColSpe, ptx::sdesc_sw128(ptx::smem_u32(S.pe[buf]) + 32 * kk),
+                            ptx::sdesc_sw128(ptx::smem_u32(S.qpe) + 32 * kk), id_pe, kk > 0);
+          else if (kk < 2)   // 64 E4M3 RoPE codes: two steps of 32
+            ptx::mma_f8f6f4_ss(T0 + kColSpe, ptx::sdesc_sw128(ptx::smem_u32(S.pe[buf]) + 32 * kk),
+                               ptx::sdesc_sw128(ptx::smem_u32(S.qpe) + 32 * kk), id_qk, kk > 0);
         }
-        ptx::mma_commit(&S.s_full);
-      };
-      bool ok = ptx::mbar_wait(&S.q_ready, 0, abort) && ptx::mbar_wait(&S.e_full[0], 0, abort);
-      if (ok) {
-        ptx::tc_fence_after();
-        issue_qk(0);
       }
-      for (int tile = 0; ok && tile < ntiles; ++tile) {
-        const int buf = tile & 1;
-        if (tile + 1 < ntiles) {
-          // next tile's QK^T once its rows have landed and the softmax has read S
-          if (!ptx::mbar_wait(&S.e_full[buf ^ 1], ((tile + 1) >> 1) & 1, abort) ||
-              !ptx::mbar_wait(&S.s_free, tile & 1, abort)) {
-            ok = false;
-            break;
-          }
+      ptx::mma_commit(&S.s_full);
+    };
+    // O_b^T (+)= C_b^T . B_b^T, 32 keys per step.  A: the latent tile read
+    // MN-major (dims contiguous; 8-key swizzle atoms 1,024 B apart).  B: 8-key
+    // x 16-B core matrices, the three terms 128 B apart, 8-key groups 384 B
+    // apart.  The first tile of a (token, head group) overwrites O; it waits
+    // until the epilogue of the one before has read O.
+    auto issue_pv = [&](int kk, bool first) {
+      const int buf = kk & 1;
+#pragma unroll
+      for (int st = 0; st < kKT / 32; ++st) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          ptx::mma_f8f6f4_ss(T0 + kColO + kOStride * b,
+                             ptx::sdesc(ptx::smem_u32(S.lat[buf][b]) + 4096 * st, 16384, 1024, 2),
+                             ptx::sdesc(ptx::smem_u32(S.pb[b]) + 1536 * st, 384, 128, 0), id_pv,
+                             !first || st > 0);
+      }
+      ptx::mma_commit(&S.pv_done);
+      ptx::mma_commit(&S.lat_free[buf]);
+    };
+    // Two cursors over the CTA's tiles: the next QK^T and the next PV.  A
+    // tile's QK^T needs its rows, the softmax done reading the last S (S is
+    // one accumulator) and, for the first tile of a (token, head group), the
+    // staged query; its PV needs its weights and, for the first tile of a
+    // (token, head group) after the first, the epilogue of the one before
+    // done reading O.  Whichever is ready goes first; QK^T runs at most one
+    // tile ahead of PV.
+    Cur cq, cv;
+    cur_start(cq, P, ub, ue);
+    cur_start(cv, P, ub, ue);
+    bool ok = true;
+    uint32_t idle = 0;
+    while (ok && cv.valid) {
+      int act = 0;   // 1: PV of cv, 2: QK^T of cq, -1: gave up
+      if (lane == 0) {
+        const bool pv_first = cv.jj == 0 && cv.seg > 0;
+        const bool pv_ready = cv.k < cq.k && ptx::mbar_test_wait(&S.p_full, cv.k & 1) &&
+                              (!pv_first || ptx::mbar_test_wait(&S.o_free, (cv.seg - 1) & 1));
+        if (pv_ready) {
+          act = 1;
+        } else if (cq.valid && cq.k <= cv.k + 1 && (cq.jj > 0 || ptx::mbar_test_wait(&S.q_ready, cq.seg & 1)) &&
+                   ptx::mbar_test_wait(&S.full[cq.k & 1], (cq.k >> 1) & 1) &&
+                   (cq.k == 0 || ptx::mbar_test_wait(&S.s_free, (cq.k - 1) & 1))) {
+          act = 2;
+        } else if (*abort || ++idle > (1u << 22)) {
+          act = -1;
+        } else {
+          // sleep on the barrier the next step most likely waits for
+          if (cv.k < cq.k) ptx::mbar_try_wait_ns(&S.p_full, cv.k & 1, 200);
+          else if (cq.valid) ptx::mbar_try_wait_ns(&S.full[cq.k & 1], (cq.k >> 1) & 1, 200);
+        }
+        if (act == 1) {
           ptx::tc_fence_after();
-          issue_qk(buf ^ 1);
+          issue_pv(cv.k, cv.jj == 0);
+        } else if (act == 2) {
+          // the copies are generic-proxy writes: order them before the MMAs' reads
+          ptx::fence_proxy_async();
+          ptx::tc_fence_after();
+          issue_qk(cq.k & 1);
         }
-        if (!ptx::mbar_wait(&S.p_full, tile & 1, abort)) {
-          ok = false;
-          break;
-        }
-        ptx::tc_fence_after();
-        // O_b^T += C_b^T . B_b^T, 32 keys per step.  A: the latent tile read
-        // MN-major (dims contiguous; 8-key swizzle atoms 1,024 B apart).  B:
-        // 8-key x 16-B core matrices, the three terms 128 B apart, 8-key
-        // groups 384 B apart.
-#pragma unroll
-        for (int k = 0; k < kKT / 32; ++k) {
-#pragma unroll
-          for (int b = 0; b < 4; ++b)
-            ptx::mma_f8f6f4_ss(T0 + kColO + kOStride * b, ptx::sdesc(ptx::smem_u32(S.lat[buf][b]) + 4096 * k, 16384, 1024, 2),
-                               ptx::sdesc(ptx::smem_u32(S.pb[b]) + 1536 * k, 384, 128, 0), id_pv, (tile | k) != 0);
-        }
-        ptx::mma_commit(&S.pv_done);
-        ptx::mma_commit(&S.e_free[buf]);
       }
+      act = __shfl_sync(0xffffffffu, act, 0);
+      if (act == 1) {
+        cur_next(cv, P, ue);
+        idle = 0;
+      } else if (act == 2) {
+        cur_next(cq, P, ue);
+        idle = 0;
+      } else if (act < 0) {
+        ok = false;
+      }
+    }
+    if (lane == 0) {
       if (!ok) *abort = 1;
+      // every MMA this thread issued has finished before TMEM is released
       ptx::mma_commit(&S.drain);
       ptx::mbar_wait(&S.drain, 0, nullptr, 1u << 20);
     }
     __syncwarp();
   } else {
-    // ================= softmax: warps 0-3, thread = key row / latent dim =================
-    const int row = warp * 32 + lane;
-    {
-      // Query of the 16 heads.  Nope part: q = s_h (hi + lo), hi and lo E4M3 and
-      // s_h a power of two >= amax_h / 448, so q / s_h, its rounding to hi and
-      // the residual lo are exact in fp32, and lo is exact in E4M3 (a bf16 has
-      // 8 significant bits, hi takes 4, the residual the other 4) down to
-      // E4M3's subnormal step.  RoPE part copied as bf16.
-      const int Dq = SML_LATENT_DIM + P.rope_dim;
-      const int h = row >> 3, part = row & 7;   // 8 threads per head, 64 nope dims each
-      const uint16_t* qh = P.q + ((size_t)t * P.H + hg * kHC + h) * Dq;
-      uint4 v[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = __ldg(reinterpret_cast<const uint4*>(qh + 64 * part) + i);
-      uint4 pv = make_uint4(0u, 0u, 0u, 0u);
-      if (P.rope_dim) pv = __ldg(reinterpret_cast<const uint4*>(qh + SML_LATENT_DIM) + part);   // 8 bf16
-      float amax = 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[k] << 16)), fabsf(__uint_as_float(w[k] & 0xffff0000u))));
-      }
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-      int e2 = 0;
-      if (amax > 0.f) frexpf(amax / 448.f, &e2);        // amax / 448 < 2^e2
-      const float qscale = ldexpf(1.f, e2), inv = ldexpf(1.f, -e2);
-      if (part == 0) S.qs[h] = qscale;
-      // dims [64 part, 64 part + 64) -> block part / 2, 16-B chunks 4 (part % 2) + c
-      const int b = part >> 1;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t hw[4], lw[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          // elements 16 c + 4 k .. + 3 of this thread's 64
-          const uint4 vv = v[2 * c + (k >> 1)];
-          const uint32_t wa = (k & 1) ? vv.z : vv.x, wb = (k & 1) ? vv.w : vv.y;
-          float x0 = __uint_as_float(wa << 16) * inv, x1 = __uint_as_float(wa & 0xffff0000u) * inv;
-          float x2 = __uint_as_float(wb << 16) * inv, x3 = __uint_as_float(wb & 0xffff0000u) * inv;
-          const uint32_t h01 = split_e4m3x2(x0, x1), h23 = split_e4m3x2(x2, x3);
-          hw[k] = h01 | (h23 << 16);
-          lw[k] = f2_to_e4m3x2(x0, x1) | (f2_to_e4m3x2(x2, x3) << 16);
-        }
-        const int chunk = 4 * (part & 1) + c;
-        st_shared_v4(sw128(ptx::smem_u32(S.q8[b]), h, chunk), hw[0], hw[1], hw[2], hw[3]);
-        st_shared_v4(sw128(ptx::smem_u32(S.q8[b]), h + kHC, chunk), lw[0], lw[1], lw[2], lw[3]);
-      }
-      st_shared_v4(sw128(ptx::smem_u32(S.qpe), h, part), pv.x, pv.y, pv.z, pv.w);
+    // ================= softmax: warps 0-7 =================
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    const int q4 = warp & 3, hh = warp >> 2;   // TMEM lane quarter (keys / dims), head half
+    const int row = 32 * q4 + lane;
+    const int tid = threadIdx.x;                // 0 .. 255
+    const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
+    // The query of a (token, head group) is staged, and q_ready signalled,
+    // before the epilogue of the non-empty one before it: the MMA issues the
+    // first QK^T of the next before the last PV of the current, and that PV
+    // is what the epilogue waits for.
+    auto stage = [&](const Seg& s) {
+      stage_query<kPlain>(P, S, s.t, s.g, tid);
       ptx::fence_proxy_async();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&S.q_ready);
-    }
-    const float zscale = P.sm_scale * (P.ssmax ? P.ssmax_s * logf((float)max(n, 1)) : 1.f);
-    float lrow[kHC];   // this key row's share of the row sums
-#pragma unroll
-    for (int h = 0; h < kHC; ++h) lrow[h] = 0.f;
-    if (row < kHC) {
-      S.hm[row] = -INFINITY;
-      S.hsig[row] = 0.f;
-    }
-    bool ok = softmax_all(warp_wait(&S.q_ready, 0, abort));   // S.qs; orders the init above
-    for (int tile = 0; ok && tile < ntiles; ++tile) {
-      const int buf = tile & 1;
-      if (!softmax_all(warp_wait(&S.e_full[buf], (tile >> 1) & 1, abort) && warp_wait(&S.s_full, tile & 1, abort))) {
-        ok = false;
-        break;
+    };
+    int k = 0;
+    bool ok = true, staged = false;
+    for (long long u = ub; u < ue;) {
+      const Seg s = segment_at(P, u, ue);
+      u += s.nj;
+      // every softmax thread is done with the last (token, head group): its S.qs and S.xsum
+      ok = softmax_all(ok);
+      if (!ok) break;
+      float* pout = P.ws.part_out + s.slot * kHC * SML_LATENT_DIM;
+      float* plse = P.ws.part_lse + s.slot * kHC;
+      if (s.ne == 0) {
+        // no selected key in this CTA's tiles of it: an empty partial (lse = -inf drops out of the merge)
+        for (int i = tid; i < kHC * SML_LATENT_DIM; i += kSoftmaxThreads) pout[i] = 0.f;
+        if (tid < kHC) plse[tid] = -INFINITY;
+        continue;
       }
-      ptx::tc_fence_after();
-      const bool valid = S.rowid[tile * kKT + row] >= 0;
-      float sc[4];
+      if (!staged) stage(s);
+      staged = false;
+      ok = softmax_all(ok);   // S.qs visible to every softmax thread
+      float qsh[8];
 #pragma unroll
-      for (int b = 0; b < 4; ++b) sc[b] = S.sc[buf][row][b];
-      // z = zscale * (s_h * sum_b scale_b (S_b,hi + S_b,lo) + S_pe), fp32
-      float z[kHC];
-      {
+      for (int h = 0; h < 8; ++h) qsh[h] = S.qs[8 * hh + h];
+      // logits in log2 units: z log2(e), so that p = 2^(z - m)
+      const float zscale = P.sm_scale * (P.ssmax ? P.ssmax_s * logf((float)s.nss) : 1.f) * kLog2e;
+      // per head of this half (identical in all its threads): running max m,
+      // weight scale sigma (0 = not set yet), and this key row's row-sum share
+      float m[8], sig[8], isig[8], lrow[8];
 #pragma unroll
-        for (int h = 0; h < kHC; ++h) z[h] = 0.f;
+      for (int h = 0; h < 8; ++h) {
+        m[h] = -INFINITY;
+        sig[h] = 0.f;
+        isig[h] = 0.f;
+        lrow[h] = 0.f;
+      }
+      for (int jj = 0; jj < s.ne; ++jj, ++k) {
+        const int buf = k & 1;
+        ok = ok && warp_wait(&S.full[buf], (k >> 1) & 1, abort) && warp_wait(&S.s_full, k & 1, abort);
+        if (!ok) *abort = 1;
+        ok = softmax_all(ok);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const bool valid = S.rowid[k & 3][row] >= 0;
+        float sc[4];
+        if (kPlain) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b) sc[b] = valid ? P.latent_scale : 0.f;
+        } else {
+          const float4 v4 = *reinterpret_cast<const float4*>(&S.sc[buf][row][0]);
+          sc[0] = v4.x;
+          sc[1] = v4.y;
+          sc[2] = v4.z;
+          sc[3] = v4.w;
+        }
+        // z = zscale * (s_h * sum_b scale_b (S_b,hi + S_b,lo) + S_pe), fp32
+        float z[8];
+#pragma unroll
+        for (int h = 0; h < 8; ++h) z[h] = 0.f;
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
-          uint32_t v[32];
-          ptx::tmem_ld32(T0 + kColS + 32 * b + lane_off, v);
-          ptx::tmem_wait_ld(v);
+          uint32_t vh[8], vl[8];
+          ptx::tmem_ld8(T0 + kColS + 32 * b + 8 * hh + lane_off, vh);
+          ptx::tmem_ld8(T0 + kColS + 32 * b + kHC + 8 * hh + lane_off, vl);
+          ptx::tmem_wait_ld(vh, vl);
 #pragma unroll
-          for (int h = 0; h < kHC; ++h) z[h] = fmaf(sc[b], __uint_as_float(v[h]) + __uint_as_float(v[kHC + h]), z[h]);
+          for (int h = 0; h < 8; ++h) z[h] = fmaf(sc[b], __uint_as_float(vh[h]) + __uint_as_float(vl[h]), z[h]);
         }
 #pragma unroll
-        for (int h = 0; h < kHC; ++h) z[h] *= S.qs[h];
+        for (int h = 0; h < 8; ++h) z[h] *= qsh[h];
         if (P.rope_dim) {
-          // plain E4M3 keys hold codes: their scale multiplies the RoPE term
-          const float pe_scale = kPlain ? P.latent_scale : 1.f;
-          uint32_t v[16];
-          ptx::tmem_ld16(T0 + kColSpe + lane_off, v);
-          ptx::tmem_wait_ld(v);
+          if (kPlain) {
+            // RoPE codes under the pool scale, both query terms
+            uint32_t vh[8], vl[8];
+            ptx::tmem_ld8(T0 + kColSpe + 8 * hh + lane_off, vh);
+            ptx::tmem_ld8(T0 + kColSpe + kHC + 8 * hh + lane_off, vl);
+            ptx::tmem_wait_ld(vh, vl);
 #pragma unroll
-          for (int h = 0; h < kHC; ++h) z[h] = fmaf(pe_scale, __uint_as_float(v[h]), z[h]);
+            for (int h = 0; h < 8; ++h)
+              z[h] = fmaf(qsh[h] * P.latent_scale, __uint_as_float(vh[h]) + __uint_as_float(vl[h]), z[h]);
+          } else {
+            uint32_t v[8];
+            ptx::tmem_ld8(T0 + kColSpe + 8 * hh + lane_off, v);
+            ptx::tmem_wait_ld(v);
+#pragma unroll
+            for (int h = 0; h < 8; ++h) z[h] += __uint_as_float(v[h]);
+          }
         }
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&S.s_free);   // S read: the next tile's QK^T may overwrite it
 #pragma unroll
-        for (int h = 0; h < kHC; ++h) z[h] = valid ? z[h] * zscale : -INFINITY;
+        for (int h = 0; h < 8; ++h) z[h] = valid ? z[h] * zscale : -INFINITY;
+        // Tile statistics: each head's maximum over the 128 keys, and the
+        // tile's largest block scale (masked rows were zero-filled: scale 0).
+        {
+          float* xm = S.xmax[k & 1][hh][q4];
+#pragma unroll
+          for (int h = 0; h < 8; ++h) {
+            const float w = ptx::warp_max_f32(z[h]);
+            if (lane == 0) xm[h] = w;
+          }
+          const float scw = ptx::warp_max_f32(fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])));
+          if (lane == 0) xm[8] = scw;
+        }
+        half_sync(hh);
+        float tm[8], SC = 0.f;
+#pragma unroll
+        for (int h = 0; h < 8; ++h) tm[h] = -INFINITY;
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const float* xm = S.xmax[k & 1][hh][qq];
+#pragma unroll
+          for (int h = 0; h < 8; ++h) tm[h] = fmaxf(tm[h], xm[h]);
+          SC = fmaxf(SC, xm[8]);
+        }
+        // Lazily raised running max m_h and weight scale sigma_h.  The tile's
+        // weights are at most 2^(tmax_h - m_h) * SC and must stay <= 448
+        // sigma_h; sigma_h is reset to the power of two just above U_h / 448
+        // (U_h below, with a margin for the approximate 2^x) whenever U_h
+        // leaves [28, 448] sigma_h, so the dominant weights keep all 12 bits
+        // of the three-term split.  O holds sum(weights / sigma), so both
+        // changes rescale it by f_h = 2^(m_old - m_new) * sigma_old /
+        // sigma_new (exact for the sigma part: powers of two).
+        float f[8];
+        bool any = false;
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+          float alpha = 1.f;
+          if (tm[h] > m[h] + kLazyRescale || (m[h] == -INFINITY && tm[h] != -INFINITY)) {
+            alpha = ex2(m[h] - tm[h]);   // 0 when m was -inf
+            m[h] = tm[h];
+          }
+          const float U = tm[h] == -INFINITY ? 0.f : fmaxf(ex2(tm[h] - m[h]) * 1.001f, 1.f) * SC;
+          float beta = 1.f;
+          if (U > 0.f && (U > 448.f * sig[h] || U < 28.f * sig[h])) {
+            // U / 448 in [2^(E - 127), 2^(E - 126)): sigma = 2^(E - 126), 1 / sigma = 2^(126 - E)
+            const uint32_t E = (__float_as_uint(U * (1.f / 448.f)) >> 23) & 0xffu;
+            const float ns = __uint_as_float((E + 1u) << 23), nis = __uint_as_float((253u - E) << 23);
+            beta = sig[h] > 0.f ? sig[h] * nis : 1.f;
+            sig[h] = ns;
+            isig[h] = nis;
+          }
+          f[h] = alpha * beta;
+          any = any || f[h] != 1.f;
+          lrow[h] *= alpha;
+        }
+        // The previous tile's PV reads the weight tiles and accumulates into
+        // O: wait for it before rescaling O or overwriting the weights (the
+        // previous (token, head group)'s last PV was waited for by its
+        // epilogue).
+        if (jj > 0) {
+          ok = warp_wait(&S.pv_done, (k - 1) & 1, abort);
+          if (!ok) {
+            *abort = 1;
+            continue;   // the next softmax_all ends every softmax warp
+          }
+          ptx::tc_fence_after();
+          if (any) {
+#pragma unroll 1
+            for (int b = 0; b < 4; ++b) {   // this thread: latent dim 128 b + row, this half's heads
+#pragma unroll
+              for (int term = 0; term < 3; ++term) {
+                uint32_t ov[8];
+                const uint32_t a = T0 + kColO + kOStride * b + kHC * term + 8 * hh + lane_off;
+                ptx::tmem_ld8(a, ov);
+                ptx::tmem_wait_ld(ov);
+#pragma unroll
+                for (int h = 0; h < 8; ++h) ov[h] = __float_as_uint(__uint_as_float(ov[h]) * f[h]);
+                ptx::tmem_st8(a, ov);
+              }
+            }
+            ptx::tmem_wait_st();
+          }
+        }
+        // p = 2^(z - m) (0 for a masked key); weights x = p * scale_b / sigma as hi + mid + lo (E4M3)
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+          const float p = z[h] == -INFINITY ? 0.f : ex2(z[h] - m[h]);
+          lrow[h] += p;
+          z[h] = p * isig[h];
+        }
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          uint32_t wh[2], wm[2], wl[2];
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq) {   // heads 4 qq .. 4 qq + 3 of this half
+            uint32_t h01, m01, l01, h23, m23, l23;
+            split3_e4m3x2(z[4 * qq] * sc[b], z[4 * qq + 1] * sc[b], h01, m01, l01);
+            split3_e4m3x2(z[4 * qq + 2] * sc[b], z[4 * qq + 3] * sc[b], h23, m23, l23);
+            wh[qq] = h01 | (h23 << 16);
+            wm[qq] = m01 | (m23 << 16);
+            wl[qq] = l01 | (l23 << 16);
+          }
+          const uint32_t pb = ptx::smem_u32(S.pb[b]) + (row >> 3) * 384 + (row & 7) * 16 + 8 * hh;
+          st_shared_v2(pb, wh[0], wh[1]);
+          st_shared_v2(pb + 128, wm[0], wm[1]);
+          st_shared_v2(pb + 256, wl[0], wl[1]);
+        }
+        ptx::fence_proxy_async();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&S.p_full);
       }
-      // the tile's largest block scale (masked rows were zero-filled: scale 0)
-      float scm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) scm = fmaxf(scm, __shfl_xor_sync(0xffffffffu, scm, o));
-      if (lane == 0) S.scw[tile & 1][warp] = scm;
-      const bool any = tile_stats(S, row, z, tile);
-#pragma unroll
-      for (int h = 0; h < kHC; ++h) lrow[h] *= S.halpha[h];
-      // The previous tile's PV reads the weight tiles and accumulates into O:
-      // wait for it before rescaling O or overwriting the weights.
-      if (tile > 0) {
-        if (!softmax_all(warp_wait(&S.pv_done, (tile - 1) & 1, abort))) {
-          ok = false;
+      // the next non-empty (token, head group)'s query
+      for (long long v = u; ok && v < ue;) {
+        const Seg nx = segment_at(P, v, ue);
+        v += nx.nj;
+        if (nx.ne > 0) {
+          stage(nx);
+          staged = true;
           break;
         }
-        ptx::tc_fence_after();
-        if (any) {
+      }
+      // ---- epilogue of this (token, head group) ----
+      ok = ok && warp_wait(&S.pv_done, (k - 1) & 1, abort);
+      if (!ok) *abort = 1;
+      ok = softmax_all(ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      // row sums over the 128 keys (four warps of this half)
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        float v = lrow[h];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) S.xsum[hh][q4][h] = v;
+      }
+      half_sync(hh);
+      float osc[8];
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        const float l = S.xsum[hh][0][h] + S.xsum[hh][1][h] + S.xsum[hh][2][h] + S.xsum[hh][3][h];
+        osc[h] = l > 0.f ? sig[h] / l : 0.f;
+        if (q4 == 0 && lane == h) plse[8 * hh + h] = l > 0.f ? (m[h] + log2f(l)) * kLn2 : -INFINITY;
+      }
+      // out = sigma_h (hi + mid + lo) / l_h: this thread's latent dim 128 b + row
 #pragma unroll 1
-          for (int b = 0; b < 4; ++b) {   // this thread: latent dim 128 b + row
-            uint32_t ov[32], ow[16];
-            ptx::tmem_ld32(T0 + kColO + kOStride * b + lane_off, ov);
-            ptx::tmem_ld16(T0 + kColO + kOStride * b + 32 + lane_off, ow);
-            ptx::tmem_wait_ld(ov, ow);
-#pragma unroll
-            for (int h = 0; h < kHC; ++h) {
-              const float f = S.hf[h];
-              ov[h] = __float_as_uint(__uint_as_float(ov[h]) * f);
-              ov[kHC + h] = __float_as_uint(__uint_as_float(ov[kHC + h]) * f);
-              ow[h] = __float_as_uint(__uint_as_float(ow[h]) * f);
-            }
-            ptx::tmem_st32(T0 + kColO + kOStride * b + lane_off, ov);
-            ptx::tmem_st16(T0 + kColO + kOStride * b + 32 + lane_off, ow);
-          }
-          ptx::tmem_wait_st();
-        }
-      }
-      // p = exp(z - m); weights x = p * scale_b / sigma as hi + mid + lo (E4M3)
-#pragma unroll
-      for (int h = 0; h < kHC; ++h) {
-        const float p = z[h] == -INFINITY ? 0.f : expf(z[h] - S.hm[h]);
-        lrow[h] += p;
-        z[h] = p * S.hinv[h];
-      }
-#pragma unroll
       for (int b = 0; b < 4; ++b) {
-        uint32_t wh[4], wm[4], wl[4];
+        uint32_t oh[8], om[8], ol[8];
+        const uint32_t a = T0 + kColO + kOStride * b + 8 * hh + lane_off;
+        ptx::tmem_ld8(a, oh);
+        ptx::tmem_ld8(a + kHC, om);
+        ptx::tmem_ld8(a + 2 * kHC, ol);
+        ptx::tmem_wait_ld(oh, om);
+        ptx::reg_fence(ol);
+        const int dim = 128 * b + row;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {   // heads 4 q .. 4 q + 3
-          float x0 = z[4 * q] * sc[b], x1 = z[4 * q + 1] * sc[b];
-          float x2 = z[4 * q + 2] * sc[b], x3 = z[4 * q + 3] * sc[b];
-          const uint32_t h01 = split_e4m3x2(x0, x1), h23 = split_e4m3x2(x2, x3);
-          const uint32_t m01 = split_e4m3x2(x0, x1), m23 = split_e4m3x2(x2, x3);
-          wh[q] = h01 | (h23 << 16);
-          wm[q] = m01 | (m23 << 16);
-          wl[q] = f2_to_e4m3x2(x0, x1) | (f2_to_e4m3x2(x2, x3) << 16);
-        }
-        const uint32_t pb = ptx::smem_u32(S.pb[b]) + (row >> 3) * 384 + (row & 7) * 16;
-        st_shared_v4(pb, wh[0], wh[1], wh[2], wh[3]);
-        st_shared_v4(pb + 128, wm[0], wm[1], wm[2], wm[3]);
-        st_shared_v4(pb + 256, wl[0], wl[1], wl[2], wl[3]);
+        for (int h = 0; h < 8; ++h)
+          pout[(size_t)(8 * hh + h) * SML_LATENT_DIM + dim] =
+              (__uint_as_float(oh[h]) + __uint_as_float(om[h]) + __uint_as_float(ol[h])) * osc[h];
       }
-      ptx::fence_proxy_async();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&S.p_full);
+      if (lane == 0) ptx::mbar_arrive(&S.o_free);
     }
-    ok = softmax_all(ok && warp_wait(&S.pv_done, (ntiles - 1) & 1, abort));
     if (!ok) *abort = 1;
-    ptx::tc_fence_after();
-    // Row sums over the 128 key lanes, then each head's output scale
-    // sigma_h / l_h and its log-sum-exp.
-    column_reduce<false>(S, row, lrow);
-    if (row < kHC) {
-      const float lsum = S.hstat[row];
-      S.hosc[row] = lsum > 0.f ? S.hsig[row] / lsum : 0.f;
-      P.ws.part_lse[slot0 + (size_t)row * P.ws.splits] = lsum > 0.f ? S.hm[row] + logf(lsum) : -INFINITY;
-    }
-  }
-
-  // Output, sigma_h (hi + mid + lo) / l_h per head, by every warp but the MMA
-  // issuer (the gather warps are idle by now): unit (block b, TMEM lane
-  // quarter q) goes to a warp whose quarter is q.  The named barrier orders
-  // the last PV (the softmax warps waited for it) and S.hosc before the reads;
-  // every path of warps 0-14, a timed-out one included, reaches it.
-  if (warp != kWarpMma) {
-    asm volatile("bar.sync 3, %0;" ::"n"(32 * kWarpMma) : "memory");
-    ptx::tc_fence_after();
-    const int q = warp & 3;
-    const int nq = (kWarpMma - 1 - q) / 4 + 1;   // warps 0..14 with quarter q
-    float osc[kHC];
-#pragma unroll
-    for (int h = 0; h < kHC; ++h) osc[h] = S.hosc[h];
-#pragma unroll 1
-    for (int b = warp >> 2; b < 4; b += nq) {
-      uint32_t ov[32], ow[16];
-      ptx::tmem_ld32(T0 + kColO + kOStride * b + lane_off, ov);
-      ptx::tmem_ld16(T0 + kColO + kOStride * b + 32 + lane_off, ow);
-      ptx::tmem_wait_ld(ov, ow);
-      const int dim = 128 * b + 32 * q + lane;
-#pragma unroll
-      for (int h = 0; h < kHC; ++h) {
-        const float o = __uint_as_float(ov[h]) + __uint_as_float(ov[kHC + h]) + __uint_as_float(ow[h]);
-        P.ws.part_out[(slot0 + (size_t)h * P.ws.splits) * SML_LATENT_DIM + dim] = o * osc[h];
-      }
-    }
   }
 
   ptx::tc_fence_before();
@@ -697,24 +880,30 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_tc_kernel(const Params
   }
 }
 
-// out[t,h,:] = sum_s exp(lse_s - lse) O_s,  lse = ln sum_s exp(lse_s).
+// out[t,h,:] = sum_s exp(lse_s - lse) O_s,  lse = ln sum_s exp(lse_s), over
+// the partials of every CTA whose range touched (t, h's head group).
 __global__ void __launch_bounds__(128)
 lse_merge_kernel(int H, MlaWs ws, float* __restrict__ out, float* __restrict__ lse) {
-  const int h = blockIdx.x, t = blockIdx.y, S = ws.splits;
+  const int h = blockIdx.x, t = blockIdx.y;
   if (threadIdx.x == 0) ptx::griddep_launch_dependents();
   ptx::griddep_wait();   // the partials come from the previous kernel
-  const size_t base = ((size_t)t * H + h) * S;
+  const MlaPlan& m = ws.plan;
+  const int tg = t * m.hg + h / kHC, hl = h % kHC;
+  const long long u0 = (long long)tg * m.tpt;
+  const int n = cta_of(m, u0 + m.tpt - 1) - cta_of(m, u0) + 1;
+  const size_t base = (size_t)tg * m.smax;
   float mx = -INFINITY;
-  for (int s = 0; s < S; ++s) mx = fmaxf(mx, ws.part_lse[base + s]);
+  for (int s = 0; s < n; ++s) mx = fmaxf(mx, ws.part_lse[(base + s) * kHC + hl]);
   float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
   float den = 0.f;
   if (mx != -INFINITY) {
-    for (int s = 0; s < S; ++s) {
-      const float ls = ws.part_lse[base + s];
+    for (int s = 0; s < n; ++s) {
+      const float ls = ws.part_lse[(base + s) * kHC + hl];
       if (ls == -INFINITY) continue;
       const float w = expf(ls - mx);
       den += w;
-      const float4 v = reinterpret_cast<const float4*>(ws.part_out + (base + s) * SML_LATENT_DIM)[threadIdx.x];
+      const float4 v =
+          reinterpret_cast<const float4*>(ws.part_out + ((base + s) * kHC + hl) * SML_LATENT_DIM)[threadIdx.x];
       o.x = fmaf(w, v.x, o.x);
       o.y = fmaf(w, v.y, o.y);
       o.z = fmaf(w, v.z, o.z);
@@ -732,25 +921,25 @@ lse_merge_kernel(int H, MlaWs ws, float* __restrict__ out, float* __restrict__ l
 
 }  // namespace
 
-int mla_splits(const sml_problem& p, int* keys_per_split) {
-  // Splits of whole 128-key tiles, at most 512 keys: about one CTA per SM for
-  // the whole problem, so the per-CTA set-up is paid once per SM and the
-  // staging of a tile overlaps the math of the one before.
-  const int tiles = (p.topk + kKT - 1) / kKT;
-  const int ctas = p.num_tokens * (p.num_heads / kHC);
-  int tps = (int)(((long long)ctas * tiles + 148 - 1) / 148);
-  tps = tps < 1 ? 1 : (tps > kMaxSplit / kKT ? kMaxSplit / kKT : tps);
-  if (tps > tiles) tps = tiles;
-  const int kps = tps * kKT;
-  if (keys_per_split) *keys_per_split = kps;
-  return (p.topk + kps - 1) / kps;
+MlaPlan mla_plan(const sml_problem& p) {
+  MlaPlan m;
+  m.hg = p.num_heads / kHC;
+  m.tpt = (p.topk + kKT - 1) / kKT;
+  m.units = (long long)p.num_tokens * m.hg * m.tpt;
+  const int sms = device_sm_count();
+  m.ctas = (int)(m.units < sms ? m.units : sms);
+  // every CTA holds at least `per` units, so a run of tpt units touches at
+  // most 1 + ceil((tpt - 1) / per) CTAs
+  const long long per = m.units / m.ctas;
+  m.smax = (int)((m.tpt - 1 + per - 1) / per) + 1;
+  return m;
 }
 
 cudaError_t launch_sparse_mla(const sml_problem& p, const uint16_t* q, const sml_cache& latent,
                               const int32_t* idx, const int32_t* idx_len,
                               float* out, float* lse, const MlaWs& ws, int32_t* status,
                               cudaStream_t stream) {
-  if (latent.num_pages > (int64_t)(INT32_MAX / SML_PAGE_TOKENS)) return cudaErrorInvalidValue;
+  if (latent.num_pages > (int64_t)(INT32_MAX / SML_PAGE_TOKENS)) return cudaErrorInvalidValue;   // int32 row ids
   Params P;
   P.B = p.num_requests;
   P.T = p.num_tokens;
@@ -765,6 +954,8 @@ cudaError_t launch_sparse_mla(const sml_problem& p, const uint16_t* q, const sml
   P.cu_q = p.cu_q;
   P.ctx_len = p.ctx_len;
   P.block_table = p.block_table;
+  P.vis_len = p.vis_len;
+  P.ssmax_len = p.ssmax_len;
   P.q = q;
   P.latent = static_cast<const uint8_t*>(latent.base);
   P.latent_pages = latent.num_pages;
@@ -775,13 +966,13 @@ cudaError_t launch_sparse_mla(const sml_problem& p, const uint16_t* q, const sml
   P.ws = ws;
   P.status = status;
   const size_t smem = sizeof(Smem) + 1024;
-  auto kernel = plain ? sparse_mla_tc_kernel<true> : sparse_mla_tc_kernel<false>;
+  auto kernel = plain ? sparse_mla_kernel<true> : sparse_mla_kernel<false>;
   cudaError_t e = set_max_smem(reinterpret_cast<const void*>(kernel), smem);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(kernel, dim3(ws.splits, p.num_heads / kHC, p.num_tokens), dim3(kThreads), smem, stream, 0, P);
+  e = launch_pdl(kernel, dim3(ws.plan.ctas), dim3(kThreads), smem, stream, 0, P);
   if (e != cudaSuccess) return e;
-  return launch_pdl(lse_merge_kernel, dim3(p.num_heads, p.num_tokens), dim3(128), 0, stream, 0, p.num_heads, ws, out,
-                    lse);
+  return launch_pdl(lse_merge_kernel, dim3(p.num_heads, p.num_tokens), dim3(128), 0, stream, 0, p.num_heads, ws,
+                    out, lse);
 }
 
 }  // namespace sml

@@ -86,16 +86,16 @@ extern "C" int sml_sparse_mla_decode_noalloc(const sml_problem* p, const void* q
   MlaWs ws{};
   size_t need = 0;
   if (code == SML_OK) {
-    ws.splits = mla_splits(*p, &ws.keys_per_split);
-    const size_t slots = (size_t)p->num_tokens * p->num_heads * ws.splits;
+    ws.plan = mla_plan(*p);
+    const size_t slots = mla_slots(ws.plan, p->num_tokens) * 16;
     const size_t out_bytes = align_up(slots * SML_LATENT_DIM * sizeof(float));
     need = out_bytes + align_up(slots * sizeof(float));
     if (need > kNoallocScratchBytes) {
       char buf[200];
       snprintf(buf, sizeof buf,
-               "problem needs %zu bytes of split scratch (T=%d x H=%d x %d splits), the built-in "
+               "problem needs %zu bytes of split scratch (T=%d x H=%d x %d slots per 16 heads), the built-in "
                "scratch holds %zu; use sml_sparse_mla_decode with a workspace",
-               need, p->num_tokens, p->num_heads, ws.splits, kNoallocScratchBytes);
+               need, p->num_tokens, p->num_heads, ws.plan.smax, kNoallocScratchBytes);
       fail(SML_ERR_UNSUPPORTED, buf);
     }
   }
@@ -107,7 +107,7 @@ extern "C" int sml_sparse_mla_decode_noalloc(const sml_problem* p, const void* q
   cudaError_t e = device_addresses(&addr);
   if (e == cudaSuccess) {
     char* b = static_cast<char*>(addr.scratch);
-    const size_t slots = (size_t)p->num_tokens * p->num_heads * ws.splits;
+    const size_t slots = mla_slots(ws.plan, p->num_tokens) * 16;
     ws.part_out = reinterpret_cast<float*>(b);
     ws.part_lse = reinterpret_cast<float*>(b + align_up(slots * SML_LATENT_DIM * sizeof(float)));
     e = launch_sparse_mla(*p, static_cast<const uint16_t*>(q), latent, idx, idx_len, out, lse, ws, addr.status,

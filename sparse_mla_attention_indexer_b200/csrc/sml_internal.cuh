@@ -37,11 +37,25 @@ struct TopkWs {
   int chunks;          // ceil(max_ctx / kTopkChunk)
 };
 
+// Sparse MLA work split.  A unit is (query token, group of 16 heads, tile of
+// 128 selected keys); units are numbered token-major, then head group, then
+// tile, and a persistent grid of `ctas` CTAs takes equal contiguous ranges of
+// them.  A CTA writes one partial result (per head: output and LSE) for every
+// (token, head group) its range touches; a (token, head group) has at most
+// `smax` such CTAs, and its partials sit in slots [tg * smax, tg * smax + n)
+// in CTA order, n = the CTAs that touch it.
+struct MlaPlan {
+  int hg;              // head groups, H / 16
+  int tpt;             // tiles per (token, head group), ceil(topk / 128)
+  long long units;     // T * hg * tpt
+  int ctas;            // min(SMs, units)
+  int smax;            // slots per (token, head group)
+};
+
 struct MlaWs {
-  float* part_out;     // [T, H, S, 512]
-  float* part_lse;     // [T, H, S]
-  int splits;          // S
-  int keys_per_split;  // multiple of 64
+  float* part_out;     // [T * hg * smax * 16, 512]
+  float* part_lse;     // [T * hg * smax * 16]
+  MlaPlan plan;
 };
 
 // Message returned by sml_last_error() on this host thread.
@@ -50,7 +64,10 @@ void set_last_error(const std::string& msg);
 // Region sizes, in bytes (host).
 size_t topk_region_bytes(const sml_problem& p);
 size_t mla_region_bytes(const sml_problem& p);
-int mla_splits(const sml_problem& p, int* keys_per_split);
+// The plan of a problem on the current device (its SM count sets `ctas`).
+MlaPlan mla_plan(const sml_problem& p);
+// Partial slots of a plan (16 heads each): T * hg * smax.
+inline size_t mla_slots(const MlaPlan& m, int T) { return (size_t)T * m.hg * m.smax; }
 
 // ---- device helpers ---------------------------------------------------------------
 __device__ __forceinline__ void raise_fault(int32_t* status, int bits) {
@@ -86,9 +103,10 @@ __device__ __forceinline__ int request_of_warp(const int32_t* __restrict__ cu_q,
 }
 
 // Query range, context length and visible length of request r, checked against
-// the problem: 0 <= q0, Q >= 1, q0 + Q <= T, Q <= L <= max_ctx and
-// ceil(L / 64) <= max_pages.  Anything else is SML_FAULT_LENGTHS and the
-// request is skipped, so no index derived from it leaves its buffer.
+// the problem: 0 <= q0, Q >= 1, q0 + Q <= T, Q <= L <= max_ctx (0 <= L when
+// the visible lengths are given per token) and ceil(L / 64) <= max_pages.
+// Anything else is SML_FAULT_LENGTHS and the request is skipped, so no index
+// derived from it leaves its buffer.
 struct Req {
   int q0, Q, L;
   bool ok;
@@ -96,14 +114,33 @@ struct Req {
 
 __device__ __forceinline__ Req load_request(const int32_t* __restrict__ cu_q,
                                             const int32_t* __restrict__ ctx_len, int r, int T,
-                                            int max_ctx, int max_pages) {
+                                            int max_ctx, int max_pages, bool given_vis = false) {
   Req q;
   q.q0 = __ldg(cu_q + r);
   q.Q = __ldg(cu_q + r + 1) - q.q0;
   q.L = __ldg(ctx_len + r);
-  q.ok = q.q0 >= 0 && q.Q >= 1 && q.q0 <= T - q.Q && q.L >= q.Q && q.L <= max_ctx &&
+  q.ok = q.q0 >= 0 && q.Q >= 1 && q.q0 <= T - q.Q && q.L >= (given_vis ? 0 : q.Q) && q.L <= max_ctx &&
          (q.L + SML_PAGE_TOKENS - 1) / SML_PAGE_TOKENS <= max_pages;
   return q;
+}
+
+// n_t of query token t of request rq (rq.ok, t in its range): vis[t] when the
+// problem gives the visible lengths (clamped into [0, L]; a value outside it
+// is reported through *bad), else the causal rule L - Q + j + 1.
+__device__ __forceinline__ int visible_len(const int32_t* __restrict__ vis, const Req& rq, int t, bool* bad) {
+  if (!vis) return rq.L - rq.Q + (t - rq.q0) + 1;
+  const int n = __ldg(vis + t);
+  if (n < 0 || n > rq.L) {
+    *bad = true;
+    return n < 0 ? 0 : rq.L;
+  }
+  return n;
+}
+
+// The n of token t's SSMax factors: ssmax_len[t] (at least 1) when given, else n_t.
+__device__ __forceinline__ int ssmax_len_of(const int32_t* __restrict__ ssl, int t, int n) {
+  const int m = ssl ? __ldg(ssl + t) : n;
+  return m < 1 ? 1 : m;
 }
 
 // Host-side per-device caches for the launchers (thread-safe): the SM count,
@@ -157,6 +194,8 @@ cudaError_t launch_latent_write(const void* c, const void* kpe, const int32_t* s
                                 int32_t* status, cudaStream_t stream);
 cudaError_t launch_dcp_merge(const sml_dcp_ranks& rk, int T, int K, float* mscore, int32_t* mpos, int32_t* mlen,
                              int32_t* status, cudaStream_t stream);
+cudaError_t launch_dcp_pack(int T, int K, const float* scores, int64_t stride, const int32_t* idx,
+                            const int32_t* len, float* cand, int32_t* status, cudaStream_t stream);
 cudaError_t launch_dcp_split(int R, int I, int T, int K, const int32_t* sel, const int32_t* sel_len,
                              const int32_t* mpos, int32_t* const* local_idx, int32_t* const* local_len,
                              int32_t* status, cudaStream_t stream);

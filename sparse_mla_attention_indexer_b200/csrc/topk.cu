@@ -503,7 +503,7 @@ __device__ float row_floor(const float* row, int n, int k, SelectShared& sh) {
 
 __global__ void __launch_bounds__(kTopkThreads, 1)
 topk_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32_t* __restrict__ cu_q,
-            const int32_t* __restrict__ ctx_len, const float* __restrict__ scores,
+            const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ vis_len, const float* __restrict__ scores,
             int32_t* __restrict__ idx, int32_t* __restrict__ idx_len, TopkWs ws,
             int32_t* status) {
   extern __shared__ uint32_t skeys[];  // kTopkChunk keys
@@ -514,8 +514,8 @@ topk_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32_t* __re
   if (tid == 0) ptx::griddep_launch_dependents();
   ptx::griddep_wait();   // the scores come from the previous kernel
   const int r = request_of_warp(cu_q, B, t);
-  const Req rq = load_request(cu_q, ctx_len, r, T, max_ctx, max_pages);
-  const int q0 = rq.q0, Q = rq.Q, L = rq.L;
+  const Req rq = load_request(cu_q, ctx_len, r, T, max_ctx, max_pages, vis_len != nullptr);
+  const int q0 = rq.q0, Q = rq.Q;
   int32_t* out = idx + (size_t)t * K;
   if (!rq.ok || t < q0 || t - q0 >= Q) {
     if (c == 0) {
@@ -527,7 +527,16 @@ topk_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32_t* __re
     }
     return;
   }
-  const int n = L - Q + (t - q0) + 1;
+  bool bad_n = false;
+  const int n = visible_len(vis_len, rq, t, &bad_n);
+  if (bad_n && c == 0 && tid == 0) raise_fault(status, SML_FAULT_LENGTHS);
+  if (n == 0) {   // nothing visible: an empty selection
+    if (c == 0) {
+      for (int i = tid; i < K; i += nt) out[i] = -1;
+      if (tid == 0) idx_len[t] = 0;
+    }
+    return;
+  }
   const int nch = (n + kTopkChunk - 1) / kTopkChunk;
   if (c >= nch) return;
   const int c0 = c * kTopkChunk;
@@ -774,7 +783,8 @@ __device__ __forceinline__ void cluster_hist_sum(ClusterShared& S, int nb, int C
 
 __global__ void __launch_bounds__(kTopkThreads, 1)
 topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32_t* __restrict__ cu_q,
-                    const int32_t* __restrict__ ctx_len, const float* __restrict__ scores,
+                    const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ vis_len,
+                    const float* __restrict__ scores,
                     int32_t* __restrict__ idx, int32_t* __restrict__ idx_len, int32_t* status) {
   extern __shared__ __align__(16) uint8_t tk_smem[];
   uint32_t* keys = reinterpret_cast<uint32_t*>(tk_smem);
@@ -787,7 +797,7 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
   // Everything up to the first cluster barrier depends only on the row, so an
   // early return is taken by the whole cluster or by none of it.
   const int r = request_of_warp(cu_q, B, t);
-  const Req rq = load_request(cu_q, ctx_len, r, T, max_ctx, max_pages);
+  const Req rq = load_request(cu_q, ctx_len, r, T, max_ctx, max_pages, vis_len != nullptr);
   int32_t* out = idx + (size_t)t * K;
   if (!rq.ok || t < rq.q0 || t - rq.q0 >= rq.Q) {
     if (c == 0) {
@@ -799,7 +809,9 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
     }
     return;
   }
-  const int n = rq.L - rq.Q + (t - rq.q0) + 1;
+  bool bad_n = false;
+  const int n = visible_len(vis_len, rq, t, &bad_n);
+  if (bad_n && c == 0 && tid == 0) raise_fault(status, SML_FAULT_LENGTHS);
   if (n <= K) {
     if (c == 0) {
       for (int i = tid; i < K; i += nt) out[i] = i < n ? i : -1;
@@ -1202,16 +1214,16 @@ cudaError_t launch_topk(const sml_problem& p, const float* scores, int32_t* idx,
     cudaError_t e = set_max_smem(reinterpret_cast<const void*>(topk_cluster_kernel), smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(topk_cluster_kernel, dim3(ws.chunks, p.num_tokens), dim3(kTopkThreads), smem, stream, ws.chunks,
-                      p.num_requests, p.num_tokens, p.topk, p.max_ctx, p.max_pages, p.cu_q, p.ctx_len, scores, idx,
-                      idx_len, status);
+                      p.num_requests, p.num_tokens, p.topk, p.max_ctx, p.max_pages, p.cu_q, p.ctx_len, p.vis_len,
+                      scores, idx, idx_len, status);
   }
   // chunk keys, or (last CTA of a row) candidate keys, then segment starts
   const size_t smem = (size_t)kLevel2Keys * sizeof(uint32_t) + (kMaxSegChunks + 1) * sizeof(int);
   cudaError_t e = set_max_smem(reinterpret_cast<const void*>(topk_kernel), smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(topk_kernel, dim3(ws.chunks, p.num_tokens), dim3(kTopkThreads), smem, stream, 0, p.num_requests,
-                    p.num_tokens, p.topk, p.max_ctx, p.max_pages, p.cu_q, p.ctx_len, scores, idx, idx_len, ws,
-                    status);
+                    p.num_tokens, p.topk, p.max_ctx, p.max_pages, p.cu_q, p.ctx_len, p.vis_len, scores, idx, idx_len,
+                    ws, status);
 }
 
 }  // namespace sml

@@ -67,6 +67,8 @@ class Problem(ctypes.Structure):
         ("cu_q", ctypes.c_void_p),
         ("ctx_len", ctypes.c_void_p),
         ("block_table", ctypes.c_void_p),
+        ("vis_len", ctypes.c_void_p),
+        ("ssmax_len", ctypes.c_void_p),
     ]
 
 
@@ -83,7 +85,8 @@ class DcpRanks(ctypes.Structure):
                 ("scores", ctypes.c_void_p * SML_DCP_MAX_RANKS),
                 ("score_stride", ctypes.c_int64 * SML_DCP_MAX_RANKS),
                 ("idx", ctypes.c_void_p * SML_DCP_MAX_RANKS),
-                ("idx_len", ctypes.c_void_p * SML_DCP_MAX_RANKS)]
+                ("idx_len", ctypes.c_void_p * SML_DCP_MAX_RANKS),
+                ("packed", ctypes.c_int32)]
 
 
 class E4M3Latent(NamedTuple):
@@ -121,6 +124,7 @@ def lib() -> ctypes.CDLL:
         L.sml_indexer_q_quant.argtypes = [vp, ctypes.c_int32, vp, vp, vp]
         i32p = ctypes.c_int32
         L.sml_dcp_merge_candidates.argtypes = [ctypes.POINTER(DcpRanks), i32p, i32p, vp, vp, vp, vp, vp]
+        L.sml_dcp_pack_candidates.argtypes = [i32p, i32p, vp, ctypes.c_int64, vp, vp, vp, vp, vp]
         L.sml_dcp_split_selection.argtypes = [i32p, i32p, i32p, i32p, vp, vp, vp, ctypes.POINTER(vp),
                                               ctypes.POINTER(vp), vp, vp]
         L.sml_lse_combine.argtypes = [i32p, i32p, i32p, ctypes.POINTER(vp), ctypes.POINTER(vp), vp, vp, vp]
@@ -131,7 +135,8 @@ def lib() -> ctypes.CDLL:
                      "sml_sparse_mla_decode_noalloc", "sml_run_layer", "sml_read_device_status",
                      "sml_noalloc_read_status",
                      "sml_indexer_k_cache_write", "sml_latent_cache_write", "sml_indexer_q_quant",
-                     "sml_dcp_merge_candidates", "sml_dcp_split_selection", "sml_lse_combine"):
+                     "sml_dcp_merge_candidates", "sml_dcp_split_selection", "sml_lse_combine",
+                     "sml_dcp_pack_candidates"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -173,8 +178,11 @@ def _nbytes(t) -> int:
 
 
 def make_problem(*, num_heads, topk, rope_dim, cu_q, ctx_len, block_table, max_ctx=None,
-                 ssmax=False, sm_scale, ssmax_s=0.4, ssmax_s_index=0.4, num_tokens=None) -> Problem:
-    """Problem struct for device tensors cu_q [B+1], ctx_len [B], block_table [B, max_pages] (int32)."""
+                 ssmax=False, sm_scale, ssmax_s=0.4, ssmax_s_index=0.4, num_tokens=None,
+                 vis_len=None, ssmax_len=None) -> Problem:
+    """Problem struct for device tensors cu_q [B+1], ctx_len [B], block_table [B, max_pages]
+    (int32), and optionally vis_len [T] / ssmax_len [T] (int32 overrides of n_t and of the
+    SSMax n)."""
     B = ctx_len.numel()
     return Problem(num_requests=B,
                    num_tokens=int(num_tokens) if num_tokens is not None else int(cu_q[-1]),
@@ -183,7 +191,7 @@ def make_problem(*, num_heads, topk, rope_dim, cu_q, ctx_len, block_table, max_c
                    max_ctx=int(max_ctx) if max_ctx is not None else int(ctx_len.max()),
                    ssmax=int(bool(ssmax)), sm_scale=sm_scale, ssmax_s=ssmax_s,
                    ssmax_s_index=ssmax_s_index, cu_q=_p(cu_q), ctx_len=_p(ctx_len),
-                   block_table=_p(block_table))
+                   block_table=_p(block_table), vis_len=_p(vis_len), ssmax_len=_p(ssmax_len))
 
 
 def cache(pool, page_bytes: int) -> Cache:
@@ -279,13 +287,22 @@ def _ptrs(tensors):
     return arr
 
 
+def sml_dcp_pack_candidates(scores, idx, idx_len, cand_scores, workspace=None, stream=None):
+    """One rank's candidates for the exchange: cand_scores [T, topk] = scores at idx (NaN padding)."""
+    T, K = idx.shape
+    _check(lib().sml_dcp_pack_candidates(T, K, _p(scores), scores.shape[1], _p(idx), _p(idx_len),
+                                         _p(cand_scores), _p(workspace), _s(stream)))
+
+
 def sml_dcp_merge_candidates(scores, idx, idx_len, interleave, topk, merged_scores, merged_pos, merged_len,
-                             workspace=None, stream=None):
-    """Ranks' top-k results (lists of per-rank tensors: scores [T, stride_r],
-    idx [T, topk], idx_len [T]) -> candidates in global position order."""
+                             workspace=None, stream=None, packed=False):
+    """Ranks' top-k results (lists of per-rank tensors: scores [T, stride_r] -- or, packed,
+    [T, topk] from sml_dcp_pack_candidates -- idx [T, topk], idx_len [T]) -> candidates in
+    global position order."""
     rk = DcpRanks()
     rk.num_ranks = len(scores)
     rk.interleave = interleave
+    rk.packed = int(bool(packed))
     for r, (sc, ix, ln) in enumerate(zip(scores, idx, idx_len)):
         rk.scores[r] = _p(sc)
         rk.score_stride[r] = sc.shape[1]

@@ -92,3 +92,52 @@ def test_two_gloo_ranks_partition_the_batch():
         p.join(timeout=120)
     assert all(p.exitcode == 0 for p in procs)
     assert q.get(timeout=10) is True
+
+
+def test_rank_arrays_count_each_querys_visible_tokens_by_the_oracle_rule():
+    rng = np.random.default_rng(5)
+    ctx = np.array([1100, 9000, 4097, 700], dtype=np.int32)
+    qc = np.array([1, 4, 2, 3])
+    cu_q = np.concatenate([[0], np.cumsum(qc)]).astype(np.int32)
+    n = dcp.visible_lengths(cu_q, ctx)
+    for R, I in ((2, 64), (3, 64), (8, 128), (5, 192)):
+        tot = np.zeros_like(n)
+        for r in range(R):
+            local_len, vis, glob = dcp.rank_arrays(cu_q, ctx, r, R, I)
+            assert np.array_equal(glob, n)
+            for t in range(len(n)):
+                assert vis[t] == np.sum(odcp.owner(np.arange(n[t]), R, I) == r)   # brute force
+            for b, L in enumerate(ctx):
+                assert local_len[b] == np.sum(odcp.owner(np.arange(L), R, I) == r)
+            tot += vis
+        assert np.array_equal(tot, n)                                            # the ranks partition every query
+    assert rng is not None
+
+
+def _gather_main(rank, world, port, out_q):
+    import torch
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    t = torch.full((3, 5), float(rank)) + torch.arange(5.0)
+    got = dcp._all_gather(t)
+    out_q.put((rank, [x.numpy() for x in got]))
+    dist.destroy_process_group()
+
+
+def test_exchange_gathers_every_ranks_array_in_rank_order():
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_gather_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank in range(2):
+        for src in range(2):
+            assert np.array_equal(res[rank][src], np.full((3, 5), float(src)) + np.arange(5.0))
