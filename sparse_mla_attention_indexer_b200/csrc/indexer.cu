@@ -365,7 +365,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
       }
       if (*abort) {
         // Let copies already issued land before the CTA's shared memory goes away.
-        for (int i = 0; i < kStages; ++i) ptx::mbar_wait(&S.full[i], phase ^ (i >= stage ? 1u : 0u), nullptr, 1u << 16);
+        for (int i = 0; i < kStages; ++i) ptx::mbar_wait(&S.full[i], phase ^ (i >= stage ? 1u : 0u), nullptr, 100000u);
       }
     }
     __syncwarp();
@@ -411,7 +411,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     if (lane == 0) {
       // Every MMA this thread issued has finished before TMEM is released.
       ptx::mma_commit(&S.drain);
-      ptx::mbar_wait(&S.drain, 0, nullptr, 1u << 20);
+      ptx::mbar_wait(&S.drain, 0, nullptr, 100000u);
     }
     __syncwarp();
   } else {

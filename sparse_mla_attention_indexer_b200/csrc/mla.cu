@@ -14,38 +14,42 @@
 // with c_hat_i = e4m3 latent x its 128-element block scale.
 //
 // Work: a unit is (query token, group of 16 heads, tile of 128 selected keys).
-// One persistent CTA per SM takes an equal contiguous range of the units
-// (token-major), so every SM holds the same number of tiles whatever the
-// batch; where its range crosses a (token, head group) boundary it writes one
-// partial result per (token, head group), and a merge kernel combines the
-// partials by their LSE.  Keys are the MMA M dimension of QK^T and the K
-// dimension of PV, the 16 heads N (16 heads as M would waste 3/4 of the
-// smallest M); both products run on kind::f8f6f4 straight from the gathered
-// E4M3 tile: the latent is never converted.
-//   * warps 9-23 fill the two tile buffers: they turn the tile's selected
+// Persistent CTAs take equal contiguous ranges of the units (token-major), as
+// few CTAs as give the same longest range; where a range crosses a (token,
+// head group) boundary the CTA writes one partial result per (token, head
+// group), and a merge kernel combines the partials by their LSE.  Keys are
+// the MMA M dimension of QK^T and the K dimension of PV, the 16 heads N (16
+// heads as M would waste 3/4 of the smallest M); both products run on
+// kind::f8f6f4 straight from the gathered E4M3 tile: the latent is never
+// converted.
+//   * warps 17-31 fill the two tile buffers: they turn the tile's selected
 //     positions into pool rows (block table, bounds checks), then copy the
 //     rows with 16-B cp.async straight into place, 128-B-swizzled, a masked
 //     row as zeros; the copies arrive on the buffer's barrier by themselves,
 //     so the loaders go on to the next tile at once.  (Random 656-B rows are
 //     bound by the requests in flight per SM: measured on B200, cp.async
-//     from many warps reaches about 20 GB/s per SM whatever the shared-memory
-//     size, while register loads lose a quarter of that rate when the
-//     kernel's shared memory leaves L1 small, and TMA tile::gather4 reaches
-//     about half of it.);
-//   * warp 8 issues the MMAs (one thread):
+//     reaches about 20 GB/s per SM whatever the shared-memory size and the
+//     number of SMs gathering, while register loads lose a quarter of that
+//     rate when the kernel's shared memory leaves L1 small, and TMA
+//     tile::gather4 reaches about half of it.);
+//   * warp 16 issues the MMAs (one thread):
 //       S_b^T = C_b . [Qhi_b; Qlo_b]^T   (K-major; N = 32: both query terms),
 //       S_pe^T = K_pe . Q_pe^T           (bf16; plain E4M3: both terms),
 //       O_b^T += C_b^T . [Bhi_b; Bmid_b; Blo_b]^T  (C_b^T read MN-major from
 //       the same tile; N = 48: the three weight terms),
 //     each as soon as its inputs are ready: a tile's PV (which frees its
 //     buffer) does not wait for the next tile's QK^T, nor the reverse;
-//   * warps 0-7 (two per TMEM lane quarter: keys 32q..32q+31, heads 8 hh..
-//     8 hh + 7) stage each (token, head group)'s query, run the softmax on
-//     S^T and build the weights B_b[i, h] = p_ih scale_ib / sigma_h as three
-//     E4M3 terms whose sum carries 12 significant bits; sigma_h is a per-head
-//     power of two that keeps the terms in range, raised (and O rescaled,
-//     exactly) only when a tile would overflow; at the end of a (token, head
-//     group) they read O^T back and write its partial output and LSE.
+//   * warps 0-15 (four per TMEM lane quarter: keys 32q..32q+31, heads
+//     4 hq .. 4 hq + 3) run the softmax on S^T and build the weights
+//     B_b[i, h] = 2^(z_ih - M_h) scale_ib as three E4M3 terms whose sum
+//     carries 12 significant bits; M_h is a per-head integer exponent that
+//     keeps every weight at most 440, raised (and O rescaled, exactly) only
+//     when a tile would exceed that; at the end of a (token, head group) they
+//     read O^T back and write its partial output and LSE.  Warps 0-7 also
+//     stage each (token, head group)'s query.  The softmax is split over
+//     sixteen warps so that a tile's weights are ready well within the time
+//     the next tile's rows take to arrive: the tile buffer is then free again
+//     before the loaders need it.
 // The query is split exactly into two E4M3 terms sharing a power-of-two scale
 // per head; products of E4M3 values are exact and accumulate in fp32.
 // Every wait is bounded; a wait that gives up sets SML_FAULT_TIMEOUT and the
@@ -63,23 +67,31 @@ namespace {
 
 constexpr int kHC = 16;          // heads per unit
 constexpr int kKT = 128;         // keys per tile
-constexpr int kSoftmaxThreads = 256;   // warps 0-7
-constexpr int kWarpMma = 8;
-constexpr int kWarpLoad = 9;           // warps 9-23 copy the rows
+constexpr int kSoftmaxWarps = 16;      // warps 0-15
+constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
+constexpr int kStageWarps = 8;         // warps 0-7 stage the query (thread = head x 32-dim part)
+constexpr int kWarpMma = 16;
+constexpr int kWarpLoad = 17;          // warps 17-31 copy the rows
 constexpr int kLoadWarps = 15;
 constexpr int kLoadThreads = 32 * kLoadWarps;
-constexpr int kThreads = 32 * (kWarpLoad + kLoadWarps);   // 768: six warpgroups
-// Registers: the kernel launches with kRegsLaunch per thread; the two softmax
+constexpr int kThreads = 32 * (kWarpLoad + kLoadWarps);   // 1024: eight warpgroups
+static_assert(kLoadThreads >= kKT, "one loader thread per key of a tile looks up its pool row");
+// Registers: the kernel launches with kRegsLaunch per thread; the four softmax
 // warpgroups then raise theirs to kRegsSoftmax and the other four (MMA and
 // loaders) lower theirs to kRegsOther.  setmaxnreg.inc draws on what the
 // block launched with, so the shares must add up to it exactly.
-constexpr int kRegsLaunch = 80, kRegsSoftmax = 112, kRegsOther = 64;
-static_assert(kThreads * kRegsLaunch == 256 * kRegsSoftmax + (kThreads - 256) * kRegsOther,
+constexpr int kRegsLaunch = 64, kRegsSoftmax = 80, kRegsOther = 48;
+static_assert(kThreads * kRegsLaunch == kSoftmaxThreads * kRegsSoftmax + (kThreads - kSoftmaxThreads) * kRegsOther,
               "warpgroup register shares must add up to the launch allocation");
-static_assert(kThreads % 128 == 0 && kWarpMma == 8, "roles are whole warpgroups: 0-1 softmax, 2-5 the rest");
+static_assert(kThreads % 128 == 0 && kSoftmaxThreads % 128 == 0 && kWarpMma == kSoftmaxWarps,
+              "roles are whole warpgroups: 0-3 softmax, 4-7 the rest");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kLazyRescale = 8.f * kLog2e;   // 8 nats, in the log2 units the softmax runs in
+// Weight exponents: a key's weights are capped at 440 (E4M3's largest value
+// is 448; the margin covers the approximate 2^x and log2); an exponent that
+// has to move puts the tile's largest possible weight in (56, 112].
+constexpr float kLog2Cap = 8.78135971f;    // log2(440)
+constexpr float kLog2Head = 6.80735492f;   // log2(112)
 
 // TMEM columns
 constexpr uint32_t kColS = 0;       // S_b^T (lanes = keys): 32 columns per block b (hi | lo query term)
@@ -96,8 +108,8 @@ struct __align__(1024) Smem {
   uint8_t qpe[2 * kHC * 128];    // RoPE query, SW128: bf16 rows 0-15; plain E4M3: rows 0-15 high, 16-31 low
   uint8_t pb[4][kPBytes];        // weight terms of block b, MN-major 8-key x 16-B core matrices
   float sc[2][kKT][4];            // [buffer][key] the four block scales of the staged row
-  float xmax[2][2][4][12];       // [tile parity][head half][key quarter]: 8 head maxima, largest scale
-  float xsum[2][4][8];           // [head half][key quarter][head]: row-sum exchange
+  float xmax[2][4][4][8];        // [tile parity][head quarter][key quarter]: 4 head maxima, largest scale
+  float xsum[4][4][4];           // [head quarter][key quarter][head]: row-sum exchange
   float qs[kHC];                 // power-of-two query scale per head
   int32_t rowid[4][kKT];         // [tile % 4] pool row of each key, -1 = masked
   uint64_t full[2], lat_free[2];
@@ -185,26 +197,26 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, ok);
 }
 
-// AND of a flag over the 256 softmax threads (named barrier 3).  Every wait
+// AND of a flag over the softmax threads (named barrier 5).  Every wait
 // outcome reaches this before the next named barrier of the softmax warps, so
-// a wait that gave up ends all eight warps together instead of leaving some
+// a wait that gave up ends all of them together instead of leaving some
 // blocked at a barrier.
 __device__ __forceinline__ bool softmax_all(bool ok) {
   uint32_t r;
   asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 3, 256, p;\n selp.u32 %0, 1, 0, q;\n}"
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 5, %2, p;\n selp.u32 %0, 1, 0, q;\n}"
       : "=r"(r)
-      : "r"((uint32_t)ok)
+      : "r"((uint32_t)ok), "n"(kSoftmaxThreads)
       : "memory");
   return r != 0;
 }
 
-// AND of a flag over the loader threads (named barrier 4); also orders their
+// AND of a flag over the loader threads (named barrier 6); also orders their
 // shared-memory writes before it against reads after it.
 __device__ __forceinline__ bool loader_all(bool ok) {
   uint32_t r;
   asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 4, %2, p;\n selp.u32 %0, 1, 0, q;\n}"
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 6, %2, p;\n selp.u32 %0, 1, 0, q;\n}"
       : "=r"(r)
       : "r"((uint32_t)ok), "n"(kLoadThreads)
       : "memory");
@@ -218,11 +230,26 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// The four warps of one head half (named barrier 1 + half).
-__device__ __forceinline__ void half_sync(int half) {
-  if (half == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
-  else asm volatile("bar.sync 2, 128;" ::: "memory");
+// OR of a flag over the four warps of one head quarter (named barrier 1 +
+// quarter; also a barrier for them).
+__device__ __forceinline__ bool group_any(int hq, bool v) {
+  uint32_t r;
+  asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, 128, p;\n selp.u32 %0, 1, 0, q;\n}"
+               : "=r"(r)
+               : "r"((uint32_t)v), "r"(1 + hq)
+               : "memory");
+  return r != 0;
 }
+
+// log2(x) (the hardware approximation), x > 0.
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// The four warps of one head quarter (named barrier 1 + quarter).
+__device__ __forceinline__ void group_sync(int hq) { asm volatile("bar.sync %0, 128;" ::"r"(1 + hq) : "memory"); }
 
 __device__ __forceinline__ long long unit_begin(const MlaPlan& m, int c) { return m.units * c / m.ctas; }
 // The CTA whose range holds unit u.
@@ -241,7 +268,7 @@ struct Seg {
 };
 
 // Warp-collective (the request lookup is a 32-way search).
-__device__ Seg segment_at(const Params& P, long long u, long long e) {
+__device__ __forceinline__ Seg segment_at(const Params& P, long long u, long long e) {
   const MlaPlan& m = P.ws.plan;
   Seg s;
   s.tg = (int)(u / m.tpt);
@@ -257,6 +284,9 @@ __device__ Seg segment_at(const Params& P, long long u, long long e) {
   s.n = s.req_ok ? visible_len(P.vis_len, rq, s.t, &bad_n) : 0;
   s.req_ok = s.req_ok && !bad_n;
   s.nss = ssmax_len_of(P.ssmax_len, s.t, s.n);
+  // Everything above reads inputs no kernel of this library writes; the
+  // selection comes from the previous kernel (a no-op after the first call).
+  ptx::griddep_wait();
   const int len = s.req_ok ? __ldg(P.idx_len + s.t) : 0;
   const int len_max = min(P.K, s.n);
   s.len_bad = len < 0 || len > len_max;
@@ -272,16 +302,17 @@ __device__ Seg segment_at(const Params& P, long long u, long long e) {
 // k-th tile overall.  Warp-collective, like segment_at.
 struct Cur {
   long long u;   // the unit after segment s
-  Seg s;
+  int ne;        // segment s's non-empty tiles
   int jj, seg, k;
   bool valid;
 };
 
 __device__ __forceinline__ void cur_seek(Cur& c, const Params& P, long long ue) {
   while (c.u < ue) {
-    c.s = segment_at(P, c.u, ue);
-    c.u += c.s.nj;
-    if (c.s.ne > 0) {
+    const Seg s = segment_at(P, c.u, ue);
+    c.u += s.nj;
+    c.ne = s.ne;
+    if (s.ne > 0) {
       c.jj = 0;
       c.valid = true;
       return;
@@ -299,7 +330,7 @@ __device__ __forceinline__ void cur_start(Cur& c, const Params& P, long long ub,
 
 __device__ __forceinline__ void cur_next(Cur& c, const Params& P, long long ue) {
   ++c.k;
-  if (++c.jj < c.s.ne) return;
+  if (++c.jj < c.ne) return;
   ++c.seg;
   cur_seek(c, P, ue);
 }
@@ -379,7 +410,7 @@ __device__ __forceinline__ void stage_query(const Params& P, Smem& S, int t, int
 // fp8_ds_mla.  A template parameter, so that each path is compiled for its
 // own row layout.
 template <bool kPlain>
-__global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const Params P) {
+__global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_constant__ Params P) {
   extern __shared__ uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -392,12 +423,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const Params P)
       ptx::mbar_init(&S.full[i], kLoadThreads + 1);
       ptx::mbar_init(&S.lat_free[i], 1);   // PV of the tile done (its last reader)
     }
-    ptx::mbar_init(&S.q_ready, 8);
+    ptx::mbar_init(&S.q_ready, kStageWarps);
     ptx::mbar_init(&S.s_full, 1);
-    ptx::mbar_init(&S.s_free, 8);
-    ptx::mbar_init(&S.p_full, 8);
+    ptx::mbar_init(&S.s_free, kSoftmaxWarps);
+    ptx::mbar_init(&S.p_full, kSoftmaxWarps);
     ptx::mbar_init(&S.pv_done, 1);
-    ptx::mbar_init(&S.o_free, 8);
+    ptx::mbar_init(&S.o_free, kSoftmaxWarps);
     ptx::mbar_init(&S.drain, 1);
     S.abort = 0;
     ptx::fence_mbar_init();
@@ -410,9 +441,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const Params P)
   __syncthreads();
   ptx::tc_fence_after();
   // This CTA holds its tensor memory now, so a dependent grid scheduled on the
-  // same SM cannot starve it of columns.
+  // same SM cannot starve it of columns.  Each thread waits for the previous
+  // kernel (the selection) just before its first read of idx_len (in
+  // segment_at): the request lookups and the first query overlap that kernel.
   if (threadIdx.x == 0) ptx::griddep_launch_dependents();
-  ptx::griddep_wait();   // the selection comes from the previous kernel
   volatile int* abort = &S.abort;
   const uint32_t T0 = S.tmem_base;
 
@@ -594,26 +626,38 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const Params P)
       if (!ok) *abort = 1;
       // every MMA this thread issued has finished before TMEM is released
       ptx::mma_commit(&S.drain);
-      ptx::mbar_wait(&S.drain, 0, nullptr, 1u << 20);
+      ptx::mbar_wait(&S.drain, 0, nullptr, 100000u);
     }
     __syncwarp();
   } else {
-    // ================= softmax: warps 0-7 =================
+    // ================= softmax: warps 0-15 =================
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-    const int q4 = warp & 3, hh = warp >> 2;   // TMEM lane quarter (keys / dims), head half
+    // TMEM lane quarter (keys, and latent dims in the epilogue) and head
+    // quarter: this thread owns key (or dim) `row` for heads 4 hq .. 4 hq + 3.
+    const int q4 = warp & 3, hq = warp >> 2;
     const int row = 32 * q4 + lane;
-    const int tid = threadIdx.x;                // 0 .. 255
+    const int tid = threadIdx.x;                // 0 .. 511
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-    // The query of a (token, head group) is staged, and q_ready signalled,
-    // before the epilogue of the non-empty one before it: the MMA issues the
-    // first QK^T of the next before the last PV of the current, and that PV
-    // is what the epilogue waits for.
-    auto stage = [&](const Seg& s) {
-      stage_query<kPlain>(P, S, s.t, s.g, tid);
-      ptx::fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&S.q_ready);
+    // The query of a (token, head group) is staged (by warps 0-7), and
+    // q_ready signalled, before the epilogue of the non-empty one before it:
+    // the MMA issues the first QK^T of the next before the last PV of the
+    // current, and that PV is what the epilogue waits for.
+    auto signal_query = [&]() {
+      if (warp < kStageWarps) {
+        ptx::fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&S.q_ready);
+      }
     };
+    auto stage = [&](const Seg& s) {
+      if (warp < kStageWarps) stage_query<kPlain>(P, S, s.t, s.g, tid);
+      signal_query();
+    };
+    // The query of the range's first (token, head group) is an input, not
+    // the selection: staged before the previous kernel has finished, and
+    // signalled once that (token, head group) turns out to hold keys.
+    long long pre_tg = ub / plan.tpt;
+    if (warp < kStageWarps) stage_query<kPlain>(P, S, (int)(pre_tg / plan.hg), (int)(pre_tg % plan.hg), tid);
     int k = 0;
     bool ok = true, staged = false;
     for (long long u = ub; u < ue;) {
@@ -630,22 +674,25 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const Params P)
         if (tid < kHC) plse[tid] = -INFINITY;
         continue;
       }
-      if (!staged) stage(s);
+      if (!staged) {
+        if (s.tg == pre_tg) signal_query();
+        else stage(s);
+      }
+      pre_tg = -1;
       staged = false;
       ok = softmax_all(ok);   // S.qs visible to every softmax thread
-      float qsh[8];
+      float qsh[4];
 #pragma unroll
-      for (int h = 0; h < 8; ++h) qsh[h] = S.qs[8 * hh + h];
-      // logits in log2 units: z log2(e), so that p = 2^(z - m)
+      for (int h = 0; h < 4; ++h) qsh[h] = S.qs[4 * hq + h];
+      // logits in log2 units: z log2(e), so that p = 2^(z - M)
       const float zscale = P.sm_scale * (P.ssmax ? P.ssmax_s * logf((float)s.nss) : 1.f) * kLog2e;
-      // per head of this half (identical in all its threads): running max m,
-      // weight scale sigma (0 = not set yet), and this key row's row-sum share
-      float m[8], sig[8], isig[8], lrow[8];
+      // Per head of this quarter (identical in all its threads): the integer
+      // exponent M_h the weights are taken against (-inf until the head's
+      // first key), and this key row's share of the row sum, in units of 2^M_h.
+      float M[4], lrow[4];
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        m[h] = -INFINITY;
-        sig[h] = 0.f;
-        isig[h] = 0.f;
+      for (int h = 0; h < 4; ++h) {
+        M[h] = -INFINITY;
         lrow[h] = 0.f;
       }
       for (int jj = 0; jj < s.ne; ++jj, ++k) {
@@ -656,108 +703,101 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const Params P)
         if (!ok) break;
         ptx::tc_fence_after();
         const bool valid = S.rowid[k & 3][row] >= 0;
-        float sc[4];
-        if (kPlain) {
-#pragma unroll
-          for (int b = 0; b < 4; ++b) sc[b] = valid ? P.latent_scale : 0.f;
-        } else {
-          const float4 v4 = *reinterpret_cast<const float4*>(&S.sc[buf][row][0]);
-          sc[0] = v4.x;
-          sc[1] = v4.y;
-          sc[2] = v4.z;
-          sc[3] = v4.w;
-        }
+        // this key's block scales (plain pool: one scale, 0 for a masked key)
+        const float* scr = &S.sc[buf][row][0];
+        const float psc = valid ? P.latent_scale : 0.f;
         // z = zscale * (s_h * sum_b scale_b (S_b,hi + S_b,lo) + S_pe), fp32
-        float z[8];
-#pragma unroll
-        for (int h = 0; h < 8; ++h) z[h] = 0.f;
+        float z[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
-          uint32_t vh[8], vl[8];
-          ptx::tmem_ld8(T0 + kColS + 32 * b + 8 * hh + lane_off, vh);
-          ptx::tmem_ld8(T0 + kColS + 32 * b + kHC + 8 * hh + lane_off, vl);
+          uint32_t vh[4], vl[4];
+          ptx::tmem_ld4(T0 + kColS + 32 * b + 4 * hq + lane_off, vh);
+          ptx::tmem_ld4(T0 + kColS + 32 * b + kHC + 4 * hq + lane_off, vl);
           ptx::tmem_wait_ld(vh, vl);
+          const float scb = kPlain ? psc : scr[b];
 #pragma unroll
-          for (int h = 0; h < 8; ++h) z[h] = fmaf(sc[b], __uint_as_float(vh[h]) + __uint_as_float(vl[h]), z[h]);
+          for (int h = 0; h < 4; ++h) z[h] = fmaf(scb, __uint_as_float(vh[h]) + __uint_as_float(vl[h]), z[h]);
         }
 #pragma unroll
-        for (int h = 0; h < 8; ++h) z[h] *= qsh[h];
+        for (int h = 0; h < 4; ++h) z[h] *= qsh[h];
         if (P.rope_dim) {
           if (kPlain) {
             // RoPE codes under the pool scale, both query terms
-            uint32_t vh[8], vl[8];
-            ptx::tmem_ld8(T0 + kColSpe + 8 * hh + lane_off, vh);
-            ptx::tmem_ld8(T0 + kColSpe + kHC + 8 * hh + lane_off, vl);
+            uint32_t vh[4], vl[4];
+            ptx::tmem_ld4(T0 + kColSpe + 4 * hq + lane_off, vh);
+            ptx::tmem_ld4(T0 + kColSpe + kHC + 4 * hq + lane_off, vl);
             ptx::tmem_wait_ld(vh, vl);
 #pragma unroll
-            for (int h = 0; h < 8; ++h)
+            for (int h = 0; h < 4; ++h)
               z[h] = fmaf(qsh[h] * P.latent_scale, __uint_as_float(vh[h]) + __uint_as_float(vl[h]), z[h]);
           } else {
-            uint32_t v[8];
-            ptx::tmem_ld8(T0 + kColSpe + 8 * hh + lane_off, v);
+            uint32_t v[4];
+            ptx::tmem_ld4(T0 + kColSpe + 4 * hq + lane_off, v);
             ptx::tmem_wait_ld(v);
 #pragma unroll
-            for (int h = 0; h < 8; ++h) z[h] += __uint_as_float(v[h]);
+            for (int h = 0; h < 4; ++h) z[h] += __uint_as_float(v[h]);
           }
         }
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&S.s_free);   // S read: the next tile's QK^T may overwrite it
 #pragma unroll
-        for (int h = 0; h < 8; ++h) z[h] = valid ? z[h] * zscale : -INFINITY;
-        // Tile statistics: each head's maximum over the 128 keys, and the
-        // tile's largest block scale (masked rows were zero-filled: scale 0).
-        {
-          float* xm = S.xmax[k & 1][hh][q4];
+        for (int h = 0; h < 4; ++h) z[h] = valid ? z[h] * zscale : -INFINITY;
+        // This key's weights x_b = 2^(z - M_h) scale_b must stay within
+        // E4M3's 448: with this key's largest scale, each head's bound is
+        // 2^(z - M_h + lk).  A bound above the cap, or a head without M_h yet,
+        // sends the quarter's four warps through the exact update (a vote:
+        // after the first tile it is rare, so most tiles exchange nothing
+        // between warps here).
+        const float kmax = kPlain ? psc : fmaxf(fmaxf(scr[0], scr[1]), fmaxf(scr[2], scr[3]));
+        const float lk = kmax > 0.f ? lg2(kmax) : -INFINITY;
+        bool need = false;
 #pragma unroll
-          for (int h = 0; h < 8; ++h) {
+        for (int h = 0; h < 4; ++h) need = need || (z[h] != -INFINITY && !(z[h] - M[h] + lk <= kLog2Cap));
+        need = group_any(hq, need);
+        float f[4] = {1.f, 1.f, 1.f, 1.f};
+        bool any = false;
+        if (need) {
+          // Exact tile statistics: each head's largest logit over the 128
+          // keys and the tile's largest block scale (masked rows: scale 0).
+          float* xm = S.xmax[k & 1][hq][q4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
             const float w = ptx::warp_max_f32(z[h]);
             if (lane == 0) xm[h] = w;
           }
-          const float scw = ptx::warp_max_f32(fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])));
-          if (lane == 0) xm[8] = scw;
-        }
-        half_sync(hh);
-        float tm[8], SC = 0.f;
+          const float scw = ptx::warp_max_f32(kmax);
+          if (lane == 0) xm[4] = scw;
+          group_sync(hq);
+          float tm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY}, SC = 0.f;
 #pragma unroll
-        for (int h = 0; h < 8; ++h) tm[h] = -INFINITY;
+          for (int qq = 0; qq < 4; ++qq) {
+            const float* x = S.xmax[k & 1][hq][qq];
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          const float* xm = S.xmax[k & 1][hh][qq];
-#pragma unroll
-          for (int h = 0; h < 8; ++h) tm[h] = fmaxf(tm[h], xm[h]);
-          SC = fmaxf(SC, xm[8]);
-        }
-        // Lazily raised running max m_h and weight scale sigma_h.  The tile's
-        // weights are at most 2^(tmax_h - m_h) * SC and must stay <= 448
-        // sigma_h; sigma_h is reset to the power of two just above U_h / 448
-        // (U_h below, with a margin for the approximate 2^x) whenever U_h
-        // leaves [28, 448] sigma_h, so the dominant weights keep all 12 bits
-        // of the three-term split.  O holds sum(weights / sigma), so both
-        // changes rescale it by f_h = 2^(m_old - m_new) * sigma_old /
-        // sigma_new (exact for the sigma part: powers of two).
-        float f[8];
-        bool any = false;
-#pragma unroll
-        for (int h = 0; h < 8; ++h) {
-          float alpha = 1.f;
-          if (tm[h] > m[h] + kLazyRescale || (m[h] == -INFINITY && tm[h] != -INFINITY)) {
-            alpha = ex2(m[h] - tm[h]);   // 0 when m was -inf
-            m[h] = tm[h];
+            for (int h = 0; h < 4; ++h) tm[h] = fmaxf(tm[h], x[h]);
+            SC = fmaxf(SC, x[4]);
           }
-          const float U = tm[h] == -INFINITY ? 0.f : fmaxf(ex2(tm[h] - m[h]) * 1.001f, 1.f) * SC;
-          float beta = 1.f;
-          if (U > 0.f && (U > 448.f * sig[h] || U < 28.f * sig[h])) {
-            // U / 448 in [2^(E - 127), 2^(E - 126)): sigma = 2^(E - 126), 1 / sigma = 2^(126 - E)
-            const uint32_t E = (__float_as_uint(U * (1.f / 448.f)) >> 23) & 0xffu;
-            const float ns = __uint_as_float((E + 1u) << 23), nis = __uint_as_float((253u - E) << 23);
-            beta = sig[h] > 0.f ? sig[h] * nis : 1.f;
-            sig[h] = ns;
-            isig[h] = nis;
+          // A head whose bound 2^(tmax_h - M_h) SC exceeds the cap (or that
+          // has no M_h) takes the integer M_h that puts it in (56, 112]: 4x
+          // headroom for later tiles, and the dominant weights keep all 12
+          // bits of the three-term split (a weight of at least 4 does).  M_h
+          // is never lowered.  O and the row sums scale by f_h =
+          // 2^(M_old - M_new), exactly.
+          const float lsc = SC > 0.f ? lg2(SC) : -INFINITY;
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const float e = tm[h] + lsc;
+            if (tm[h] != -INFINITY && !(e - M[h] <= kLog2Cap)) {
+              const float Mn = ceilf(e - kLog2Head);
+              if (M[h] != -INFINITY) {
+                const float d = M[h] - Mn;   // a negative integer
+                f[h] = d < -126.f ? 0.f : __int_as_float((127 + (int)d) << 23);
+                lrow[h] *= f[h];
+                any = true;
+              }
+              M[h] = Mn;
+            }
           }
-          f[h] = alpha * beta;
-          any = any || f[h] != 1.f;
-          lrow[h] *= alpha;
         }
         // The previous tile's PV reads the weight tiles and accumulates into
         // O: wait for it before rescaling O or overwriting the weights (the
@@ -772,44 +812,41 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const Params P)
           ptx::tc_fence_after();
           if (any) {
 #pragma unroll 1
-            for (int b = 0; b < 4; ++b) {   // this thread: latent dim 128 b + row, this half's heads
+            for (int b = 0; b < 4; ++b) {   // this thread: latent dim 128 b + row, this quarter's heads
+              uint32_t ov[3][4];
+              const uint32_t a = T0 + kColO + kOStride * b + 4 * hq + lane_off;
+#pragma unroll
+              for (int term = 0; term < 3; ++term) ptx::tmem_ld4(a + kHC * term, ov[term]);
+              ptx::tmem_wait_ld(ov[0], ov[1]);
+              ptx::reg_fence(ov[2]);
 #pragma unroll
               for (int term = 0; term < 3; ++term) {
-                uint32_t ov[8];
-                const uint32_t a = T0 + kColO + kOStride * b + kHC * term + 8 * hh + lane_off;
-                ptx::tmem_ld8(a, ov);
-                ptx::tmem_wait_ld(ov);
 #pragma unroll
-                for (int h = 0; h < 8; ++h) ov[h] = __float_as_uint(__uint_as_float(ov[h]) * f[h]);
-                ptx::tmem_st8(a, ov);
+                for (int h = 0; h < 4; ++h) ov[term][h] = __float_as_uint(__uint_as_float(ov[term][h]) * f[h]);
+                ptx::tmem_st4(a + kHC * term, ov[term]);
               }
             }
             ptx::tmem_wait_st();
           }
         }
-        // p = 2^(z - m) (0 for a masked key); weights x = p * scale_b / sigma as hi + mid + lo (E4M3)
+        // p = 2^(z - M) (0 for a masked key); weights x = p * scale_b as hi + mid + lo (E4M3)
 #pragma unroll
-        for (int h = 0; h < 8; ++h) {
-          const float p = z[h] == -INFINITY ? 0.f : ex2(z[h] - m[h]);
+        for (int h = 0; h < 4; ++h) {
+          const float p = z[h] == -INFINITY ? 0.f : ex2(z[h] - M[h]);
           lrow[h] += p;
-          z[h] = p * isig[h];
+          z[h] = p;
         }
+        const uint32_t pb_off = (row >> 3) * 384 + (row & 7) * 16 + 4 * hq;
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
-          uint32_t wh[2], wm[2], wl[2];
-#pragma unroll
-          for (int qq = 0; qq < 2; ++qq) {   // heads 4 qq .. 4 qq + 3 of this half
-            uint32_t h01, m01, l01, h23, m23, l23;
-            split3_e4m3x2(z[4 * qq] * sc[b], z[4 * qq + 1] * sc[b], h01, m01, l01);
-            split3_e4m3x2(z[4 * qq + 2] * sc[b], z[4 * qq + 3] * sc[b], h23, m23, l23);
-            wh[qq] = h01 | (h23 << 16);
-            wm[qq] = m01 | (m23 << 16);
-            wl[qq] = l01 | (l23 << 16);
-          }
-          const uint32_t pb = ptx::smem_u32(S.pb[b]) + (row >> 3) * 384 + (row & 7) * 16 + 8 * hh;
-          st_shared_v2(pb, wh[0], wh[1]);
-          st_shared_v2(pb + 128, wm[0], wm[1]);
-          st_shared_v2(pb + 256, wl[0], wl[1]);
+          const float scb = kPlain ? psc : scr[b];
+          uint32_t h01, m01, l01, h23, m23, l23;
+          split3_e4m3x2(z[0] * scb, z[1] * scb, h01, m01, l01);
+          split3_e4m3x2(z[2] * scb, z[3] * scb, h23, m23, l23);
+          const uint32_t pb = ptx::smem_u32(S.pb[b]) + pb_off;
+          st_shared_b32(pb, h01 | (h23 << 16));
+          st_shared_b32(pb + 128, m01 | (m23 << 16));
+          st_shared_b32(pb + 256, l01 | (l23 << 16));
         }
         ptx::fence_proxy_async();
         ptx::tc_fence_before();
@@ -832,37 +869,36 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const Params P)
       ok = softmax_all(ok);
       if (!ok) break;
       ptx::tc_fence_after();
-      // row sums over the 128 keys (four warps of this half)
+      // row sums over the 128 keys (the quarter's four warps)
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
+      for (int h = 0; h < 4; ++h) {
         float v = lrow[h];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) S.xsum[hh][q4][h] = v;
+        if (lane == 0) S.xsum[hq][q4][h] = v;
       }
-      half_sync(hh);
-      float osc[8];
+      group_sync(hq);
+      float osc[4];
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        const float l = S.xsum[hh][0][h] + S.xsum[hh][1][h] + S.xsum[hh][2][h] + S.xsum[hh][3][h];
-        osc[h] = l > 0.f ? sig[h] / l : 0.f;
-        if (q4 == 0 && lane == h) plse[8 * hh + h] = l > 0.f ? (m[h] + log2f(l)) * kLn2 : -INFINITY;
+      for (int h = 0; h < 4; ++h) {
+        const float l = S.xsum[hq][0][h] + S.xsum[hq][1][h] + S.xsum[hq][2][h] + S.xsum[hq][3][h];
+        osc[h] = l > 0.f ? 1.f / l : 0.f;
+        if (q4 == 0 && lane == h) plse[4 * hq + h] = l > 0.f ? (M[h] + log2f(l)) * kLn2 : -INFINITY;
       }
-      // out = sigma_h (hi + mid + lo) / l_h: this thread's latent dim 128 b + row
+      // out = (hi + mid + lo) / l_h: this thread's latent dim 128 b + row
 #pragma unroll 1
       for (int b = 0; b < 4; ++b) {
-        uint32_t oh[8], om[8], ol[8];
-        const uint32_t a = T0 + kColO + kOStride * b + 8 * hh + lane_off;
-        ptx::tmem_ld8(a, oh);
-        ptx::tmem_ld8(a + kHC, om);
-        ptx::tmem_ld8(a + 2 * kHC, ol);
-        ptx::tmem_wait_ld(oh, om);
-        ptx::reg_fence(ol);
+        uint32_t o3[3][4];
+        const uint32_t a = T0 + kColO + kOStride * b + 4 * hq + lane_off;
+#pragma unroll
+        for (int term = 0; term < 3; ++term) ptx::tmem_ld4(a + kHC * term, o3[term]);
+        ptx::tmem_wait_ld(o3[0], o3[1]);
+        ptx::reg_fence(o3[2]);
         const int dim = 128 * b + row;
 #pragma unroll
-        for (int h = 0; h < 8; ++h)
-          pout[(size_t)(8 * hh + h) * SML_LATENT_DIM + dim] =
-              (__uint_as_float(oh[h]) + __uint_as_float(om[h]) + __uint_as_float(ol[h])) * osc[h];
+        for (int h = 0; h < 4; ++h)
+          pout[(size_t)(4 * hq + h) * SML_LATENT_DIM + dim] =
+              (__uint_as_float(o3[0][h]) + __uint_as_float(o3[1][h]) + __uint_as_float(o3[2][h])) * osc[h];
       }
       ptx::tc_fence_before();
       __syncwarp();
@@ -870,7 +906,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const Params P)
     }
     if (!ok) *abort = 1;
   }
-
   ptx::tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && S.abort) raise_fault(P.status, SML_FAULT_TIMEOUT);
@@ -880,41 +915,56 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const Params P)
   }
 }
 
+static_assert(SML_MAX_TOPK / kKT + 1 <= 32, "a (token, head group) has at most one partial per lane");
+
 // out[t,h,:] = sum_s exp(lse_s - lse) O_s,  lse = ln sum_s exp(lse_s), over
-// the partials of every CTA whose range touched (t, h's head group).
+// the partials of every CTA whose range touched (t, h's head group).  One
+// block per (head, token); every warp works out the partials' weights (lane s
+// holds partial s, at most 32 of them), then each thread gathers its four
+// dims of all partials with the loads issued four partials at a time.
 __global__ void __launch_bounds__(128)
 lse_merge_kernel(int H, MlaWs ws, float* __restrict__ out, float* __restrict__ lse) {
-  const int h = blockIdx.x, t = blockIdx.y;
+  const int h = blockIdx.x, t = blockIdx.y, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) ptx::griddep_launch_dependents();
   ptx::griddep_wait();   // the partials come from the previous kernel
   const MlaPlan& m = ws.plan;
   const int tg = t * m.hg + h / kHC, hl = h % kHC;
   const long long u0 = (long long)tg * m.tpt;
-  const int n = cta_of(m, u0 + m.tpt - 1) - cta_of(m, u0) + 1;
+  const int n = cta_of(m, u0 + m.tpt - 1) - cta_of(m, u0) + 1;   // <= tiles per token + 1 <= 32
   const size_t base = (size_t)tg * m.smax;
-  float mx = -INFINITY;
-  for (int s = 0; s < n; ++s) mx = fmaxf(mx, ws.part_lse[(base + s) * kHC + hl]);
+  const float ls = lane < n ? __ldcg(ws.part_lse + (base + lane) * kHC + hl) : -INFINITY;
+  float mx = ls;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const float w = (mx == -INFINITY || ls == -INFINITY) ? 0.f : expf(ls - mx);
+  float den = w;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  const float4* po = reinterpret_cast<const float4*>(ws.part_out + (base * kHC + hl) * SML_LATENT_DIM) + threadIdx.x;
+  const size_t pstride = (size_t)kHC * SML_LATENT_DIM / 4;   // float4s from one partial to the next
   float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-  float den = 0.f;
-  if (mx != -INFINITY) {
-    for (int s = 0; s < n; ++s) {
-      const float ls = ws.part_lse[(base + s) * kHC + hl];
-      if (ls == -INFINITY) continue;
-      const float w = expf(ls - mx);
-      den += w;
-      const float4 v =
-          reinterpret_cast<const float4*>(ws.part_out + ((base + s) * kHC + hl) * SML_LATENT_DIM)[threadIdx.x];
-      o.x = fmaf(w, v.x, o.x);
-      o.y = fmaf(w, v.y, o.y);
-      o.z = fmaf(w, v.z, o.z);
-      o.w = fmaf(w, v.w, o.w);
+  for (int s0 = 0; s0 < n; s0 += 4) {
+    float4 v[4];
+    float ws4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ws4[i] = __shfl_sync(0xffffffffu, w, (s0 + i) & 31);
+      v[i] = (s0 + i < n && ws4[i] != 0.f) ? __ldcg(po + (size_t)(s0 + i) * pstride) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    const float inv = 1.f / den;
-    o.x *= inv;
-    o.y *= inv;
-    o.z *= inv;
-    o.w *= inv;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float wi = s0 + i < n ? ws4[i] : 0.f;
+      o.x = fmaf(wi, v[i].x, o.x);
+      o.y = fmaf(wi, v[i].y, o.y);
+      o.z = fmaf(wi, v[i].z, o.z);
+      o.w = fmaf(wi, v[i].w, o.w);
+    }
   }
+  o.x *= inv;
+  o.y *= inv;
+  o.z *= inv;
+  o.w *= inv;
   reinterpret_cast<float4*>(out + ((size_t)t * H + h) * SML_LATENT_DIM)[threadIdx.x] = o;
   if (threadIdx.x == 0) lse[(size_t)t * H + h] = den > 0.f ? mx + logf(den) : -INFINITY;
 }
@@ -926,8 +976,17 @@ MlaPlan mla_plan(const sml_problem& p) {
   m.hg = p.num_heads / kHC;
   m.tpt = (p.topk + kKT - 1) / kKT;
   m.units = (long long)p.num_tokens * m.hg * m.tpt;
-  const int sms = device_sm_count();
-  m.ctas = (int)(m.units < sms ? m.units : sms);
+  // As few CTAs as give the same longest range: ceil(units / SMs) units per
+  // CTA at most.  (On decode, all SMs gathering at once only adds contention
+  // at the memory for the same finishing time.)
+  if (m.units < 1) {
+    m.ctas = 0;
+    m.smax = 1;
+    return m;
+  }
+  const long long sms = device_sm_count();
+  const long long most = (m.units + sms - 1) / sms;
+  m.ctas = (int)((m.units + most - 1) / most);
   // every CTA holds at least `per` units, so a run of tpt units touches at
   // most 1 + ceil((tpt - 1) / per) CTAs
   const long long per = m.units / m.ctas;
