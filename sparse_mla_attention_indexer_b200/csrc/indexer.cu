@@ -40,12 +40,13 @@ constexpr int kQRowsBytes = SML_INDEX_HEADS * SML_INDEX_DIM;      // 8,192 per q
 
 // Two shapes of the same kernel:
 //   general: 9-stage ring, query groups of up to 4 tokens (N <= 256), two
-//            256-column accumulators, two epilogue warpgroups, one CTA per SM;
+//            256-column accumulators, four epilogue warpgroups (one per query
+//            of the group, all on every item), one CTA per SM;
 //   decode (every request has one query token): 5-stage ring, one-token groups
 //            (N = 64), four 64-column accumulators, one epilogue warpgroup, and
 //            half the shared memory and TMEM, so two CTAs share each SM and
 //            keep twice the loads in flight.
-template <int kStages_, int kGroup_, int kAccBufs_, int kEpiGroups_, int kCtasPerSm_>
+template <int kStages_, int kGroup_, int kAccBufs_, int kEpiGroups_, int kCtasPerSm_, bool kQueryPerWg_>
 struct Cfg {
   static constexpr int kStages = kStages_;
   static constexpr int kGroup = kGroup_;          // query tokens per group: N = 64 * Qg
@@ -55,9 +56,13 @@ struct Cfg {
   static constexpr int kEpiGroups = kEpiGroups_;  // epilogue warpgroups, taking alternate items
   static constexpr int kThreads = 64 + 128 * kEpiGroups_;   // warp 0 TMA, warp 1 MMA, then the epilogue
   static constexpr int kCtasPerSm = kCtasPerSm_;
+  // true: epilogue warpgroup g takes query g of every item (kEpiGroups ==
+  // kGroup); false: the warpgroups take alternate items, all their queries.
+  static constexpr bool kQueryPerWg = kQueryPerWg_;
+  static_assert(!kQueryPerWg_ || kEpiGroups_ == kGroup_, "one epilogue warpgroup per query of a group");
 };
-using CfgGeneral = Cfg<9, 4, 2, 2, 1>;
-using CfgDecode = Cfg<5, 1, 4, 1, 2>;
+using CfgGeneral = Cfg<9, 4, 2, 4, 1, true>;
+using CfgDecode = Cfg<5, 1, 4, 1, 2, false>;
 
 template <class C>
 struct __align__(1024) Smem {
@@ -65,9 +70,12 @@ struct __align__(1024) Smem {
   uint8_t keys[kStages][2 * kPageKeyBytes];      // [stage][128 rows x 128 B], SW128
   uint8_t q[2][kGroup * kQRowsBytes];            // [buffer][256 rows x 128 B], SW128
   float ksc[kStages][kTile];
-  float w[kEpiGroups][kGroup * SML_INDEX_HEADS]; // per epilogue warpgroup: head weights of the group
-  float qf[kEpiGroups][kGroup];                  // per epilogue warpgroup: sq_t * c_t per query
-  int nv[kEpiGroups][kGroup];                    // per epilogue warpgroup: n_t per query
+  // per epilogue warpgroup: head weights, sq_t * c_t and n_t of its queries
+  // (the whole group, or its one query of the group when kQueryPerWg)
+  static constexpr int kWgQueries = C::kQueryPerWg ? 1 : kGroup;
+  __align__(16) float w[kEpiGroups][kWgQueries * SML_INDEX_HEADS];
+  float qf[kEpiGroups][kWgQueries];
+  int nv[kEpiGroups][kWgQueries];
   uint64_t full[kStages], empty[kStages];
   uint64_t qfull[2], qempty[2];
   uint64_t accfull[C::kAccBufs], accempty[C::kAccBufs];
@@ -279,7 +287,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       ptx::mbar_init(&S.full[i], 1);
-      ptx::mbar_init(&S.empty[i], 1 + 4);   // MMA commit + one arrive per epilogue warp
+      // MMA commit + one arrive per epilogue warp that reads the stage
+      ptx::mbar_init(&S.empty[i], 1 + (C::kQueryPerWg ? 4 * kEpiGroups : 4));
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&S.qfull[i], 1);
@@ -287,7 +296,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     }
     for (int i = 0; i < kAccBufs; ++i) {
       ptx::mbar_init(&S.accfull[i], 1);
-      ptx::mbar_init(&S.accempty[i], 4);   // the owning warpgroup's 4 warps
+      ptx::mbar_init(&S.accempty[i], C::kQueryPerWg ? 4 * kEpiGroups : 4);   // the warps that read it
     }
     ptx::mbar_init(&S.drain, 1);
     S.abort = 0;
@@ -416,11 +425,14 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     __syncwarp();
   } else {
     // ---------------- epilogue: kEpiGroups warpgroups, one thread per token row ----------------
-    // Warpgroup eg takes the items with ordinal (it - beg) = eg mod kEpiGroups.
+    // kQueryPerWg: warpgroup eg takes query eg of every item.  Otherwise
+    // warpgroup eg takes the items with ordinal (it - beg) = eg mod kEpiGroups,
+    // all the group's queries.
     const int eg = (warp - 2) >> 2;
     const int quarter = warp & 3;               // TMEM lanes 32 * quarter .. + 31
     const int row = quarter * 32 + lane;
     const int et = threadIdx.x - 64 - 128 * eg; // 0..127 within the warpgroup
+    constexpr int kWq = Smem<C>::kWgQueries;
     float* wsm = S.w[eg];
     float* qfs = S.qf[eg];
     int* nvs = S.nv[eg];
@@ -429,18 +441,20 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     int last_r = -1, last_g = -1;
     for (int it = beg; it < end; ++it, w.advance()) {
       const int j_it = it - beg;
-      if (j_it % kEpiGroups != eg) continue;
+      if (!C::kQueryPerWg && j_it % kEpiGroups != eg) continue;
       const int stage = j_it % kStages, acc = j_it % kAccBufs;
       const uint32_t phase = (j_it / kStages) & 1, accphase = (j_it / kAccBufs) & 1;
       const int qg = w.qg();
       const int j0 = kGroup * w.g;
+      // this warpgroup's queries of the group: [jb, jb + jn)
+      const int jb = C::kQueryPerWg ? eg : 0;
+      const int jn = C::kQueryPerWg ? (eg < qg ? 1 : 0) : qg;
       if (w.r != last_r || w.g != last_g) {
-        if (eg == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
-        else asm volatile("bar.sync 2, 128;" ::: "memory");
-        for (int i = et; i < qg * SML_INDEX_HEADS; i += 128)
-          wsm[i] = __ldg(P.iw + (size_t)(w.rq.q0 + j0) * SML_INDEX_HEADS + i);
-        if (et < qg) {
-          const int t = w.rq.q0 + j0 + et;
+        asm volatile("bar.sync %0, 128;" ::"r"(1 + eg) : "memory");
+        for (int i = et; i < jn * SML_INDEX_HEADS; i += 128)
+          wsm[i] = __ldg(P.iw + (size_t)(w.rq.q0 + j0 + jb) * SML_INDEX_HEADS + i);
+        if (et < jn) {
+          const int t = w.rq.q0 + j0 + jb + et;
           bool bad = false;
           const int n = visible_len(P.vis_len, w.rq, t, &bad);
           if (bad) raise_fault(P.status, SML_FAULT_LENGTHS);
@@ -448,8 +462,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
           qfs[et] = __ldg(P.iq_scale + t) * c;
           nvs[et] = n;
         }
-        if (eg == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
-        else asm volatile("bar.sync 2, 128;" ::: "memory");
+        asm volatile("bar.sync %0, 128;" ::"r"(1 + eg) : "memory");
         last_r = w.r;
         last_g = w.g;
       }
@@ -460,19 +473,27 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
       const bool row_ok = (S.valid[stage] >> (row >> 6)) & 1;
       const int s = w.tile * kTile + row;
       const uint32_t tbase = S.tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * C::kAccCols;
-      for (int j = 0; j < qg; ++j) {
+      for (int jj = 0; jj < jn && jj < kWq; ++jj) {
+        const int j = jb + jj;
         uint32_t v0[32], v1[32];
         ptx::tmem_ld32(tbase + j * SML_INDEX_HEADS, v0);
         ptx::tmem_ld32(tbase + j * SML_INDEX_HEADS + 32, v1);
         ptx::tmem_wait_ld(v0, v1);
-        const float* wj = wsm + j * SML_INDEX_HEADS;
+        const float4* wj = reinterpret_cast<const float4*>(wsm + jj * SML_INDEX_HEADS);
         float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          s0 = fmaf(wj[i], fmaxf(__uint_as_float(v0[i]), 0.f), s0);
-          s1 = fmaf(wj[32 + i], fmaxf(__uint_as_float(v1[i]), 0.f), s1);
+        for (int i = 0; i < 8; ++i) {
+          const float4 wa = wj[i], wb = wj[8 + i];
+          s0 = fmaf(wa.x, fmaxf(__uint_as_float(v0[4 * i]), 0.f), s0);
+          s0 = fmaf(wa.y, fmaxf(__uint_as_float(v0[4 * i + 1]), 0.f), s0);
+          s0 = fmaf(wa.z, fmaxf(__uint_as_float(v0[4 * i + 2]), 0.f), s0);
+          s0 = fmaf(wa.w, fmaxf(__uint_as_float(v0[4 * i + 3]), 0.f), s0);
+          s1 = fmaf(wb.x, fmaxf(__uint_as_float(v1[4 * i]), 0.f), s1);
+          s1 = fmaf(wb.y, fmaxf(__uint_as_float(v1[4 * i + 1]), 0.f), s1);
+          s1 = fmaf(wb.z, fmaxf(__uint_as_float(v1[4 * i + 2]), 0.f), s1);
+          s1 = fmaf(wb.w, fmaxf(__uint_as_float(v1[4 * i + 3]), 0.f), s1);
         }
-        if (row_ok && s < nvs[j]) P.scores[(size_t)(w.rq.q0 + j0 + j) * P.max_ctx + s] = (s0 + s1) * qfs[j] * sk;
+        if (row_ok && s < nvs[jj]) P.scores[(size_t)(w.rq.q0 + j0 + j) * P.max_ctx + s] = (s0 + s1) * qfs[jj] * sk;
       }
       ptx::tc_fence_before();
       __syncwarp();
