@@ -48,7 +48,7 @@ FLUSH_BYTES = 256 << 20
 # dram__bytes_read.sum + dram__bytes_write.sum of one indexer launch on this
 # workload, from the ncu capture summarised in profiles/ (None = not captured
 # for the current kernel).
-INDEXER_NCU_TRAFFIC_BYTES = None
+INDEXER_NCU_TRAFFIC_BYTES = 162_776_320
 # The same for one sparse-MLA launch (the merge not included); None once the
 # kernel has changed since the counters were taken.
 MLA_NCU_TRAFFIC_BYTES = 51_166_976
@@ -341,16 +341,21 @@ def time_e2e(step: Step, steps: int, warmup: int, flush):
     return float(np.mean(e2e_ms)), h_in.numel(), h_out.numel()
 
 
-def time_plain_pool(step: Step, steps: int, warmup: int, flush):
-    """The same attention over a plain per-tensor E4M3 latent pool (576-B
-    rows) with the same block table and selection: one graph of the MLA call."""
+def time_other_pool(step: Step, steps: int, warmup: int, flush, fmt: str):
+    """The same attention over another latent format ("e4m3": the plain
+    per-tensor E4M3 pool, 576-B rows; "bf16": 1,152-B rows) with the same block
+    table and selection: one graph of the MLA call."""
     dw, wl = step.dw, step.wl
     p = dw.problem(0)
     lay = dw.layers[0]
     idx, ln, out, lse = step.outs[0]
     stream = torch.cuda.current_stream()
-    plain = torch.from_numpy(synth.plain_pool(0, wl.name + "/plain_pool", wl.num_pages)).cuda()
-    lat_plain = sml.E4M3Latent(plain, synth.PLAIN_SCALE)
+    if fmt == "e4m3":
+        pool = torch.from_numpy(synth.plain_pool(0, wl.name + "/plain_pool", wl.num_pages)).cuda()
+        lat_plain = sml.E4M3Latent(pool, synth.PLAIN_SCALE)
+    else:
+        pool = torch.from_numpy(synth.bf16_pool(0, wl.name + "/bf16_pool", wl.num_pages)).cuda()
+        lat_plain = sml.Bf16Latent(pool)
     g = torch.cuda.CUDAGraph()
     sml.sml_sparse_mla_decode(p, lay.q, lat_plain, idx, ln, out, lse, step.ws, stream)
     torch.cuda.synchronize()
@@ -610,7 +615,8 @@ def main():
     with ClockSampler(torch.cuda.current_device()) as clocks:
         step_ms, stage_ms = time_step(step, args.steps, args.warmup, flush)
         e2e_ms, h2d, d2h = time_e2e(step, args.steps, args.warmup, flush)
-        plain_ms = time_plain_pool(step, args.steps, args.warmup, flush)
+        plain_ms = time_other_pool(step, args.steps, args.warmup, flush, "e4m3")
+        bf16_ms = time_other_pool(step, args.steps, args.warmup, flush, "bf16")
         reports[wl.name] = workload_report(wl, step, step_ms, stage_ms, pk)
         del step
         # the other workloads, each its own step (every rank alike)
@@ -660,6 +666,9 @@ def main():
         "latent_e4m3_576": {"sparse_mla_and_merge_ms": plain_ms,
                             "hbm_gbs": units["gathered"] * 576 / (plain_ms / 1e3) / 1e9,
                             "note": "the same selection over a plain per-tensor E4M3 latent pool (576-B rows)"},
+        "latent_bf16_1152": {"sparse_mla_and_merge_ms": bf16_ms,
+                             "hbm_gbs": units["gathered"] * 1152 / (bf16_ms / 1e3) / 1e9,
+                             "note": "the same selection over a bf16 latent pool (1,152-B rows, one tile buffer)"},
     }
     print(json.dumps(line))
 

@@ -134,11 +134,20 @@ typedef struct sml_problem {
  * takes 0).  SML_LATENT_E4M3 is the plain per-tensor E4M3 cache of the blog's
  * section "ROCm 实现细节", paragraph "FP8 潜在缓存": all 576 latent dims in FP8
  * under one per-tensor scale, 576 B per token.  Reading: a row is
- * [512 x e4m3 latent][64 x e4m3 RoPE key], value = code * scale. */
+ * [512 x e4m3 latent][64 x e4m3 RoPE key], value = code * scale.
+ * SML_LATENT_BF16 is the unquantised cache the same paragraph compares with,
+ * 1,152 B per token: a row is [512 x bf16 latent][64 x bf16 RoPE key],
+ * little-endian (sml_cache.scale is ignored).  Sparse MLA over it runs bf16 x
+ * bf16 products with fp32 accumulation and bf16 weights split in two terms
+ * (16 significant bits); its 128-key tile fills one shared-memory buffer, so
+ * its row copies do not overlap the tile's products as the E4M3 formats' do. */
 #define SML_LATENT_FP8_DS_MLA 0
 #define SML_LATENT_E4M3 1
 #define SML_LATENT_E4M3_ROW_BYTES 576
 #define SML_LATENT_E4M3_PAGE_BYTES (SML_PAGE_TOKENS * SML_LATENT_E4M3_ROW_BYTES)
+#define SML_LATENT_BF16 2
+#define SML_LATENT_BF16_ROW_BYTES 1152
+#define SML_LATENT_BF16_PAGE_BYTES (SML_PAGE_TOKENS * SML_LATENT_BF16_ROW_BYTES)
 
 /* A paged cache pool: num_pages pages starting at base (256-B aligned).  A
  * zero-initialised descriptor (format 0) is the fp8_ds_mla latent layout or
@@ -193,10 +202,11 @@ int sml_topk(const sml_problem* p, const float* scores, int32_t* idx, int32_t* i
  * selected set S_t = idx[t, 0:idx_len[t]):
  *   z_i = sm_scale * c_t * (q[t,h,0:512] . c_hat_i + q[t,h,512:576] . k_pe_i)
  *   out[t,h,:] = sum_i softmax(z)_i * c_hat_i,  lse[t,h] = ln sum_i exp(z_i)
- * with c_hat_i = e4m3 latent * its block scale, c_t = ssmax_s * ln(n_t) when
+ * with c_hat_i = e4m3 latent * its block scale (SML_LATENT_E4M3: code * the
+ * pool scale; SML_LATENT_BF16: the bf16 value), c_t = ssmax_s * ln(n_t) when
  * ssmax, else 1.  rope_dim = 0 (NoPE) drops the k_pe term.
  *   q        [T, H, 512 + rope_dim] bf16
- *   latent   pool of SML_LATENT_PAGE_BYTES pages
+ *   latent   pool of pages of its format's page size
  *   idx      [T, topk] int32 logical positions (any order; -1 padding ignored)
  *   idx_len  [T] int32 number of valid entries at the front of each idx row
  *   out      [T, H, 512] fp32;  lse [T, H] fp32 (natural log; -inf if empty)
@@ -208,9 +218,11 @@ int sml_topk(const sml_problem* p, const float* scores, int32_t* idx, int32_t* i
  * bf16 has 8 significant bits, hi takes 4, lo the other 4); smaller elements
  * keep an absolute error below 2^-10 s_h (half of E4M3's subnormal step).
  * The RoPE part (fp8_ds_mla) runs as bf16 x bf16.  The softmax is fp32; each
- * weight p_i * block scale is split into three E4M3 terms whose sum carries
- * 12 significant bits, under a per-head power-of-two scale that keeps the
- * dominant weights in E4M3's normal range. */
+ * weight 2^(z_i - M_h) * block scale is split into three E4M3 terms whose sum
+ * carries 12 significant bits, with M_h a per-head integer exponent that keeps
+ * every weight at most 440 and the dominant ones at or above 4 (in E4M3's
+ * normal range).  A SML_LATENT_BF16 pool runs bf16 x bf16 products instead,
+ * with the bf16 query as given and each weight split into two bf16 terms. */
 int sml_sparse_mla_decode(const sml_problem* p, const void* q, sml_cache latent,
                           const int32_t* idx, const int32_t* idx_len, float* out, float* lse,
                           void* workspace, size_t ws_bytes, void* stream);
@@ -287,7 +299,9 @@ int sml_indexer_k_cache_write(const void* k, const int32_t* slot, int32_t n, sml
  * k_pe NULL for a NoPE layer, whose rows get a zero RoPE key).  By the pool's
  * format: SML_LATENT_FP8_DS_MLA -> the 656-B row at page*41984 + row*656:
  * [512 e4m3][4 fp32 block scales][64 bf16 k_pe]; SML_LATENT_E4M3 -> the 576-B
- * row at page*36864 + row*576: the codes of every value / latent.scale. */
+ * row at page*36864 + row*576: the codes of every value / latent.scale;
+ * SML_LATENT_BF16 -> the 1,152-B row at page*73728 + row*1152: the values as
+ * given (c, then k_pe). */
 int sml_latent_cache_write(const void* c, const void* k_pe, const int32_t* slot, int32_t n,
                            sml_cache latent, void* workspace, void* stream);
 

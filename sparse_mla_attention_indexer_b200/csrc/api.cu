@@ -84,7 +84,7 @@ void check_cache(Checker& c, sml_cache cache, const char* what, bool latent) {
   } else if (cache.format == SML_LATENT_E4M3) {
     if (!(isfinite(cache.scale) && cache.scale > 0.f))
       c.fail(SML_ERR_INVALID_ARG, (w + ".scale not finite and positive").c_str());
-  } else if (cache.format != SML_LATENT_FP8_DS_MLA) {
+  } else if (cache.format != SML_LATENT_FP8_DS_MLA && cache.format != SML_LATENT_BF16) {
     c.fail(SML_ERR_UNSUPPORTED, (w + ".format not an SML_LATENT_* format").c_str());
   }
 }

@@ -14,10 +14,13 @@
 // with c_hat_i = e4m3 latent x its 128-element block scale.
 //
 // Work: a unit is (query token, group of 16 heads, tile of 128 selected keys).
-// Persistent CTAs take equal contiguous ranges of the units (token-major), as
-// few CTAs as give the same longest range; where a range crosses a (token,
-// head group) boundary the CTA writes one partial result per (token, head
-// group), and a merge kernel combines the partials by their LSE.  Keys are
+// Each CTA serves one head group (blockIdx.x % groups) and takes an equal
+// contiguous range of that group's (token, tile) units, token-major, as few
+// CTAs per group as give the same longest range; the CTAs of the different
+// groups with the same blockIdx.x / groups walk the same tokens' tiles at the
+// same time, so a row gathered for one group is still in L2 for the others.
+// Where a range crosses a token boundary the CTA writes one partial result
+// per (token, head group), and a merge kernel combines them by their LSE.  Keys are
 // the MMA M dimension of QK^T and the K dimension of PV, the 16 heads N (16
 // heads as M would waste 3/4 of the smallest M); both products run on
 // kind::f8f6f4 straight from the gathered E4M3 tile: the latent is never
@@ -92,6 +95,9 @@ constexpr float kLn2 = 0.6931471805599453f;
 // has to move puts the tile's largest possible weight in (56, 112].
 constexpr float kLog2Cap = 8.78135971f;    // log2(440)
 constexpr float kLog2Head = 6.80735492f;   // log2(112)
+// bf16 weights have fp32's range: the exponent only keeps 2^(z - M_h) within
+// 2^16 (a raise sets M_h at the tile's largest logit).
+constexpr float kBfLog2Cap = 16.f;
 
 // TMEM columns
 constexpr uint32_t kColS = 0;       // S_b^T (lanes = keys): 32 columns per block b (hi | lo query term)
@@ -101,18 +107,36 @@ constexpr uint32_t kOStride = 64;   // ... at kColO + kOStride b
 constexpr int kPBytes = kKT * 3 * kHC;   // one block's weight terms: 128 keys x 48 E4M3
 constexpr int kLatBlock = kKT * 128;     // one 128-dim latent block of a tile
 
+// Latent formats of the kernel's template parameter.
+constexpr int kFmtDsMla = 0, kFmtPlain = 1, kFmtBf16 = 2;
+// Tile buffers and 128-B latent blocks per tile of a format: the E4M3 tiles
+// (64 KB of latent) are double-buffered; a bf16 tile is 128 KB (eight blocks
+// of 64 dims), so one buffer is all shared memory holds.
+template <int kFmt>
+struct FmtDims {
+  static constexpr int kBufs = kFmt == kFmtBf16 ? 1 : 2;
+  static constexpr int kBlocks = kFmt == kFmtBf16 ? 8 : 4;
+  static constexpr int kTerms = kFmt == kFmtBf16 ? 2 : 3;   // weight terms (PV N = 16 kTerms)
+};
+
+template <int kFmt>
 struct __align__(1024) Smem {
-  uint8_t lat[2][4][kLatBlock];  // [buffer][block b][128 keys x 128 B] E4M3, SW128
-  uint8_t pe[2][kKT * 128];      // [buffer][128 keys x 128 B] RoPE key (64 bf16, or 64 E4M3 + 64 zeros), SW128
-  uint8_t q8[4][2 * kHC * 128];  // [block] 32 rows x 128 B, SW128: rows 0-15 high term, 16-31 low term
+  static constexpr int kBufs = FmtDims<kFmt>::kBufs, kBlocks = FmtDims<kFmt>::kBlocks;
+  uint8_t lat[kBufs][kBlocks][kLatBlock];  // [buffer][block b][128 keys x 128 B] E4M3 (128 dims) or bf16 (64 dims), SW128
+  uint8_t pe[kBufs][kKT * 128];  // [buffer][128 keys x 128 B] RoPE key (64 bf16, or 64 E4M3 + 64 zeros), SW128
+  // E4M3: [block] 32 rows x 128 B, SW128, rows 0-15 high term, 16-31 low
+  // term; bf16: the same bytes as 8 blocks of 16 rows x 128 B (64 dims)
+  uint8_t q8[4][2 * kHC * 128];
   uint8_t qpe[2 * kHC * 128];    // RoPE query, SW128: bf16 rows 0-15; plain E4M3: rows 0-15 high, 16-31 low
-  uint8_t pb[4][kPBytes];        // weight terms of block b, MN-major 8-key x 16-B core matrices
-  float sc[2][kKT][4];            // [buffer][key] the four block scales of the staged row
+  // E4M3: weight terms of block b, MN-major 8-key x 16-B core matrices; bf16:
+  // the first 8 KB, the two terms of the weights (no block scales)
+  uint8_t pb[4][kPBytes];
+  float sc[kBufs][kKT][4];       // [buffer][key] the four block scales of the staged row
   float xmax[2][4][4][8];        // [tile parity][head quarter][key quarter]: 4 head maxima, largest scale
   float xsum[4][4][4];           // [head quarter][key quarter][head]: row-sum exchange
   float qs[kHC];                 // power-of-two query scale per head
   int32_t rowid[4][kKT];         // [tile % 4] pool row of each key, -1 = masked
-  uint64_t full[2], lat_free[2];
+  uint64_t full[kBufs], lat_free[kBufs];
   uint64_t q_ready, s_full, s_free, p_full, pv_done, o_free, drain;
   uint32_t tmem_base;
   int abort;
@@ -251,10 +275,11 @@ __device__ __forceinline__ float lg2(float x) {
 // The four warps of one head quarter (named barrier 1 + quarter).
 __device__ __forceinline__ void group_sync(int hq) { asm volatile("bar.sync %0, 128;" ::"r"(1 + hq) : "memory"); }
 
-__device__ __forceinline__ long long unit_begin(const MlaPlan& m, int c) { return m.units * c / m.ctas; }
-// The CTA whose range holds unit u.
+// First unit of the i-th CTA of a head group (units of one head group).
+__device__ __forceinline__ long long unit_begin(const MlaPlan& m, int i) { return m.units * i / m.cpg; }
+// Index, within its head group's CTAs, of the CTA whose range holds unit u.
 __device__ __forceinline__ int cta_of(const MlaPlan& m, long long u) {
-  return (int)(((u + 1) * m.ctas - 1) / m.units);
+  return (int)(((u + 1) * m.cpg - 1) / m.units);
 }
 
 // One (token, head group) of a CTA's range: tiles [j0, j0 + nj) of it, of
@@ -271,12 +296,12 @@ struct Seg {
 __device__ __forceinline__ Seg segment_at(const Params& P, long long u, long long e) {
   const MlaPlan& m = P.ws.plan;
   Seg s;
-  s.tg = (int)(u / m.tpt);
+  s.t = (int)(u / m.tpt);
   s.j0 = (int)(u % m.tpt);
-  const long long seg_end = min(e, (long long)(s.tg + 1) * m.tpt);
+  s.g = blockIdx.x % m.hg;
+  s.tg = s.t * m.hg + s.g;
+  const long long seg_end = min(e, (long long)(s.t + 1) * m.tpt);
   s.nj = (int)(seg_end - u);
-  s.t = s.tg / m.hg;
-  s.g = s.tg % m.hg;
   s.r = request_of_warp(P.cu_q, P.B, s.t);
   const Req rq = load_request(P.cu_q, P.ctx_len, s.r, P.T, P.max_ctx, P.max_pages, P.vis_len != nullptr);
   s.req_ok = rq.ok && s.t >= rq.q0 && s.t - rq.q0 < rq.Q;
@@ -293,7 +318,7 @@ __device__ __forceinline__ Seg segment_at(const Params& P, long long u, long lon
   s.len = max(0, min(len, len_max));
   const int tiles = (s.len + kKT - 1) / kKT;
   s.ne = max(0, min(s.nj, tiles - s.j0));
-  s.slot = (size_t)s.tg * m.smax + (blockIdx.x - cta_of(m, (long long)s.tg * m.tpt));
+  s.slot = (size_t)s.tg * m.smax + ((int)blockIdx.x / m.hg - cta_of(m, (long long)s.t * m.tpt));
   return s;
 }
 
@@ -341,10 +366,26 @@ __device__ __forceinline__ void cur_next(Cur& c, const Params& P, long long ue) 
 // rounding to hi and the residual lo are exact in fp32, and lo is exact in
 // E4M3 (a bf16 has 8 significant bits, hi takes 4, the residual the other 4)
 // down to E4M3's subnormal step.  RoPE part: copied as bf16; for a plain E4M3
-// pool split the same way (its products are E4M3 x E4M3).
-template <bool kPlain>
-__device__ __forceinline__ void stage_query(const Params& P, Smem& S, int t, int g, int tid) {
+// pool split the same way (its products are E4M3 x E4M3).  A bf16 pool takes
+// the bf16 query as it is (bf16 x bf16 products), s_h = 1.
+template <int kFmt>
+__device__ __forceinline__ void stage_query(const Params& P, Smem<kFmt>& S, int t, int g, int tid) {
+  constexpr bool kPlain = kFmt == kFmtPlain;
   const int h = tid >> 4, p = tid & 15;
+  if constexpr (kFmt == kFmtBf16) {
+    // 16-B chunk c of the head's row: c < 64 latent dims [8 c, 8 c + 8)
+    // (block c / 8 of 64 dims, 2 KB of 16 rows each), 64-71 the RoPE part
+    const uint16_t* qh = P.q + ((size_t)t * P.H + g * kHC + h) * (SML_LATENT_DIM + P.rope_dim);
+    const int nc = P.rope_dim ? 72 : 64;
+    const uint32_t q0 = ptx::smem_u32(&S.q8[0][0]), qp = ptx::smem_u32(S.qpe);
+    for (int c = p; c < nc; c += 16) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(qh) + c);
+      const uint32_t dst = c < 64 ? sw128(q0 + (c >> 3) * (kHC * 128), h, c & 7) : sw128(qp, h, c - 64);
+      st_shared_v4(dst, v.x, v.y, v.z, v.w);
+    }
+    if (p == 0) S.qs[h] = 1.f;
+    return;
+  }
   const int Dq = SML_LATENT_DIM + P.rope_dim;
   const uint16_t* qh = P.q + ((size_t)t * P.H + g * kHC + h) * Dq;
   uint4 v[4];
@@ -409,16 +450,21 @@ __device__ __forceinline__ void stage_query(const Params& P, Smem& S, int t, int
 // kPlain: the latent pool is plain E4M3 (576-B rows under one scale); else
 // fp8_ds_mla.  A template parameter, so that each path is compiled for its
 // own row layout.
-template <bool kPlain>
+template <int kFmt>
 __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_constant__ Params P) {
+  constexpr bool kPlain = kFmt == kFmtPlain, kBf = kFmt == kFmtBf16;
+  constexpr int kBufs = FmtDims<kFmt>::kBufs, kTerms = FmtDims<kFmt>::kTerms;
+  using Sm = Smem<kFmt>;
   extern __shared__ uint8_t smem_raw[];
-  Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Sm& S = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const MlaPlan& plan = P.ws.plan;
-  const long long ub = unit_begin(plan, blockIdx.x), ue = unit_begin(plan, blockIdx.x + 1);
+  // this CTA serves head group blockIdx.x % hg: its units are that group's
+  const int gi = (int)blockIdx.x / plan.hg;
+  const long long ub = unit_begin(plan, gi), ue = unit_begin(plan, gi + 1);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kBufs; ++i) {
       // every loader thread's copies (asynchronous arrivals) + one ordinary arrival
       ptx::mbar_init(&S.full[i], kLoadThreads + 1);
       ptx::mbar_init(&S.lat_free[i], 1);   // PV of the tile done (its last reader)
@@ -454,14 +500,16 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
     // ================= loaders: pool rows, then row copies =================
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
     const int lt = threadIdx.x - 32 * kWarpLoad;   // 0 .. kLoadThreads - 1
-    constexpr int kRow = kPlain ? SML_LATENT_E4M3_ROW_BYTES : SML_LATENT_ROW_BYTES;
+    constexpr int kRow = kBf ? SML_LATENT_BF16_ROW_BYTES : kPlain ? SML_LATENT_E4M3_ROW_BYTES : SML_LATENT_ROW_BYTES;
     // A row as 16-B chunks: 0-31 the 512-B latent (chunk c: block c / 8,
     // 16-B column c % 8); fp8_ds_mla, 32 the four block scales and 33-40 the
     // bf16 RoPE key; plain E4M3, 32-35 the 64 RoPE codes (the only bytes of
     // the row the RoPE MMA reads).  The tile's chunks are numbered row-major
     // and dealt out to the loader threads in order (chunk lt + kLoadThreads
     // i), so a warp's 32 chunks are mostly of one row.
-    const int parts = kPlain ? (P.rope_dim ? 36 : 32) : (P.rope_dim ? 41 : 33);
+    // bf16: chunks 0-63 the 1,024-B latent (block c / 8 of 64 dims), 64-71
+    // the RoPE key.
+    const int parts = kBf ? (P.rope_dim ? 72 : 64) : kPlain ? (P.rope_dim ? 36 : 32) : (P.rope_dim ? 41 : 33);
     const int drow = kLoadThreads / parts, dpart = kLoadThreads - drow * parts;
     const int row0 = lt / parts, part0 = lt - row0 * parts;
     int k = 0;   // tiles so far
@@ -474,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
         else if (s.len_bad) raise_fault(P.status, SML_FAULT_TOPK_LEN);
       }
       for (int jj = 0; jj < s.ne; ++jj, ++k) {
-        const int j = s.j0 + jj, buf = k & 1;
+        const int j = s.j0 + jj, buf = k % kBufs;
         int32_t* rowid = S.rowid[k & 3];   // last used by tile k - 4, whose softmax is done
         // pool row of the tile's key lt (loaded before the buffer is free)
         if (lt < kKT) {
@@ -492,8 +540,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
           }
           rowid[lt] = rid;
         }
-        // the buffer's last tile (k - 2) has been read by its PV
-        if (k >= 2) ok = warp_wait(&S.lat_free[buf], ((k >> 1) - 1) & 1, abort);
+        // the buffer's last tile (k - kBufs) has been read by its PV
+        if (k >= kBufs) ok = warp_wait(&S.lat_free[buf], ((k / kBufs) - 1) & 1, abort);
         ok = loader_all(ok);   // the tile's row ids written, and the wait's outcome shared
         if (!ok) break;
         // the row ids are generic writes the softmax reads: released by this
@@ -512,7 +560,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
           const int id = rowid[row];
           const uint8_t* src = P.latent + (size_t)(id >= 0 ? id : 0) * kRow + 16 * part;
           uint32_t dst;
-          if (part < 32) dst = sw128(lat0 + (part >> 3) * kLatBlock, row, part & 7);
+          if (part < (kBf ? 64 : 32)) dst = sw128(lat0 + (part >> 3) * kLatBlock, row, part & 7);
+          else if (kBf) dst = sw128(pe0, row, part - 64);
           else if (kPlain) dst = sw128(pe0, row, part - 32);
           else if (part == 32) dst = sc0 + 16 * row;
           else dst = sw128(pe0, row, part - 33);
@@ -530,10 +579,32 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
   } else if (warp == kWarpMma) {
     // ================= MMA issuer =================
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
-    const uint32_t id_qk = ptx::idesc_f16(2 * kHC, 0, 0, 0);   // E4M3 x E4M3, both K-major, N = 32
-    const uint32_t id_pe = ptx::idesc_f16(kHC, 1, 0, 0);       // bf16, N = 16
-    const uint32_t id_pv = ptx::idesc_f16(3 * kHC, 0, 1, 1);   // E4M3 x E4M3, both MN-major, N = 48
+    // E4M3 x E4M3 (bf16 pool: bf16 x bf16), both K-major, N = 32 (bf16: 16)
+    const uint32_t id_qk = kBf ? ptx::idesc_f16(kHC, 1, 0, 0) : ptx::idesc_f16(2 * kHC, 0, 0, 0);
+    const uint32_t id_pe = ptx::idesc_f16(kHC, 1, 0, 0);   // bf16, N = 16
+    // both MN-major, N = 16 x the weight terms
+    const uint32_t id_pv = kBf ? ptx::idesc_f16(2 * kHC, 1, 1, 1) : ptx::idesc_f16(3 * kHC, 0, 1, 1);
     auto issue_qk = [&](int buf) {
+      if constexpr (kBf) {
+        // S^T = C . Q^T + K_pe . Q_pe^T, all into one accumulator (no block
+        // scales), 16 dims per step: 8 blocks of 64 latent dims, then RoPE.
+        const uint32_t q0 = ptx::smem_u32(&S.q8[0][0]);
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::mma_f16_ss(T0 + kColS, ptx::sdesc_sw128(ptx::smem_u32(S.lat[buf][b]) + 32 * kk),
+                            ptx::sdesc_sw128(q0 + b * (kHC * 128) + 32 * kk), id_qk, (b | kk) != 0);
+        }
+        if (P.rope_dim) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::mma_f16_ss(T0 + kColS, ptx::sdesc_sw128(ptx::smem_u32(S.pe[buf]) + 32 * kk),
+                            ptx::sdesc_sw128(ptx::smem_u32(S.qpe) + 32 * kk), id_qk, 1);
+        }
+        ptx::mma_commit(&S.s_full);
+        return;
+      }
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {   // 32 latent dims per step
 #pragma unroll
@@ -557,7 +628,26 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
     // apart.  The first tile of a (token, head group) overwrites O; it waits
     // until the epilogue of the one before has read O.
     auto issue_pv = [&](int kk, bool first) {
-      const int buf = kk & 1;
+      const int buf = kk % kBufs;
+      if constexpr (kBf) {
+        // bf16: O_m^T (+)= C_m^T . [Bhi; Blo]^T for output block m (dims
+        // 128 m .. 128 m + 127: latent blocks 2 m and 2 m + 1, whose 64-dim
+        // swizzle atoms are 16 KB apart), 16 keys per step.  B: 8-key x 16-B
+        // core matrices (8 heads of one term), the four (term, head half)
+        // ones 128 B apart, 8-key groups 512 B apart.
+        const uint32_t pb0 = ptx::smem_u32(&S.pb[0][0]);
+#pragma unroll
+        for (int st = 0; st < kKT / 16; ++st) {
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+            ptx::mma_f16_ss(T0 + kColO + kOStride * m,
+                            ptx::sdesc(ptx::smem_u32(S.lat[buf][2 * m]) + 2048 * st, 16384, 1024, 2),
+                            ptx::sdesc(pb0 + 1024 * st, 512, 128, 0), id_pv, !first || st > 0);
+        }
+        ptx::mma_commit(&S.pv_done);
+        ptx::mma_commit(&S.lat_free[buf]);
+        return;
+      }
 #pragma unroll
       for (int st = 0; st < kKT / 32; ++st) {
 #pragma unroll
@@ -591,7 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
         if (pv_ready) {
           act = 1;
         } else if (cq.valid && cq.k <= cv.k + 1 && (cq.jj > 0 || ptx::mbar_test_wait(&S.q_ready, cq.seg & 1)) &&
-                   ptx::mbar_test_wait(&S.full[cq.k & 1], (cq.k >> 1) & 1) &&
+                   ptx::mbar_test_wait(&S.full[cq.k % kBufs], (cq.k / kBufs) & 1) &&
                    (cq.k == 0 || ptx::mbar_test_wait(&S.s_free, (cq.k - 1) & 1))) {
           act = 2;
         } else if (*abort || ++idle > (1u << 22)) {
@@ -599,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
         } else {
           // sleep on the barrier the next step most likely waits for
           if (cv.k < cq.k) ptx::mbar_try_wait_ns(&S.p_full, cv.k & 1, 200);
-          else if (cq.valid) ptx::mbar_try_wait_ns(&S.full[cq.k & 1], (cq.k >> 1) & 1, 200);
+          else if (cq.valid) ptx::mbar_try_wait_ns(&S.full[cq.k % kBufs], (cq.k / kBufs) & 1, 200);
         }
         if (act == 1) {
           ptx::tc_fence_after();
@@ -608,7 +698,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
           // the copies are generic-proxy writes: order them before the MMAs' reads
           ptx::fence_proxy_async();
           ptx::tc_fence_after();
-          issue_qk(cq.k & 1);
+          issue_qk(cq.k % kBufs);
         }
       }
       act = __shfl_sync(0xffffffffu, act, 0);
@@ -650,14 +740,14 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
       }
     };
     auto stage = [&](const Seg& s) {
-      if (warp < kStageWarps) stage_query<kPlain>(P, S, s.t, s.g, tid);
+      if (warp < kStageWarps) stage_query<kFmt>(P, S, s.t, s.g, tid);
       signal_query();
     };
     // The query of the range's first (token, head group) is an input, not
     // the selection: staged before the previous kernel has finished, and
     // signalled once that (token, head group) turns out to hold keys.
-    long long pre_tg = ub / plan.tpt;
-    if (warp < kStageWarps) stage_query<kPlain>(P, S, (int)(pre_tg / plan.hg), (int)(pre_tg % plan.hg), tid);
+    long long pre_tg = (ub / plan.tpt) * plan.hg + (int)blockIdx.x % plan.hg;
+    if (warp < kStageWarps) stage_query<kFmt>(P, S, (int)(ub / plan.tpt), (int)blockIdx.x % plan.hg, tid);
     int k = 0;
     bool ok = true, staged = false;
     for (long long u = ub; u < ue;) {
@@ -696,8 +786,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
         lrow[h] = 0.f;
       }
       for (int jj = 0; jj < s.ne; ++jj, ++k) {
-        const int buf = k & 1;
-        ok = ok && warp_wait(&S.full[buf], (k >> 1) & 1, abort) && warp_wait(&S.s_full, k & 1, abort);
+        const int buf = k % kBufs;
+        ok = ok && warp_wait(&S.full[buf], (k / kBufs) & 1, abort) && warp_wait(&S.s_full, k & 1, abort);
         if (!ok) *abort = 1;
         ok = softmax_all(ok);
         if (!ok) break;
@@ -708,8 +798,16 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
         const float psc = valid ? P.latent_scale : 0.f;
         // z = zscale * (s_h * sum_b scale_b (S_b,hi + S_b,lo) + S_pe), fp32
         float z[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (kBf) {
+          // bf16: one accumulator holds the whole dot product, RoPE included
+          uint32_t v[4];
+          ptx::tmem_ld4(T0 + kColS + 4 * hq + lane_off, v);
+          ptx::tmem_wait_ld(v);
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
+          for (int h = 0; h < 4; ++h) z[h] = __uint_as_float(v[h]);
+        }
+#pragma unroll
+        for (int b = 0; b < (kBf ? 0 : 4); ++b) {
           uint32_t vh[4], vl[4];
           ptx::tmem_ld4(T0 + kColS + 32 * b + 4 * hq + lane_off, vh);
           ptx::tmem_ld4(T0 + kColS + 32 * b + kHC + 4 * hq + lane_off, vl);
@@ -720,7 +818,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
         }
 #pragma unroll
         for (int h = 0; h < 4; ++h) z[h] *= qsh[h];
-        if (P.rope_dim) {
+        if (P.rope_dim && !kBf) {
           if (kPlain) {
             // RoPE codes under the pool scale, both query terms
             uint32_t vh[4], vl[4];
@@ -749,11 +847,14 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
         // sends the quarter's four warps through the exact update (a vote:
         // after the first tile it is rare, so most tiles exchange nothing
         // between warps here).
-        const float kmax = kPlain ? psc : fmaxf(fmaxf(scr[0], scr[1]), fmaxf(scr[2], scr[3]));
-        const float lk = kmax > 0.f ? lg2(kmax) : -INFINITY;
+        // (bf16: no scales and no overflow: the bound only keeps 2^(z - M_h)
+        // within 2^kBfCap, M_h set at the tile's maximum)
+        const float kmax = kBf ? 1.f : kPlain ? psc : fmaxf(fmaxf(scr[0], scr[1]), fmaxf(scr[2], scr[3]));
+        const float lk = kBf ? 0.f : kmax > 0.f ? lg2(kmax) : -INFINITY;
+        constexpr float kCap = kBf ? kBfLog2Cap : kLog2Cap, kHead = kBf ? 0.f : kLog2Head;
         bool need = false;
 #pragma unroll
-        for (int h = 0; h < 4; ++h) need = need || (z[h] != -INFINITY && !(z[h] - M[h] + lk <= kLog2Cap));
+        for (int h = 0; h < 4; ++h) need = need || (z[h] != -INFINITY && !(z[h] - M[h] + lk <= kCap));
         need = group_any(hq, need);
         float f[4] = {1.f, 1.f, 1.f, 1.f};
         bool any = false;
@@ -787,8 +888,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
             const float e = tm[h] + lsc;
-            if (tm[h] != -INFINITY && !(e - M[h] <= kLog2Cap)) {
-              const float Mn = ceilf(e - kLog2Head);
+            if (tm[h] != -INFINITY && !(e - M[h] <= kCap)) {
+              const float Mn = ceilf(e - kHead);
               if (M[h] != -INFINITY) {
                 const float d = M[h] - Mn;   // a negative integer
                 f[h] = d < -126.f ? 0.f : __int_as_float((127 + (int)d) << 23);
@@ -816,11 +917,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
               uint32_t ov[3][4];
               const uint32_t a = T0 + kColO + kOStride * b + 4 * hq + lane_off;
 #pragma unroll
-              for (int term = 0; term < 3; ++term) ptx::tmem_ld4(a + kHC * term, ov[term]);
+              for (int term = 0; term < kTerms; ++term) ptx::tmem_ld4(a + kHC * term, ov[term]);
               ptx::tmem_wait_ld(ov[0], ov[1]);
-              ptx::reg_fence(ov[2]);
+              if (kTerms > 2) ptx::reg_fence(ov[2]);
 #pragma unroll
-              for (int term = 0; term < 3; ++term) {
+              for (int term = 0; term < kTerms; ++term) {
 #pragma unroll
                 for (int h = 0; h < 4; ++h) ov[term][h] = __float_as_uint(__uint_as_float(ov[term][h]) * f[h]);
                 ptx::tmem_st4(a + kHC * term, ov[term]);
@@ -836,9 +937,26 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
           lrow[h] += p;
           z[h] = p;
         }
+        if constexpr (kBf) {
+          // bf16 weights as hi + lo (bf16 each: 16 significant bits): B is
+          // 8-key x 16-B core matrices of 8 heads, (term, head half) 128 B
+          // apart, 8-key groups 512 B apart
+          uint32_t hi[2], lo[2];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const __nv_bfloat162 hv = __floats2bfloat162_rn(z[2 * i], z[2 * i + 1]);
+            const float2 hf = __bfloat1622float2(hv);
+            const __nv_bfloat162 lv = __floats2bfloat162_rn(z[2 * i] - hf.x, z[2 * i + 1] - hf.y);
+            hi[i] = *reinterpret_cast<const uint32_t*>(&hv);
+            lo[i] = *reinterpret_cast<const uint32_t*>(&lv);
+          }
+          const uint32_t pb = ptx::smem_u32(&S.pb[0][0]) + (row >> 3) * 512 + (hq >> 1) * 128 + (row & 7) * 16 + (hq & 1) * 8;
+          st_shared_v2(pb, hi[0], hi[1]);
+          st_shared_v2(pb + 256, lo[0], lo[1]);
+        }
         const uint32_t pb_off = (row >> 3) * 384 + (row & 7) * 16 + 4 * hq;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
+        for (int b = 0; b < (kBf ? 0 : 4); ++b) {
           const float scb = kPlain ? psc : scr[b];
           uint32_t h01, m01, l01, h23, m23, l23;
           split3_e4m3x2(z[0] * scb, z[1] * scb, h01, m01, l01);
@@ -891,14 +1009,15 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
         uint32_t o3[3][4];
         const uint32_t a = T0 + kColO + kOStride * b + 4 * hq + lane_off;
 #pragma unroll
-        for (int term = 0; term < 3; ++term) ptx::tmem_ld4(a + kHC * term, o3[term]);
+        for (int term = 0; term < kTerms; ++term) ptx::tmem_ld4(a + kHC * term, o3[term]);
         ptx::tmem_wait_ld(o3[0], o3[1]);
-        ptx::reg_fence(o3[2]);
+        if (kTerms > 2) ptx::reg_fence(o3[2]);
         const int dim = 128 * b + row;
 #pragma unroll
         for (int h = 0; h < 4; ++h)
           pout[(size_t)(4 * hq + h) * SML_LATENT_DIM + dim] =
-              (__uint_as_float(o3[0][h]) + __uint_as_float(o3[1][h]) + __uint_as_float(o3[2][h])) * osc[h];
+              (__uint_as_float(o3[0][h]) + __uint_as_float(o3[1][h]) + (kTerms > 2 ? __uint_as_float(o3[2][h]) : 0.f)) *
+              osc[h];
       }
       ptx::tc_fence_before();
       __syncwarp();
@@ -929,7 +1048,7 @@ lse_merge_kernel(int H, MlaWs ws, float* __restrict__ out, float* __restrict__ l
   ptx::griddep_wait();   // the partials come from the previous kernel
   const MlaPlan& m = ws.plan;
   const int tg = t * m.hg + h / kHC, hl = h % kHC;
-  const long long u0 = (long long)tg * m.tpt;
+  const long long u0 = (long long)t * m.tpt;   // the token's first unit in its head group
   const int n = cta_of(m, u0 + m.tpt - 1) - cta_of(m, u0) + 1;   // <= tiles per token + 1 <= 32
   const size_t base = (size_t)tg * m.smax;
   const float ls = lane < n ? __ldcg(ws.part_lse + (base + lane) * kHC + hl) : -INFINITY;
@@ -975,21 +1094,25 @@ MlaPlan mla_plan(const sml_problem& p) {
   MlaPlan m;
   m.hg = p.num_heads / kHC;
   m.tpt = (p.topk + kKT - 1) / kKT;
-  m.units = (long long)p.num_tokens * m.hg * m.tpt;
-  // As few CTAs as give the same longest range: ceil(units / SMs) units per
-  // CTA at most.  (On decode, all SMs gathering at once only adds contention
-  // at the memory for the same finishing time.)
+  m.units = (long long)p.num_tokens * m.tpt;
   if (m.units < 1) {
+    m.cpg = 0;
     m.ctas = 0;
     m.smax = 1;
     return m;
   }
+  // Per head group, as few CTAs as give the same longest range: ceil(units /
+  // its share of the SMs) units per CTA at most.  (On decode, all SMs
+  // gathering at once only adds contention at the memory for the same
+  // finishing time.)
   const long long sms = device_sm_count();
-  const long long most = (m.units + sms - 1) / sms;
-  m.ctas = (int)((m.units + most - 1) / most);
+  const long long share = sms / m.hg > 0 ? sms / m.hg : 1;
+  const long long most = (m.units + share - 1) / share;
+  m.cpg = (int)((m.units + most - 1) / most);
+  m.ctas = m.hg * m.cpg;
   // every CTA holds at least `per` units, so a run of tpt units touches at
   // most 1 + ceil((tpt - 1) / per) CTAs
-  const long long per = m.units / m.ctas;
+  const long long per = m.units / m.cpg;
   m.smax = (int)((m.tpt - 1 + per - 1) / per) + 1;
   return m;
 }
@@ -1024,8 +1147,9 @@ cudaError_t launch_sparse_mla(const sml_problem& p, const uint16_t* q, const sml
   P.idx_len = idx_len;
   P.ws = ws;
   P.status = status;
-  const size_t smem = sizeof(Smem) + 1024;
-  auto kernel = plain ? sparse_mla_kernel<true> : sparse_mla_kernel<false>;
+  const bool bf16 = latent.format == SML_LATENT_BF16;
+  const size_t smem = (bf16 ? sizeof(Smem<kFmtBf16>) : plain ? sizeof(Smem<kFmtPlain>) : sizeof(Smem<kFmtDsMla>)) + 1024;
+  auto kernel = bf16 ? sparse_mla_kernel<kFmtBf16> : plain ? sparse_mla_kernel<kFmtPlain> : sparse_mla_kernel<kFmtDsMla>;
   cudaError_t e = set_max_smem(reinterpret_cast<const void*>(kernel), smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kernel, dim3(ws.plan.ctas), dim3(kThreads), smem, stream, 0, P);

@@ -80,7 +80,7 @@ extern "C" int sml_sparse_mla_decode_noalloc(const sml_problem* p, const void* q
   if (latent.num_pages < 1) fail(SML_ERR_INVALID_ARG, "latent.num_pages < 1");
   if (latent.format == SML_LATENT_E4M3) {
     if (!(isfinite(latent.scale) && latent.scale > 0.f)) fail(SML_ERR_INVALID_ARG, "latent.scale not finite and positive");
-  } else if (latent.format != SML_LATENT_FP8_DS_MLA) {
+  } else if (latent.format != SML_LATENT_FP8_DS_MLA && latent.format != SML_LATENT_BF16) {
     fail(SML_ERR_UNSUPPORTED, "latent.format not an SML_LATENT_* format");
   }
   MlaWs ws{};

@@ -175,6 +175,46 @@ latent_write_plain_kernel(const uint4* __restrict__ c, const uint4* __restrict__
   }
 }
 
+// The bf16 pool (blog, section "ROCm 实现细节", paragraph "FP8 潜在缓存": 1,152 B
+// per token per layer in bf16): a row is the token's 512 latent and 64 RoPE
+// values as given, no quantisation.  Two new tokens per warp: lane l copies
+// latent bytes [32 l, 32 l + 32); lanes 0..7 the RoPE bytes 1,024 + 16 l
+// (zeros without a RoPE key).
+__global__ void __launch_bounds__(32 * kWarpsPerCta)
+latent_write_bf16_kernel(const uint4* __restrict__ c, const uint4* __restrict__ kpe,
+                         const int32_t* __restrict__ slot, int n, uint8_t* __restrict__ cache, long long slots,
+                         int32_t* status) {
+  ptx::griddep_wait();
+  if (threadIdx.x == 0) ptx::griddep_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int step = gridDim.x * kWarpsPerCta * kTokPerWarp;
+  for (int i0 = (blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5)) * kTokPerWarp; i0 < n; i0 += step) {
+    int s[kTokPerWarp];
+    uint4 v0[kTokPerWarp], v1[kTokPerWarp], pe[kTokPerWarp];
+#pragma unroll
+    for (int u = 0; u < kTokPerWarp; ++u) {
+      const int i = i0 + u;
+      s[u] = i < n ? __ldg(slot + i) : -1;
+      pe[u] = make_uint4(0, 0, 0, 0);
+      if (i < n) {
+        const uint4* src = c + (size_t)i * (SML_LATENT_DIM / 8) + 2 * lane;
+        v0[u] = __ldg(src);
+        v1[u] = __ldg(src + 1);
+        if (kpe && lane < 8) pe[u] = __ldg(kpe + (size_t)i * (SML_ROPE_DIM / 8) + lane);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kTokPerWarp; ++u) {
+      if (!slot_ok(s[u], slots, lane, status)) continue;
+      uint8_t* row = cache + (size_t)(s[u] / SML_PAGE_TOKENS) * SML_LATENT_BF16_PAGE_BYTES +
+                     (size_t)(s[u] % SML_PAGE_TOKENS) * SML_LATENT_BF16_ROW_BYTES;
+      reinterpret_cast<uint4*>(row)[2 * lane] = v0[u];
+      reinterpret_cast<uint4*>(row)[2 * lane + 1] = v1[u];
+      if (lane < 8) reinterpret_cast<uint4*>(row + 2 * SML_LATENT_DIM)[lane] = pe[u];
+    }
+  }
+}
+
 // One CTA per query token: 64 x 128 bf16 in (16 KB), one block.
 constexpr int kQThreads = 256;
 constexpr int kQVec = SML_INDEX_HEADS * SML_INDEX_DIM / 8 / kQThreads;   // uint4 loads per thread: 4
@@ -230,6 +270,9 @@ cudaError_t launch_latent_write(const void* c, const void* kpe, const int32_t* s
   const dim3 grid(token_grid(n, kWarpsPerCta * kTokPerWarp, 8)), block(32 * kWarpsPerCta);
   uint8_t* base = static_cast<uint8_t*>(const_cast<void*>(cache.base));
   const long long slots = (long long)cache.num_pages * SML_PAGE_TOKENS;
+  if (cache.format == SML_LATENT_BF16)
+    return launch_pdl(latent_write_bf16_kernel, grid, block, 0, stream, 0, static_cast<const uint4*>(c),
+                      static_cast<const uint4*>(kpe), slot, n, base, slots, status);
   if (cache.format == SML_LATENT_E4M3)
     return launch_pdl(latent_write_plain_kernel, grid, block, 0, stream, 0, static_cast<const uint4*>(c),
                       static_cast<const uint4*>(kpe), slot, n, cache.scale, base, slots, status);

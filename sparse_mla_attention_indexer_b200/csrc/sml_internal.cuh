@@ -44,11 +44,16 @@ struct TopkWs {
 // (token, head group) its range touches; a (token, head group) has at most
 // `smax` such CTAs, and its partials sit in slots [tg * smax, tg * smax + n)
 // in CTA order, n = the CTAs that touch it.
+// Sparse-MLA work plan.  Head group g is served by the CTAs with blockIdx.x
+// % hg == g; those cpg CTAs split its T * tpt (token, tile) units into equal
+// contiguous ranges (token-major), so the hg CTAs with the same blockIdx.x /
+// hg walk the same tokens' tiles together and read each row while it is in L2.
 struct MlaPlan {
   int hg;              // head groups, H / 16
   int tpt;             // tiles per (token, head group), ceil(topk / 128)
-  long long units;     // T * hg * tpt
-  int ctas;            // min(SMs, units)
+  long long units;     // units of one head group: T * tpt
+  int cpg;             // CTAs per head group
+  int ctas;            // hg * cpg
   int smax;            // slots per (token, head group)
 };
 

@@ -36,6 +36,8 @@ class DeviceWorkload:
         self.latent = torch.from_numpy(wl.latent).to(device)
         if wl.latent_format == "e4m3":
             self.latent = sml.E4M3Latent(self.latent, wl.latent_scale)
+        elif wl.latent_format == "bf16":
+            self.latent = sml.Bf16Latent(self.latent)
         self.index_cache = torch.from_numpy(wl.index_cache).to(device)
         self.layers = [DeviceLayer(lay, device) for lay in wl.layers]
         self.T, self.H, self.K = wl.T, wl.num_heads, wl.topk

@@ -40,9 +40,11 @@ SML_STAGE_LAYER = 4
 PAGE_TOKENS = 64
 LATENT_PAGE_BYTES = 64 * 656
 LATENT_E4M3_PAGE_BYTES = 64 * 576
+LATENT_BF16_PAGE_BYTES = 64 * 1152
 INDEX_PAGE_BYTES = 64 * 132
 SML_LATENT_FP8_DS_MLA = 0
 SML_LATENT_E4M3 = 1
+SML_LATENT_BF16 = 2
 
 
 class SmlError(RuntimeError):
@@ -87,6 +89,11 @@ class DcpRanks(ctypes.Structure):
                 ("idx", ctypes.c_void_p * SML_DCP_MAX_RANKS),
                 ("idx_len", ctypes.c_void_p * SML_DCP_MAX_RANKS),
                 ("packed", ctypes.c_int32)]
+
+
+class Bf16Latent(NamedTuple):
+    """A latent pool in bf16 (1,152-B rows: 512 latent then 64 RoPE values)."""
+    pool: torch.Tensor
 
 
 class E4M3Latent(NamedTuple):
@@ -202,7 +209,9 @@ def cache(pool, page_bytes: int) -> Cache:
 
 
 def latent_cache(latent) -> Cache:
-    """Descriptor of a latent pool: a uint8 tensor (fp8_ds_mla) or an E4M3Latent."""
+    """Descriptor of a latent pool: a uint8 tensor (fp8_ds_mla), an E4M3Latent or a Bf16Latent."""
+    if isinstance(latent, Bf16Latent):
+        return Cache(_p(latent.pool), _nbytes(latent.pool) // LATENT_BF16_PAGE_BYTES, SML_LATENT_BF16, 0.0)
     if isinstance(latent, E4M3Latent):
         return Cache(_p(latent.pool), _nbytes(latent.pool) // LATENT_E4M3_PAGE_BYTES, SML_LATENT_E4M3,
                      float(latent.scale))

@@ -37,6 +37,8 @@ LATENT_ROW = 656
 LATENT_PAGE = PAGE * LATENT_ROW
 PLAIN_ROW = 576                      # plain per-tensor E4M3 latent row
 PLAIN_PAGE = PAGE * PLAIN_ROW
+BF16_ROW = 1152                      # bf16 latent row: 512 latent + 64 RoPE values
+BF16_PAGE = PAGE * BF16_ROW
 PLAIN_SCALE = 8.0 / 448.0            # pool scale of plain E4M3 latents: N(0, 1) values within +-8
 INDEX_PAGE = PAGE * 132
 E4M3_MAX = 448.0
@@ -97,7 +99,7 @@ class Workload:
     ssmax_s: float = 0.4
     ssmax_s_index: float = 0.4
     sm_scale: float = 1.0 / math.sqrt(576.0)
-    latent_format: str = "fp8_ds_mla"   # or "e4m3": 576-B rows under one pool scale
+    latent_format: str = "fp8_ds_mla"   # or "e4m3": 576-B rows under one pool scale; or "bf16": 1,152-B rows
     latent_scale: float = 0.0
 
     @property
@@ -174,7 +176,8 @@ def _fill_index(seed: int, name: str, num_pages: int, chunk_pages: int = 2048) -
 
 def _scribble_tails(wl: Workload, rng: np.random.Generator):
     """Random bytes in the unused rows of each request's last page."""
-    lat = wl.latent.reshape(wl.num_pages, PAGE, PLAIN_ROW if wl.latent_format == "e4m3" else LATENT_ROW)
+    row = {"e4m3": PLAIN_ROW, "bf16": BF16_ROW}.get(wl.latent_format, LATENT_ROW)
+    lat = wl.latent.reshape(wl.num_pages, PAGE, row)
     idx = wl.index_cache.reshape(wl.num_pages, INDEX_PAGE)
     for r in range(wl.B):
         L = int(wl.ctx_len[r])
@@ -213,6 +216,21 @@ def plain_pool(seed: int, name: str, num_pages: int, chunk_pages: int = 512) -> 
     return out.reshape(-1)
 
 
+def bf16_pool(seed: int, name: str, num_pages: int, chunk_pages: int = 512) -> np.ndarray:
+    """bf16 latent pool: 576 values N(0, 1) per row (512 latent, 64 RoPE), as
+    bf16 bits (float32 rounded to nearest even), little-endian."""
+    out = np.empty((num_pages, BF16_PAGE), dtype=np.uint8)
+
+    def fill(i, p0, p1):
+        x = stream(seed, f"{name}/bf16/{i}").standard_normal(((p1 - p0) * PAGE, PLAIN_ROW), dtype=np.float32)
+        b = x.view(np.uint32)
+        h = ((b + np.uint32(0x7FFF) + ((b >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)).astype("<u2")
+        out[p0:p1] = h.view(np.uint8).reshape(p1 - p0, BF16_PAGE)
+
+    _chunked(num_pages, chunk_pages, fill)
+    return out.reshape(-1)
+
+
 def make_workload(name: str, ctx_len, q_count, num_heads: int, topk: int = 2048,
                   layers=(("rope", 64, True, None),), permuted: bool = True, ssmax: bool = False,
                   seed: int = 0, extra_pages: int = 0, latent_format: str = "fp8_ds_mla") -> Workload:
@@ -220,8 +238,8 @@ def make_workload(name: str, ctx_len, q_count, num_heads: int, topk: int = 2048,
 
     ``layers``: tuples (tag, rope_dim, with_indexer, reuse_from).
     ``extra_pages``: unused pages appended to the pool (random bytes).
-    ``latent_format``: "fp8_ds_mla" (656-B rows) or "e4m3" (576-B rows, one
-    pool scale PLAIN_SCALE).
+    ``latent_format``: "fp8_ds_mla" (656-B rows), "e4m3" (576-B rows, one
+    pool scale PLAIN_SCALE) or "bf16" (1,152-B rows).
     """
     ctx_len = np.asarray(ctx_len, dtype=np.int32)
     q_count = np.asarray(q_count, dtype=np.int32)
@@ -241,10 +259,12 @@ def make_workload(name: str, ctx_len, q_count, num_heads: int, topk: int = 2048,
         block_table[r, :pages_per[r]] = phys[off:off + pages_per[r]]
         off += pages_per[r]
     plain = latent_format == "e4m3"
-    assert plain or latent_format == "fp8_ds_mla"
+    assert latent_format in ("fp8_ds_mla", "e4m3", "bf16")
+    latent = (plain_pool(seed, name, num_pages) if plain else
+              bf16_pool(seed, name, num_pages) if latent_format == "bf16" else _fill_latent(seed, name, num_pages))
     wl = Workload(name=name, num_heads=num_heads, topk=topk, cu_q=cu_q, ctx_len=ctx_len,
                   block_table=block_table, num_pages=num_pages,
-                  latent=plain_pool(seed, name, num_pages) if plain else _fill_latent(seed, name, num_pages),
+                  latent=latent,
                   index_cache=_fill_index(seed, name, num_pages),
                   ssmax=ssmax, latent_format=latent_format, latent_scale=PLAIN_SCALE if plain else 0.0)
     _scribble_tails(wl, stream(seed, name + "/tails"))

@@ -25,6 +25,8 @@ def oracle_latent(wl):
     """The workload's latent pool as the oracle reads it."""
     if wl.latent_format == "e4m3":
         return formats.PlainE4M3Pool(wl.latent, wl.latent_scale)
+    if wl.latent_format == "bf16":
+        return formats.Bf16Pool(wl.latent)
     return wl.latent
 
 

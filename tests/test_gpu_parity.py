@@ -301,6 +301,31 @@ def test_plain_e4m3_latent_batched_decode_full():
     parity.check_attention(wl, 0, r["idx"], r["len"], r["out"], r["lse"])
 
 
+# --- the bf16 latent pool (1,152-B rows) ---------------------------------------------
+
+@pytest.mark.parametrize("case", [0, 1, 2, 4])
+def test_bf16_latent_small_every_element(case):
+    L, Q, H, K, rope, ssmax, perm = SMALL[case]
+    wl = synth.make_workload(f"bf16_{case}", L, Q, H, topk=K, permuted=perm, ssmax=ssmax,
+                             layers=(("l0", rope, True, None),), extra_pages=3, latent_format="bf16")
+    dw = DeviceWorkload(wl)
+    r = run_stages(dw)
+    parity.check_topk(wl, r["scores"], r["idx"], r["len"])
+    parity.check_attention(wl, 0, r["idx"], r["len"], r["out"], r["lse"])
+    r2 = run_layer(dw)
+    assert np.array_equal(r2["out"], r["out"]) and np.array_equal(r2["lse"], r["lse"], equal_nan=True)
+
+
+def test_bf16_latent_batched_decode_full():
+    base = synth.batched_decode()
+    wl = synth.make_workload("batched_decode_bf16", base.ctx_len, np.ones(base.B, np.int32), 16,
+                             latent_format="bf16")
+    dw = DeviceWorkload(wl)
+    r = run_stages(dw)
+    parity.check_topk(wl, r["scores"], r["idx"], r["len"])
+    parity.check_attention(wl, 0, r["idx"], r["len"], r["out"], r["lse"])
+
+
 def test_plain_e4m3_rejects_a_bad_scale():
     wl = synth.make_workload("plain_bad", [300], [1], 16, topk=64, latent_format="e4m3")
     dw = DeviceWorkload(wl)

@@ -156,3 +156,25 @@ def test_plain_e4m3_latent_write_bit_exact(n, pages, skip, rope):
     got = pool.cpu().numpy()
     diff = np.nonzero(got != want.data)[0]
     assert diff.size == 0, f"{diff.size} bytes differ, first at {diff[:8]}"
+
+
+@pytest.mark.parametrize("n,pages,skip,rope", [(10003, 160, 101, True), (300, 6, 7, False)])
+def test_bf16_latent_write_bit_exact(n, pages, skip, rope):
+    """The bf16 latent writer stores every row exactly as the oracle's writer
+    does (values as given, zeros for a NoPE row's RoPE key), skip markers and
+    untouched rows included."""
+    from oracle import formats as F
+    c = synth.producer_rows(7, f"bc/{n}", n, 512, spread=False)
+    kpe = synth.producer_rows(7, f"bkpe/{n}", n, 64, spread=False) if rope else None
+    slot = synth.producer_slots(7, f"bslot/{n}", n, pages, skip)
+    pool0 = synth.stream(7, f"bpool/{n}").integers(0, 256, pages * synth.BF16_PAGE, dtype=np.uint8)
+    want, bad = PR.write_latent_bf16(F.Bf16Pool(pool0), c, kpe, slot)
+    assert not bad
+    pool = dev(pool0)
+    ws = status_ws()
+    sml.sml_latent_cache_write(bf16_dev(c), None if kpe is None else bf16_dev(kpe), dev(slot),
+                               sml.Bf16Latent(pool), ws)
+    assert sml.sml_read_device_status(ws)[0] == sml.SML_OK
+    got = pool.cpu().numpy()
+    diff = np.nonzero(got != want.data)[0]
+    assert diff.size == 0, f"{diff.size} bytes differ, first at {diff[:8]}"
