@@ -46,7 +46,8 @@ constexpr int kQRowsBytes = SML_INDEX_HEADS * SML_INDEX_DIM;      // 8,192 per q
 //            (N = 64), four 64-column accumulators, one epilogue warpgroup, and
 //            half the shared memory and TMEM, so two CTAs share each SM and
 //            keep twice the loads in flight.
-template <int kStages_, int kGroup_, int kAccBufs_, int kEpiGroups_, int kCtasPerSm_, bool kQueryPerWg_>
+template <int kStages_, int kGroup_, int kAccBufs_, int kEpiGroups_, int kCtasPerSm_, bool kQueryPerWg_,
+          int kQBufs_>
 struct Cfg {
   static constexpr int kStages = kStages_;
   static constexpr int kGroup = kGroup_;          // query tokens per group: N = 64 * Qg
@@ -56,28 +57,31 @@ struct Cfg {
   static constexpr int kEpiGroups = kEpiGroups_;  // epilogue warpgroups, taking alternate items
   static constexpr int kThreads = 64 + 128 * kEpiGroups_;   // warp 0 TMA, warp 1 MMA, then the epilogue
   static constexpr int kCtasPerSm = kCtasPerSm_;
-  // true: epilogue warpgroup g takes query g of every item (kEpiGroups ==
-  // kGroup); false: the warpgroups take alternate items, all their queries.
+  // true: every epilogue warpgroup works on every item, warpgroup g on
+  // queries [g kWgQ, (g + 1) kWgQ) of the group; false: the warpgroups take
+  // alternate items, all their queries.
   static constexpr bool kQueryPerWg = kQueryPerWg_;
-  static_assert(!kQueryPerWg_ || kEpiGroups_ == kGroup_, "one epilogue warpgroup per query of a group");
+  static constexpr int kWgQ = kQueryPerWg_ ? kGroup_ / kEpiGroups_ : kGroup_;
+  static_assert(!kQueryPerWg_ || kGroup_ % kEpiGroups_ == 0, "whole query shares per warpgroup");
+  static constexpr int kQBufs = kQBufs_;   // query-group buffers
 };
-using CfgGeneral = Cfg<9, 4, 2, 4, 1, true>;
-using CfgDecode = Cfg<5, 1, 4, 1, 2, false>;
+using CfgGeneral = Cfg<9, 4, 2, 4, 1, true, 2>;
+using CfgDecode = Cfg<5, 1, 4, 1, 2, false, 2>;
 
 template <class C>
 struct __align__(1024) Smem {
   static constexpr int kStages = C::kStages, kGroup = C::kGroup, kEpiGroups = C::kEpiGroups;
   uint8_t keys[kStages][2 * kPageKeyBytes];      // [stage][128 rows x 128 B], SW128
-  uint8_t q[2][kGroup * kQRowsBytes];            // [buffer][256 rows x 128 B], SW128
+  uint8_t q[C::kQBufs][kGroup * kQRowsBytes];    // [buffer][256 rows x 128 B], SW128
   float ksc[kStages][kTile];
   // per epilogue warpgroup: head weights, sq_t * c_t and n_t of its queries
   // (the whole group, or its one query of the group when kQueryPerWg)
-  static constexpr int kWgQueries = C::kQueryPerWg ? 1 : kGroup;
+  static constexpr int kWgQueries = C::kWgQ;
   __align__(16) float w[kEpiGroups][kWgQueries * SML_INDEX_HEADS];
   float qf[kEpiGroups][kWgQueries];
   int nv[kEpiGroups][kWgQueries];
   uint64_t full[kStages], empty[kStages];
-  uint64_t qfull[2], qempty[2];
+  uint64_t qfull[C::kQBufs], qempty[C::kQBufs];
   uint64_t accfull[C::kAccBufs], accempty[C::kAccBufs];
   uint64_t drain;
   int valid[kStages];                            // bit p: page p of the tile was loaded
@@ -290,7 +294,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
       // MMA commit + one arrive per epilogue warp that reads the stage
       ptx::mbar_init(&S.empty[i], 1 + (C::kQueryPerWg ? 4 * kEpiGroups : 4));
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::kQBufs; ++i) {
       ptx::mbar_init(&S.qfull[i], 1);
       ptx::mbar_init(&S.qempty[i], 1);
     }
@@ -329,8 +333,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
       int qcount = 0, last_r = -1, last_g = -1;
       for (int it = beg; it < end; ++it, w.advance()) {
         if (w.r != last_r || w.g != last_g) {
-          const int qb = qcount & 1;
-          if (!ptx::mbar_wait(&S.qempty[qb], ((qcount >> 1) & 1) ^ 1, abort)) { *abort = 1; break; }
+          const int qb = qcount % C::kQBufs;
+          if (!ptx::mbar_wait(&S.qempty[qb], ((qcount / C::kQBufs) & 1) ^ 1, abort)) { *abort = 1; break; }
           const int qg = w.qg();
           ptx::mbar_arrive_expect_tx(&S.qfull[qb], qg * kQRowsBytes);
           for (int j = 0; j < qg; ++j)
@@ -389,8 +393,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
       for (int it = beg; it < end; ++it, w.advance()) {
         if (w.r != last_r || w.g != last_g) {
           if (qcount > 0) ptx::mma_commit(&S.qempty[qb]);   // previous group's queries free once read
-          qb = qcount & 1;
-          if (!ptx::mbar_wait(&S.qfull[qb], (qcount >> 1) & 1, abort)) { *abort = 1; break; }
+          qb = qcount % C::kQBufs;
+          if (!ptx::mbar_wait(&S.qfull[qb], (qcount / C::kQBufs) & 1, abort)) { *abort = 1; break; }
           ++qcount;
           last_r = w.r;
           last_g = w.g;
@@ -447,8 +451,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
       const int qg = w.qg();
       const int j0 = kGroup * w.g;
       // this warpgroup's queries of the group: [jb, jb + jn)
-      const int jb = C::kQueryPerWg ? eg : 0;
-      const int jn = C::kQueryPerWg ? (eg < qg ? 1 : 0) : qg;
+      const int jb = C::kQueryPerWg ? eg * kWq : 0;
+      const int jn = C::kQueryPerWg ? max(0, min(kWq, qg - jb)) : qg;
       if (w.r != last_r || w.g != last_g) {
         asm volatile("bar.sync %0, 128;" ::"r"(1 + eg) : "memory");
         for (int i = et; i < jn * SML_INDEX_HEADS; i += 128)
