@@ -910,8 +910,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
             *abort = 1;
             continue;   // the next softmax_all ends every softmax warp
           }
-          ptx::tc_fence_after();
           if (any) {
+            ptx::tc_fence_after();   // TMEM accesses after the wait (none when nothing is rescaled)
 #pragma unroll 1
             for (int b = 0; b < 4; ++b) {   // this thread: latent dim 128 b + row, this quarter's heads
               uint32_t ov[3][4];
