@@ -194,7 +194,10 @@ int sml_indexer_scores(const sml_problem* p, const void* iq8, const float* iq_sc
  *   scores   [T, max_ctx] fp32 (row stride max_ctx), read for s < n_t only
  *   idx      [T, topk] int32 out: the selected positions in ASCENDING order,
  *            then -1 padding
- *   idx_len  [T] int32 out: min(topk, n_t) */
+ *   idx_len  [T] int32 out: min(topk, n_t)
+ * cu_q / ctx_len inconsistent with the problem set SML_FAULT_LENGTHS (the row
+ * gets len 0); a copy of a row's scores into shared memory that outlives its
+ * wait limit sets SML_FAULT_TIMEOUT (that row's selection is then unspecified). */
 int sml_topk(const sml_problem* p, const float* scores, int32_t* idx, int32_t* idx_len,
              void* workspace, size_t ws_bytes, void* stream);
 

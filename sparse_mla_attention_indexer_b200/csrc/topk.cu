@@ -7,10 +7,11 @@
 //
 //  * scores become order-preserving 32-bit keys (-0 -> +0, NaN lowest);
 //  * a 1,024-key sample places a floor below the k-th largest value; one pass
-//    histograms the values at or above it into 2,048 buckets linear in value
-//    up to the row's maximum (so the shared-memory atomics touch about k values
-//    and spread over the bins) and finds the bucket that holds the k-th
-//    largest value; if the sample misjudged, the pass covers every value;
+//    histograms the values at or above it into 2,048 buckets (512 where one
+//    cluster selects a row) linear in value up to the row's maximum (so the
+//    shared-memory atomics touch about k values and spread over the bins) and
+//    finds the bucket that holds the k-th largest value; if the sample
+//    misjudged, the pass covers every value;
 //  * only that bucket's keys (a handful, typically) go through an exact radix
 //    select (11 / 11 / 10 key bits) to find the k-th largest key tau and how
 //    many keys equal to tau are taken; a row whose threshold bucket is huge
@@ -700,16 +701,25 @@ topk_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32_t* __re
 // Rows of up to kClusterMax chunks: the chunks' CTAs form one thread-block
 // cluster and select together, in one level, exchanging histograms, the keys
 // of the threshold bucket and the selected counts through distributed shared
-// memory at hardware cluster barriers.  Each CTA makes one pass over its chunk
-// that histograms the values at or above a sampled floor and compacts them,
-// in position order, into per-warp candidate lists; every later step touches
-// only those candidates.
+// memory at hardware cluster barriers.  Each CTA lands its chunk's raw scores
+// in shared memory with one bulk asynchronous copy (a CTA's plain loads top out
+// near 20 GB/s), places a floor from a strided sample meanwhile, then makes one
+// pass over the chunk that compacts the values at or above the floor, in
+// position order, into per-warp candidate lists in place; the histogram (512
+// buckets linear in value from the floor) and every later step touch only
+// those candidates.
 
 constexpr int kClusterMax = 8;
 constexpr int kWarps = kTopkThreads / 32;
 constexpr int kSegMax = kTopkChunk / kWarps;   // positions per warp segment
+constexpr int kLinBuckets = 512;              // value-linear buckets of the candidate histogram
+static_assert(kLinBuckets <= kBuckets && kLinBuckets % kTopkThreads == 0, "one pass of bins per thread");
+constexpr int kBulkPiece = 4096;              // positions per bulk copy instruction (16 KB)
+constexpr uint32_t kBulkWaitUs = 200000;      // limit on the wait for the chunk's copy
+static_assert(kSegMax % 128 == 0, "warp segments are whole 128-position steps");
 
 struct ClusterShared {
+  uint64_t full;                   // the chunk's bulk copy has landed
   int hist[kBuckets];              // this CTA's histogram (read by the whole cluster)
   int gh[kBuckets];                // the cluster's histogram
   uint16_t cpos[kWarps][kSegMax];  // candidate positions (chunk-local) per warp, ascending
@@ -724,6 +734,7 @@ struct ClusterShared {
   int warp_a[32], warp_b[32];
   float red_lo[32], red_hi[32];
   int bcast[2];
+  int bcast_tot;
   uint32_t bcast_tau;
   float bcast_f;
 };
@@ -759,9 +770,8 @@ __device__ __forceinline__ uint32_t ld_cluster(const void* p, uint32_t rank) {
 // S.gh = the sum over the cluster of every CTA's S.hist[0, nb).  The caller
 // passes a cluster barrier before any CTA rebuilds S.hist.
 __device__ __forceinline__ void cluster_hist_sum(ClusterShared& S, int nb, int C) {
-  __syncthreads();
-  cluster_sync();
-  // nb / blockDim.x bins per thread (2 or 4), every remote load in flight at once
+  cluster_sync();   // covers this CTA's threads too
+  // up to kBuckets / blockDim.x bins per thread, every remote load in flight at once
   constexpr int kPer = kBuckets / kTopkThreads;
   uint32_t v[kPer][kClusterMax];
 #pragma unroll
@@ -781,6 +791,42 @@ __device__ __forceinline__ void cluster_hist_sum(ClusterShared& S, int nb, int C
   __syncthreads();
 }
 
+// One warp: over hist[0, NB) (NB a multiple of 32), the bin holding the
+// need-th largest element and how many lie in the bins above it, into
+// sh.bcast[0] and sh.bcast[1] (left alone when the histogram holds fewer than
+// need); returns the histogram's total in every lane.
+template <int NB, typename Sh>
+__device__ __forceinline__ int bin_scan_warp(int need, const int* hist, Sh& sh) {
+  const int lane = threadIdx.x & 31;
+  constexpr int kPer = NB / 32;
+  const int top = NB - 1 - lane * kPer;   // lane l holds bins top, top - 1, ..., descending
+  int h[kPer];
+  int local = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    h[j] = hist[top - j];
+    local += h[j];
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int above = incl - local;
+  if (above < need && need <= incl) {
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      if (above < need && need <= above + h[j]) {
+        sh.bcast[0] = top - j;
+        sh.bcast[1] = above;
+      }
+      above += h[j];
+    }
+  }
+  return __shfl_sync(0xffffffffu, incl, 31);
+}
+
 __global__ void __launch_bounds__(kTopkThreads, 1)
 topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32_t* __restrict__ cu_q,
                     const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ vis_len,
@@ -793,13 +839,22 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
   const int C = (int)cluster_size(), c = (int)cluster_rank();
   const int t = blockIdx.y;
   if (tid == 0) ptx::griddep_launch_dependents();
-  ptx::griddep_wait();   // the scores come from the previous kernel
-  // Everything up to the first cluster barrier depends only on the row, so an
-  // early return is taken by the whole cluster or by none of it.
+  // The request lookup reads inputs that no kernel of this library writes, so
+  // it runs before the wait; every global write and every read of the scores
+  // follows it.  Everything up to the first cluster barrier depends only on
+  // the row, so an early return is taken by the whole cluster or by none of it.
   const int r = request_of_warp(cu_q, B, t);
   const Req rq = load_request(cu_q, ctx_len, r, T, max_ctx, max_pages, vis_len != nullptr);
+  const bool row_ok = rq.ok && t >= rq.q0 && t - rq.q0 < rq.Q;
+  bool bad_n = false;
+  const int n = row_ok ? visible_len(vis_len, rq, t, &bad_n) : 0;
+  if (tid == 0) {
+    ptx::mbar_init(&S.full, 1);
+    ptx::fence_mbar_init();
+  }
+  ptx::griddep_wait();   // the scores come from the previous kernel
   int32_t* out = idx + (size_t)t * K;
-  if (!rq.ok || t < rq.q0 || t - rq.q0 >= rq.Q) {
+  if (!row_ok) {
     if (c == 0) {
       for (int i = tid; i < K; i += nt) out[i] = -1;
       if (tid == 0) {
@@ -809,8 +864,6 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
     }
     return;
   }
-  bool bad_n = false;
-  const int n = visible_len(vis_len, rq, t, &bad_n);
   if (bad_n && c == 0 && tid == 0) raise_fault(status, SML_FAULT_LENGTHS);
   if (n <= K) {
     if (c == 0) {
@@ -824,37 +877,25 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
   const int c0 = min(n, c * per), cn = min(n, c0 + per) - c0;
   const float* row = scores + (size_t)t * max_ctx;
 
-  // 1. this chunk's keys into shared memory; the row's sample straight from
-  //    global memory (every CTA takes the same sample, so all agree on it),
-  //    its loads issued together with the chunk's.
+  // 1. this chunk's raw scores into shared memory (keys[] holds float bits
+  //    until the candidate pass turns them into keys): one bulk asynchronous
+  //    copy of its 16-B aligned part where the row allows it, plain loads
+  //    otherwise; the row's sample straight from global memory (every CTA
+  //    takes the same sample, so all agree on it) while the copy flies.
+  const bool bulk = (reinterpret_cast<uintptr_t>(row + c0) & 15) == 0;
+  const int n_bulk = bulk ? (cn & ~3) : 0;
+  if (tid == 0) {
+    ptx::mbar_arrive_expect_tx(&S.full, (uint32_t)n_bulk * 4u);
+    for (int o = 0; o < n_bulk; o += kBulkPiece)
+      ptx::bulk_load(keys + o, row + c0 + o, (uint32_t)min(kBulkPiece, n_bulk - o) * 4u, &S.full);
+  }
+  for (int i = n_bulk + tid; i < cn; i += nt) keys[i] = __float_as_uint(__ldcg(row + c0 + i));
   const int ns = min(kSample, n);
   float sraw[kSample / kTopkThreads];
 #pragma unroll
   for (int u = 0; u < kSample / kTopkThreads; ++u) {
     const int j = tid + u * nt;
     sraw[u] = j < ns ? __ldcg(row + (int)((long long)j * n / ns)) : NAN;
-  }
-  if ((reinterpret_cast<uintptr_t>(row + c0) & 15) == 0) {
-    // 16-B loads, all of a thread's issued before any is used
-    const float4* src = reinterpret_cast<const float4*>(row + c0);
-    const int n4 = cn >> 2;
-    constexpr int kV = kTopkChunk / 4 / kTopkThreads;   // float4s per thread
-    float4 v[kV];
-#pragma unroll
-    for (int u = 0; u < kV; ++u) {
-      const int i = tid + u * nt;
-      v[u] = i < n4 ? __ldcg(src + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < kV; ++u) {
-      const int i = tid + u * nt;
-      if (i < n4)
-        reinterpret_cast<uint4*>(keys)[i] = make_uint4(order_key(v[u].x), order_key(v[u].y), order_key(v[u].z), order_key(v[u].w));
-    }
-    for (int i = 4 * n4 + tid; i < cn; i += nt) keys[i] = order_key(__ldcg(row + c0 + i));
-  } else {
-#pragma unroll 8
-    for (int i = tid; i < cn; i += nt) keys[i] = order_key(__ldcg(row + c0 + i));
   }
   float sv[kSample / kTopkThreads];
   float lo = INFINITY, hi = -INFINITY;
@@ -880,6 +921,7 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
     S.red_hi[warp] = hi;
   }
   for (int b = tid; b < 256; b += nt) S.samp_hist[b] = 0;
+  for (int b = tid; b < kLinBuckets; b += nt) S.hist[b] = 0;
   if (tid == 0) S.bcast_f = -INFINITY;
   __syncthreads();
   lo = INFINITY;
@@ -931,92 +973,111 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
     __syncthreads();
     floor_v = S.bcast_f;
   }
-  // Fine buckets: 0 = NaN / -inf, 1 .. kBuckets-2 linear in value from the
+  // Fine buckets: 0 = NaN / -inf, 1 .. kLinBuckets-2 linear in value from the
   // floor (or the sample's minimum) to the sample's maximum, clamped at both
-  // ends, kBuckets-1 = +inf: monotone in the key.
+  // ends, kLinBuckets-1 = +inf: monotone in the key.
   bool full = !(floor_v > -INFINITY);
   float base_v = full ? lo : floor_v;
-  float scale = finite_range && hi > base_v ? (float)(kBuckets - 3) / (hi - base_v) : 0.f;
+  float scale = finite_range && hi > base_v ? (float)(kLinBuckets - 3) / (hi - base_v) : 0.f;
   auto bucket = [&](uint32_t key) -> int {
     const float v = key_value(key);
-    if (v == INFINITY) return kBuckets - 1;
+    if (v == INFINITY) return kLinBuckets - 1;
     if (!(v > -INFINITY)) return 0;
-    return 1 + (int)fminf(fmaxf((v - base_v) * scale, 0.f), (float)(kBuckets - 3));
+    return 1 + (int)fminf(fmaxf((v - base_v) * scale, 0.f), (float)(kLinBuckets - 3));
   };
-  // 3. one pass over the chunk: candidates (key >= the floor's key; every key
-  //    when there is no floor) into per-warp lists in position order, and the
-  //    histogram of their buckets.
-  const int seg = ((cn + kWarps - 1) / kWarps + 31) & ~31;
+  // 3. one pass over the chunk, each warp over its own segment (a multiple of
+  //    128 positions, 4 per lane), 4 values per lane at a time: the candidates
+  //    (key >= the floor's key; every key when there is no floor) are
+  //    compacted in place, keys to the front of the warp's segment of keys[]
+  //    (a candidate's slot never lies after its own position, and every lane
+  //    has read its values before the ballots let any lane write) and their
+  //    chunk positions to cpos, both in position order; then the histogram of
+  //    the candidates' buckets.  Afterwards candidate j of a warp is key
+  //    keys[wb + j] at chunk position cpos[warp][j].
+  if (n_bulk > 0 && !ptx::mbar_wait(&S.full, 0, nullptr, kBulkWaitUs)) {
+    // The copy outlived its limit: flag the row and give the copy one more
+    // bounded wait, so that no copy is left writing when the CTA goes on.
+    if (tid == 0) raise_fault(status, SML_FAULT_TIMEOUT);
+    ptx::mbar_wait(&S.full, 0, nullptr, kBulkWaitUs);
+  }
+  __syncthreads();   // the plain-loaded tail, and every lane past the copy
+  const int seg = ((cn + kWarps - 1) / kWarps + 127) & ~127;
   const int wb = min(cn, warp * seg), we = min(cn, wb + seg);
   const unsigned below = (1u << lane) - 1u;
   int total = 0;
   for (int attempt = 0; attempt < 2; ++attempt) {
-    const uint32_t fkey = full ? 0u : order_key(base_v);
-    for (int b = tid; b < kBuckets; b += nt) S.hist[b] = 0;
-    __syncthreads();
+    // key >= the floor's key is value >= the floor for every non-NaN value
+    // (order_key is monotone and ties -0 with +0); NaN passes only when full
+    const float fv = base_v;
     int cnt = 0;
-    for (int i0 = wb; i0 < we; i0 += 32) {
-      const int i = i0 + lane;
-      const uint32_t key = i < we ? keys[i] : 0u;
-      const bool cand = i < we && key >= fkey;
-      const unsigned m = __ballot_sync(0xffffffffu, cand);
-      if (cand) {
-        S.cpos[warp][cnt + __popc(m & below)] = (uint16_t)i;
-        atomicAdd(&S.hist[bucket(key)], 1);
-      }
-      cnt += __popc(m);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (wb + 4 * lane < we) v = *reinterpret_cast<const float4*>(keys + wb + 4 * lane);
+    for (int i0 = wb; i0 < we; i0 += 128) {
+      const int i = i0 + 4 * lane;
+      // the next window's values before this window's writes, which land at
+      // or before this window's positions and so never in the next window
+      float4 vn = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i + 128 < we) vn = *reinterpret_cast<const float4*>(keys + i + 128);
+      const bool cx = i < we && (full || v.x >= fv), cy = i + 1 < we && (full || v.y >= fv);
+      const bool cz = i + 2 < we && (full || v.z >= fv), cw = i + 3 < we && (full || v.w >= fv);
+      // the lanes' candidate counts (0..4) bit by bit: ranks without a scan
+      const int nc = (int)cx + (int)cy + (int)cz + (int)cw;
+      const unsigned b0 = __ballot_sync(0xffffffffu, nc & 1), b1 = __ballot_sync(0xffffffffu, nc & 2),
+                     b2 = __ballot_sync(0xffffffffu, nc & 4);
+      const int px = cnt + __popc(b0 & below) + 2 * __popc(b1 & below) + 4 * __popc(b2 & below);
+      const int py = px + (int)cx, pz = py + (int)cy, pw = pz + (int)cz;
+      cnt += __popc(b0) + 2 * __popc(b1) + 4 * __popc(b2);
+      if (cx) { keys[wb + px] = order_key(v.x); S.cpos[warp][px] = (uint16_t)i; }
+      if (cy) { keys[wb + py] = order_key(v.y); S.cpos[warp][py] = (uint16_t)(i + 1); }
+      if (cz) { keys[wb + pz] = order_key(v.z); S.cpos[warp][pz] = (uint16_t)(i + 2); }
+      if (cw) { keys[wb + pw] = order_key(v.w); S.cpos[warp][pw] = (uint16_t)(i + 3); }
+      v = vn;
     }
+    __syncwarp();
+    for (int j = lane; j < cnt; j += 32) atomicAdd(&S.hist[bucket(keys[wb + j])], 1);
     if (lane == 0) S.wcnt[warp] = cnt;
-    cluster_hist_sum(S, kBuckets, C);
-    int part = 0;
-    for (int b = tid; b < kBuckets; b += nt) part += S.gh[b];
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    if (lane == 0) S.warp_a[warp] = part;
+    cluster_hist_sum(S, kLinBuckets, C);
+    // the cluster's total, and (when it reaches K) the threshold bucket
+    if (warp == 0) {
+      const int tot = bin_scan_warp<kLinBuckets>(K, S.gh, S);
+      if (lane == 0) {
+        S.bcast_tot = tot;
+        S.nbk = 0;
+        S.above = 0;
+      }
+    }
     __syncthreads();
-    total = 0;
-    for (int w = 0; w < kWarps; ++w) total += S.warp_a[w];
+    total = S.bcast_tot;
     if (full || total >= K) break;   // the same in every CTA of the cluster
     full = true;                     // the sample misjudged: every key is a candidate
     base_v = lo;
-    scale = finite_range ? (float)(kBuckets - 3) / width : 0.f;
+    scale = finite_range ? (float)(kLinBuckets - 3) / width : 0.f;
     __syncthreads();
     cluster_sync();                  // every CTA has read this histogram before it is rebuilt
+    // the compaction overwrote the chunk: its raw scores again, and a clean histogram
+    for (int i = tid; i < cn; i += nt) keys[i] = __float_as_uint(__ldcg(row + c0 + i));
+    for (int b = tid; b < kLinBuckets; b += nt) S.hist[b] = 0;
+    __syncthreads();
   }
   // 4. the threshold bucket (the same in every CTA), and this CTA's count of
   //    keys above it
-  if (tid == 0) S.nbk = 0;
-  int bk, need;
-  {
-    int bin, above;
-    find_bin(kBuckets, K, S.gh, S, &bin, &above);
-    bk = bin;
-    need = K - above;
-  }
+  const int bk = S.bcast[0], need = K - S.bcast[1];
   const int wn = S.wcnt[warp];
   {
     int part = 0;
-    for (int b = bk + 1 + tid; b < kBuckets; b += nt) part += S.hist[b];
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    if (lane == 0) S.warp_b[warp] = part;
+    for (int b = bk + 1 + tid; b < kLinBuckets; b += nt) part += S.hist[b];
+    part = __reduce_add_sync(0xffffffffu, part);
+    if (lane == 0 && part > 0) atomicAdd(&S.above, part);
   }
   // 5. this CTA's keys in the threshold bucket, published with that count
   for (int j = lane; j < wn; j += 32) {
-    const uint32_t key = keys[S.cpos[warp][j]];
+    const uint32_t key = keys[wb + j];
     if (bucket(key) == bk) {
       const int slot = atomicAdd(&S.nbk, 1);
       if (slot < kCandCap) S.bkeys[slot] = key;
     }
   }
-  __syncthreads();
-  if (tid == 0) {
-    int a = 0;
-    for (int w = 0; w < kWarps; ++w) a += S.warp_b[w];
-    S.above = a;
-  }
-  __syncthreads();
-  cluster_sync();   // also: every CTA is done reading the others' histograms
+  cluster_sync();   // S.nbk, S.above, S.bkeys complete; every CTA is done reading the others' histograms
   // every CTA's bucket-key count and count above, one round of remote loads
   if (warp == 0 && lane < C) {
     S.nbq[lane] = (int)ld_cluster(&S.nbk, lane);
@@ -1068,28 +1129,25 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
     }
     __syncthreads();
     if (warp == 0) {
-      // CTA q selects above_q + (its bucket keys > tau) + its share of the ties
-      int o = 0, eq_before = 0, off = 0;
+      // The CTAs before this one select their keys above the bucket, their
+      // bucket keys > tau, and the ties in CTA order until take runs out:
+      // min(E, take) ties in all, E = their keys == tau.
+      int o = 0, ab = 0;
       for (int q = 0; q < c; ++q) {
-        const int m = S.nbq[q];
-        int gt = 0, eq = 0;
-        for (int j = lane; j < m; j += 32) {
-          const uint32_t x = S.gkeys[o + j];
-          gt += x > tau;
-          eq += x == tau;
-        }
-#pragma unroll
-        for (int w = 16; w >= 1; w >>= 1) {
-          gt += __shfl_xor_sync(0xffffffffu, gt, w);
-          eq += __shfl_xor_sync(0xffffffffu, eq, w);
-        }
-        off += S.abq[q] + gt + max(0, min(eq, take - eq_before));
-        eq_before += eq;
-        o += m;
+        o += S.nbq[q];
+        ab += S.abq[q];
       }
+      int gt = 0, eq = 0;
+      for (int j = lane; j < o; j += 32) {
+        const uint32_t x = S.gkeys[j];
+        gt += x > tau;
+        eq += x == tau;
+      }
+      gt = __reduce_add_sync(0xffffffffu, gt);
+      eq = __reduce_add_sync(0xffffffffu, eq);
       if (lane == 0) {
-        S.bcast[0] = off;
-        S.bcast[1] = max(0, take - eq_before);
+        S.bcast[0] = ab + gt + min(eq, take);
+        S.bcast[1] = max(0, take - eq);
       }
     }
   } else {
@@ -1103,7 +1161,7 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
       for (int b = tid; b < nb; b += nt) S.hist[b] = 0;
       __syncthreads();
       for (int j = lane; j < wn; j += 32) {
-        const uint32_t key = keys[S.cpos[warp][j]];
+        const uint32_t key = keys[wb + j];
         if (bucket(key) == bk && (key & pmask) == prefix) atomicAdd(&S.hist[(key >> shift) & (uint32_t)(nb - 1)], 1);
       }
       cluster_hist_sum(S, nb, C);
@@ -1120,7 +1178,7 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
     int cg = 0, ce = 0;
     for (int j0 = 0; j0 < wn; j0 += 32) {
       const int j = j0 + lane;
-      const uint32_t key = j < wn ? keys[S.cpos[warp][j]] : 0u;
+      const uint32_t key = j < wn ? keys[wb + j] : 0u;
       cg += __popc(__ballot_sync(0xffffffffu, j < wn && key > tau));
       ce += __popc(__ballot_sync(0xffffffffu, j < wn && key == tau));
     }
@@ -1160,7 +1218,7 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
   int cgt = 0, ceq = 0;
   for (int j0 = 0; j0 < wn; j0 += 32) {
     const int j = j0 + lane;
-    const uint32_t key = j < wn ? keys[S.cpos[warp][j]] : 0u;
+    const uint32_t key = j < wn ? keys[wb + j] : 0u;
     cgt += __popc(__ballot_sync(0xffffffffu, j < wn && key > tau));
     ceq += __popc(__ballot_sync(0xffffffffu, j < wn && key == tau));
   }
@@ -1192,7 +1250,7 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
   for (int j0 = 0; j0 < wn; j0 += 32) {
     const int j = j0 + lane;
     const int pos = j < wn ? S.cpos[warp][j] : 0;
-    const uint32_t key = j < wn ? keys[pos] : 0u;
+    const uint32_t key = j < wn ? keys[wb + j] : 0u;
     const bool gt = j < wn && key > tau, eq = j < wn && key == tau;
     const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
     const int gb = g + __popc(bg & below), eb = e + __popc(be & below);
