@@ -107,15 +107,49 @@ def test_cache_format_checks_without_cuda(L):
     assert "index_cache.format" in sml.sml_last_error()
 
 
-def test_cache_descriptors_of_both_latent_forms():
+def test_cache_descriptors_of_every_latent_form():
     ds = torch.zeros(3 * sml.LATENT_PAGE_BYTES, dtype=torch.uint8)
     c = sml.latent_cache(ds)
     assert (c.num_pages, c.format) == (3, sml.SML_LATENT_FP8_DS_MLA)
     plain = torch.zeros(5 * sml.LATENT_E4M3_PAGE_BYTES, dtype=torch.uint8)
     c = sml.latent_cache(sml.E4M3Latent(plain, 0.25))
     assert (c.num_pages, c.format, c.scale) == (5, sml.SML_LATENT_E4M3, 0.25)
+    bf = torch.zeros(2 * sml.LATENT_BF16_PAGE_BYTES, dtype=torch.uint8)
+    c = sml.latent_cache(sml.Bf16Latent(bf))
+    assert (c.num_pages, c.format) == (2, sml.SML_LATENT_BF16)
     c = sml.cache(None, sml.INDEX_PAGE_BYTES)
     assert (c.base, c.num_pages, c.format) == (None, 0, 0)
+
+
+def _header_defines():
+    """The integer #defines of include/sml.h, each evaluated from the ones before it."""
+    import os
+    import re
+    path = os.path.join(os.path.dirname(__file__), "..", "include", "sml.h")
+    vals = {}
+    for line in open(path, encoding="utf-8"):
+        m = re.match(r"#define\s+(SML_\w+)\s+(.+?)\s*(/\*.*)?$", line.strip())
+        if not m or m.group(1) == "SML_H_":
+            continue
+        expr = m.group(2)
+        if not re.fullmatch(r"[\sA-Z0-9_x()*+\-]+", expr):
+            continue
+        vals[m.group(1)] = eval(expr, {"__builtins__": {}}, dict(vals))
+    return vals
+
+
+def test_binding_constants_match_the_header():
+    h = _header_defines()
+    for name in ("SML_OK", "SML_ERR_INVALID_ARG", "SML_ERR_UNSUPPORTED", "SML_ERR_WORKSPACE", "SML_ERR_CUDA",
+                 "SML_ERR_DEVICE_FAULT", "SML_ERR_TIMEOUT", "SML_FAULT_PAGE", "SML_FAULT_INDEX",
+                 "SML_FAULT_LENGTHS", "SML_FAULT_TOPK_LEN", "SML_FAULT_TIMEOUT", "SML_STAGE_INDEXER",
+                 "SML_STAGE_TOPK", "SML_STAGE_MLA", "SML_STAGE_LAYER", "SML_LATENT_FP8_DS_MLA",
+                 "SML_LATENT_E4M3", "SML_LATENT_BF16", "SML_DCP_MAX_RANKS"):
+        assert getattr(sml, name) == h[name], name
+    assert sml.LATENT_PAGE_BYTES == h["SML_LATENT_PAGE_BYTES"] == 64 * 656
+    assert sml.LATENT_E4M3_PAGE_BYTES == h["SML_LATENT_E4M3_PAGE_BYTES"] == 64 * 576
+    assert sml.LATENT_BF16_PAGE_BYTES == h["SML_LATENT_BF16_PAGE_BYTES"] == 64 * 1152
+    assert sml.INDEX_PAGE_BYTES == h["SML_INDEX_PAGE_BYTES"] == 64 * 132
 
 
 def test_dcp_entry_points_reject_bad_arguments_without_cuda(L):
