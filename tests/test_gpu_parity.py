@@ -146,6 +146,24 @@ def test_topk_ties_signed_zero_nan_inf():
     _topk_case(rows, 1)
 
 
+def test_topk_cluster_heavy_ties():
+    """Rows of one cluster (at most 8 chunks) whose threshold bucket holds more
+    than 4,096 keys, so the cluster runs its radix select over that bucket:
+    exact zeros below fewer than K positive scores (the floor falls to the
+    zeros' bin, every key is a candidate), an all-zero row, and signed zeros
+    with a few larger keys; each with K = 2048 and K = 7."""
+    rng = np.random.default_rng(4)
+    zeros_below = np.zeros(31_000, dtype=np.float32)
+    zeros_below[rng.choice(31_000, 1000, replace=False)] = rng.random(1000).astype(np.float32) + 0.5
+    all_zero = np.zeros(60_000, dtype=np.float32)
+    signed = np.where(rng.random(45_000) < 0.5, 0.0, -0.0).astype(np.float32)
+    signed[rng.choice(45_000, 3, replace=False)] = 2.0
+    signed[rng.choice(45_000, 5000, replace=False)] = -1.0
+    rows = [zeros_below, all_zero, signed]
+    _topk_case(rows, 2048)
+    _topk_case(rows, 7)
+
+
 def test_topk_two_level_rows_with_ties_across_chunks():
     rng = np.random.default_rng(2)
     big = rng.standard_normal(100_000).astype(np.float32)
