@@ -164,6 +164,24 @@ def test_topk_cluster_heavy_ties():
     _topk_case(rows, 7)
 
 
+def test_topk_cluster_misjudged_floor_and_unaligned_rows():
+    """Rows of one cluster: a row whose large keys sit only at the strided
+    sample's positions, so fewer than K keys pass the sampled floor and every
+    CTA reselects over its chunk reloaded from global memory; and a row
+    stride (max_ctx = 30,001) that leaves rows 1..3 off a 16-B boundary, so
+    their chunks arrive by plain loads instead of the bulk copy."""
+    rng = np.random.default_rng(5)
+    n = 20_000
+    misjudged = np.zeros(n, dtype=np.float32)
+    pos = (np.arange(1024, dtype=np.int64) * n) // 1024          # the kernel's strided sample
+    misjudged[pos] = 10.0 + np.arange(1024, dtype=np.float32) * 1e-3
+    rows = [rng.standard_normal(30_001).astype(np.float32), misjudged,
+            rng.standard_normal(29_999).astype(np.float32),
+            np.round(rng.standard_normal(25_003) * 3).astype(np.float32)]
+    _topk_case(rows, 2048)
+    _topk_case(rows, 7)
+
+
 def test_topk_two_level_rows_with_ties_across_chunks():
     rng = np.random.default_rng(2)
     big = rng.standard_normal(100_000).astype(np.float32)
