@@ -225,7 +225,11 @@ int sml_topk(const sml_problem* p, const float* scores, int32_t* idx, int32_t* i
  * carries 12 significant bits, with M_h a per-head integer exponent that keeps
  * every weight at most 440 and the dominant ones at or above 4 (in E4M3's
  * normal range).  A SML_LATENT_BF16 pool runs bf16 x bf16 products instead,
- * with the bf16 query as given and each weight split into two bf16 terms. */
+ * with the bf16 query as given and each weight split into two bf16 terms.
+ * Ordering: the kernel starts early behind the previous kernel of `stream`
+ * and reads the problem's cu_q, ctx_len, vis_len and ssmax_len before it
+ * waits for that kernel (idx, idx_len, q and the cache after), so those four
+ * arrays must not be written by the call of this library just before it. */
 int sml_sparse_mla_decode(const sml_problem* p, const void* q, sml_cache latent,
                           const int32_t* idx, const int32_t* idx_len, float* out, float* lse,
                           void* workspace, size_t ws_bytes, void* stream);

@@ -309,7 +309,8 @@ __device__ __forceinline__ Seg segment_at(const Params& P, long long u, long lon
   s.n = s.req_ok ? visible_len(P.vis_len, rq, s.t, &bad_n) : 0;
   s.req_ok = s.req_ok && !bad_n;
   s.nss = ssmax_len_of(P.ssmax_len, s.t, s.n);
-  // Everything above reads inputs no kernel of this library writes; the
+  // Everything above reads the problem's request arrays, which no call of this
+  // library produces for a sparse-MLA call (the interface requires it); the
   // selection comes from the previous kernel (a no-op after the first call).
   ptx::griddep_wait();
   const int len = s.req_ok ? __ldg(P.idx_len + s.t) : 0;

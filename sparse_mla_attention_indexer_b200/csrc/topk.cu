@@ -838,21 +838,22 @@ topk_cluster_kernel(int B, int T, int K, int max_ctx, int max_pages, const int32
   const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
   const int C = (int)cluster_size(), c = (int)cluster_rank();
   const int t = blockIdx.y;
-  if (tid == 0) ptx::griddep_launch_dependents();
-  // The request lookup reads inputs that no kernel of this library writes, so
-  // it runs before the wait; every global write and every read of the scores
-  // follows it.  Everything up to the first cluster barrier depends only on
-  // the row, so an early return is taken by the whole cluster or by none of it.
+  if (tid == 0) {
+    ptx::griddep_launch_dependents();
+    ptx::mbar_init(&S.full, 1);
+    ptx::fence_mbar_init();
+  }
+  // The scores come from the previous kernel, and so may the lengths (the
+  // candidate merge of context parallelism writes the merged rows' lengths,
+  // which its global selection passes as ctx_len): every global read follows
+  // the wait.  Everything up to the first cluster barrier depends only on the
+  // row, so an early return is taken by the whole cluster or by none of it.
+  ptx::griddep_wait();
   const int r = request_of_warp(cu_q, B, t);
   const Req rq = load_request(cu_q, ctx_len, r, T, max_ctx, max_pages, vis_len != nullptr);
   const bool row_ok = rq.ok && t >= rq.q0 && t - rq.q0 < rq.Q;
   bool bad_n = false;
   const int n = row_ok ? visible_len(vis_len, rq, t, &bad_n) : 0;
-  if (tid == 0) {
-    ptx::mbar_init(&S.full, 1);
-    ptx::fence_mbar_init();
-  }
-  ptx::griddep_wait();   // the scores come from the previous kernel
   int32_t* out = idx + (size_t)t * K;
   if (!row_ok) {
     if (c == 0) {
