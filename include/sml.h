@@ -227,9 +227,9 @@ int sml_topk(const sml_problem* p, const float* scores, int32_t* idx, int32_t* i
  * normal range).  A SML_LATENT_BF16 pool runs bf16 x bf16 products instead,
  * with the bf16 query as given and each weight split into two bf16 terms.
  * Ordering: the kernel starts early behind the previous kernel of `stream`
- * and reads the problem's cu_q, ctx_len, vis_len and ssmax_len before it
- * waits for that kernel (idx, idx_len, q and the cache after), so those four
- * arrays must not be written by the call of this library just before it. */
+ * and reads the problem's cu_q, ctx_len, vis_len and ssmax_len, and q, before
+ * it waits for that kernel (idx, idx_len and the cache after), so those must
+ * not be written by the call of this library just before it. */
 int sml_sparse_mla_decode(const sml_problem* p, const void* q, sml_cache latent,
                           const int32_t* idx, const int32_t* idx_len, float* out, float* lse,
                           void* workspace, size_t ws_bytes, void* stream);
