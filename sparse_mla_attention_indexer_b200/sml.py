@@ -4,6 +4,30 @@ Argument marshalling only: every entry point takes torch tensors (device
 memory) or plain ints, passes their addresses and sizes to the C ABI and raises
 ``SmlError`` on a non-zero status.  Every step of the computation runs in the
 library's CUDA kernels; if ``libsml.so`` is missing the first call raises.
+
+One decode layer, every tensor on the GPU in the layout ``include/sml.h``
+gives (cu_q [B + 1], ctx_len [B] and block_table [B, max_pages] int32; q
+[T, H, 576] bf16; iq [T, 64, 128] bf16; iw [T, 64] fp32; the two page pools
+uint8)::
+
+    from sparse_mla_attention_indexer_b200 import sml
+    p = sml.make_problem(num_heads=16, topk=2048, rope_dim=64, cu_q=cu_q, ctx_len=ctx_len,
+                         block_table=block_table, max_ctx=max_ctx, num_tokens=T,
+                         sm_scale=576 ** -0.5)
+    ws = torch.empty(sml.sml_workspace_size(p, sml.SML_STAGE_LAYER), dtype=torch.uint8,
+                     device="cuda")
+    sml.sml_workspace_init(ws)                                   # once per workspace
+    sml.sml_indexer_k_cache_write(k_new, slot, index_pool, ws)   # the new tokens ...
+    sml.sml_latent_cache_write(c_new, k_pe_new, slot, latent_pool, ws)   # ... into the caches
+    sml.sml_indexer_q_quant(iq, iq8, iq_scale)
+    sml.sml_run_layer(p, q, iq8, iq_scale, iw, latent_pool, index_pool, None, None,
+                      idx, idx_len, out, lse, ws)                # indexer, top-k, sparse MLA
+    code, bits = sml.sml_read_device_status(ws)                  # synchronises the stream
+
+``max_ctx`` and ``num_tokens`` given explicitly keep ``make_problem`` from
+reading the device arrays.  A shared-indexer layer passes the owner layer's
+idx / idx_len as reuse_idx / reuse_len; the stages run one by one through
+``sml_indexer_scores``, ``sml_topk`` and ``sml_sparse_mla_decode``.
 """
 from __future__ import annotations
 
