@@ -50,7 +50,7 @@ FLUSH_BYTES = 256 << 20
 # for the current kernel).
 INDEXER_NCU_TRAFFIC_BYTES = 162_049_024
 # The same for one sparse-MLA launch (the merge not included); None once the
-# kernel has changed since the counters were taken.
+# kernel's loads or stores have changed since the counters were taken.
 MLA_NCU_TRAFFIC_BYTES = 51_031_552
 
 
